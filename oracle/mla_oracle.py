@@ -1,0 +1,305 @@
+"""fp64 CPU oracle for one decode step of Multi-head Latent Attention (MLA).
+
+TEST INFRASTRUCTURE.  Only the test suite, the smoke check and the CPU
+baseline leg of the benchmark use this module.  It shares no code, tables or
+helpers with the CUDA path and imports nothing from it.
+
+What it follows (page addresses as printed, with their section names):
+
+* deepforge.srivtx.xyz "DeepSeek-V2" page, §1 "Theory from first principles",
+  subsection "Store a latent, rebuild the keys and values" and the box
+  "MLA: compress once, reconstruct in attention": each token stores one
+  latent ``c_t = W_DKV h_t`` (512-dim) plus one 64-dim key that carries RoPE;
+  keys and values are rebuilt per head by the up-projections ``k = W_UK c``
+  and ``v = W_UV c``; because those maps are linear, ``W_UK`` can be folded
+  into the query and ``W_UV`` into the output projection ("absorption").
+* Same page, subsection "The bottleneck at inference time": to produce token
+  t, the query of t is compared against the keys of all earlier tokens and
+  their values are mixed -- plain softmax attention over the cache.
+* crackai.dev "DeepSeek-V2" page, "How It Works": up-projections differ per
+  head; a small decoupled RoPE key set carries position separately.
+
+The primary path, :func:`attention_nonabsorbed`, does NOT use absorption: it
+rebuilds per-head keys ``k_{i,t} = [W_UK,i c_t ; RoPE(k_rope_t)]`` and values
+``v_{i,t} = W_UV,i c_t`` explicitly and runs textbook softmax attention.
+:func:`attention_absorbed` is the independent absorbed formulation used only
+to pin the absorption identity.
+
+Readings of points the pages leave open (each is listed in the design doc):
+
+* R1  the 64-dim RoPE key is one vector per token, shared by all heads
+      (576 = 512 + 64 numbers per token only adds up that way).
+* R2  the current query tokens are appended to the cache before attention;
+      query j of S_q sits at position L - S_q + j and sees positions <= its own.
+* R3  queries come from a dense ``W_Q``: per head ``[q_nope (d_n) ; q_rope (d_r)]``.
+* R4  RoPE rotates consecutive pairs (x_2k, x_2k+1) by angle pos * theta_k with
+      theta_k = base^(-2k/d_r).
+* R6  ``W_UK[i]`` has shape [d_n, d_c] and ``W_UV[i]`` has shape [d_v, d_c]
+      (k = W_UK c, v = W_UV c).
+* R7  d_v = d_n.
+* R8  the RoPE key is ``W_KR h_t`` followed by RoPE at the token's position.
+"""
+
+from __future__ import annotations
+
+import numpy as np
+
+F64 = np.float64
+
+
+# ---------------------------------------------------------------------------
+# Cache-size arithmetic (deepforge page, §1 "The bottleneck at inference time"
+# and the cache-size listing after "What the design buys"; crackai page,
+# "Key Takeaways for Interviews": MHA caches 2*n_heads*d_head, GQA caches
+# 2*n_groups*d_head, MLA caches d_latent plus the small RoPE part).
+# ---------------------------------------------------------------------------
+
+def cache_elems_per_token(kind: str, *, n_heads: int = 0, d_head: int = 0,
+                          n_groups: int = 0, d_latent: int = 0,
+                          d_rope: int = 0) -> int:
+    """Numbers cached per token per layer for MHA, GQA or MLA."""
+    if kind == "mha":
+        return 2 * n_heads * d_head
+    if kind == "gqa":
+        return 2 * n_groups * d_head
+    if kind == "mla":
+        return d_latent + d_rope
+    raise ValueError(kind)
+
+
+def dense_cache_bytes(n_heads: int, d_head: int, layers: int, ctx: int,
+                      bytes_per: int = 2) -> int:
+    """Bytes of a full key+value cache: one key and one value per head."""
+    return cache_elems_per_token("mha", n_heads=n_heads, d_head=d_head) \
+        * layers * ctx * bytes_per
+
+
+def mla_cache_bytes(d_latent: int, d_rope: int, layers: int, ctx: int,
+                    bytes_per: int = 2) -> int:
+    """Bytes of the MLA cache: one latent and one RoPE key per token."""
+    return cache_elems_per_token("mla", d_latent=d_latent, d_rope=d_rope) \
+        * layers * ctx * bytes_per
+
+
+def gqa_equivalent_groups(d_latent: int, d_rope: int, d_head: int) -> float:
+    """Number of GQA groups whose cache equals the MLA cache per token."""
+    return (d_latent + d_rope) / (2.0 * d_head)
+
+
+# ---------------------------------------------------------------------------
+# Elementary steps
+# ---------------------------------------------------------------------------
+
+def rope(x, pos, base: float = 10000.0):
+    """Rotary position embedding over consecutive pairs (reading R4).
+
+    ``x`` has shape [..., d] with d even; ``pos`` broadcasts against
+    ``x.shape[:-1]``.  Pair k, i.e. (x[2k], x[2k+1]), is rotated by the angle
+    ``pos * base**(-2k/d)``.  All arithmetic in fp64.
+    """
+    x = np.asarray(x, dtype=F64)
+    d = x.shape[-1]
+    if d % 2:
+        raise ValueError("RoPE width must be even")
+    if d == 0:
+        return x.copy()
+    k = np.arange(d // 2, dtype=F64)
+    theta = np.power(F64(base), -2.0 * k / d)
+    ang = np.asarray(pos, dtype=F64)[..., None] * theta
+    cos, sin = np.cos(ang), np.sin(ang)
+    x0 = x[..., 0::2]
+    x1 = x[..., 1::2]
+    y = np.empty(np.broadcast_shapes(x.shape, ang.shape[:-1] + (d,)), dtype=F64)
+    y[..., 0::2] = x0 * cos - x1 * sin
+    y[..., 1::2] = x0 * sin + x1 * cos
+    return y
+
+
+def project(x, w):
+    """Dense projection y = W x for every row of x (x: [..., in], w: [out, in])."""
+    return np.asarray(x, dtype=F64) @ np.asarray(w, dtype=F64).T
+
+
+def _softmax_attend(scores, values):
+    """Textbook softmax with max subtraction; returns (p, out, lse)."""
+    m = scores.max()
+    e = np.exp(scores - m)
+    z = e.sum()
+    p = e / z
+    return p, p @ values, m + np.log(z)
+
+
+# ---------------------------------------------------------------------------
+# Attention over one sequence's cache
+# ---------------------------------------------------------------------------
+
+def attention_nonabsorbed(q, C, KR, W_UK, W_UV, scale):
+    """Non-absorbed MLA attention for the S_q query tokens of ONE sequence.
+
+    q    [S_q, H, d_n + d_r]  per-head query, RoPE already applied to the
+                              last d_r entries
+    C    [L, d_c]             cached latents c_t, t = 0..L-1
+    KR   [L, d_r]             cached RoPE keys (already rotated)
+    W_UK [H, d_n, d_c], W_UV [H, d_v, d_c]
+
+    For head i the keys are rebuilt as k_{i,t} = [W_UK[i] c_t ; KR_t] and the
+    values as v_{i,t} = W_UV[i] c_t.  Query j (position L - S_q + j) attends to
+    t <= L - S_q + j.  Returns dict with
+      o     [S_q, H, d_v]  attention output per head,
+      o_lat [S_q, H, d_c]  sum_t p_t c_t (latent-space output),
+      lse   [S_q, H]       natural-log partition of the scaled scores,
+      p     list of [S_q][H] probability rows.
+    """
+    q = np.asarray(q, dtype=F64)
+    C = np.asarray(C, dtype=F64)
+    KR = np.asarray(KR, dtype=F64)
+    S_q, H, _ = q.shape
+    L = C.shape[0]
+    d_v = W_UV.shape[1]
+    d_c = C.shape[1]
+    if L < S_q:
+        raise ValueError("context shorter than the query block")
+    o = np.zeros((S_q, H, d_v))
+    o_lat = np.zeros((S_q, H, d_c))
+    lse = np.zeros((S_q, H))
+    probs = [[None] * H for _ in range(S_q)]
+    for i in range(H):
+        K_i = np.concatenate([C @ np.asarray(W_UK[i], dtype=F64).T, KR], axis=1)
+        V_i = C @ np.asarray(W_UV[i], dtype=F64).T
+        for j in range(S_q):
+            vis = L - S_q + j + 1
+            s = scale * (K_i[:vis] @ q[j, i])
+            p, o[j, i], lse[j, i] = _softmax_attend(s, V_i[:vis])
+            o_lat[j, i] = p @ C[:vis]
+            probs[j][i] = p
+    return {"o": o, "o_lat": o_lat, "lse": lse, "p": probs}
+
+
+def attention_absorbed(q, C, KR, W_UK, W_UV, scale):
+    """Absorbed formulation of the same attention (identity check only).
+
+    W_UK folds into the query: q_lat_i = W_UK[i]^T q_nope_i, so the score is
+    q_lat_i . c_t + q_rope_i . KR_t; W_UV folds into the output:
+    o_i = W_UV[i] (sum_t p_t c_t).
+    """
+    q = np.asarray(q, dtype=F64)
+    C = np.asarray(C, dtype=F64)
+    KR = np.asarray(KR, dtype=F64)
+    S_q, H, _ = q.shape
+    d_n = W_UK.shape[1]
+    L = C.shape[0]
+    o = np.zeros((S_q, H, W_UV.shape[1]))
+    o_lat = np.zeros((S_q, H, C.shape[1]))
+    lse = np.zeros((S_q, H))
+    q_lat = np.zeros((S_q, H, C.shape[1]))
+    for i in range(H):
+        Wk = np.asarray(W_UK[i], dtype=F64)
+        Wv = np.asarray(W_UV[i], dtype=F64)
+        for j in range(S_q):
+            vis = L - S_q + j + 1
+            q_lat[j, i] = Wk.T @ q[j, i, :d_n]
+            s = scale * (C[:vis] @ q_lat[j, i] + KR[:vis] @ q[j, i, d_n:])
+            p, o_lat[j, i], lse[j, i] = _softmax_attend(s, C[:vis])
+            o[j, i] = Wv @ o_lat[j, i]
+    return {"o": o, "o_lat": o_lat, "lse": lse, "q_lat": q_lat}
+
+
+# ---------------------------------------------------------------------------
+# One whole decode step of a batch
+# ---------------------------------------------------------------------------
+
+def decode_step(h_new, c_prior, krpre_prior, W_Q, W_DKV, W_KR, W_UK, W_UV,
+                W_O, scale, rope_base, n_heads, seqs=None):
+    """One MLA decode step for a batch, non-absorbed, fp64.
+
+    h_new        [B, S_q, d_model]   hidden states of the new tokens
+    c_prior      list of [L_b - S_q, d_c] latents already cached
+    krpre_prior  list of [L_b - S_q, d_r] RoPE keys of those tokens BEFORE
+                 rotation (rotated here by their positions 0..)
+    W_Q [H*(d_n+d_r), d_model], W_DKV [d_c, d_model], W_KR [d_r, d_model],
+    W_UK [H, d_n, d_c], W_UV [H, d_v, d_c], W_O [d_model, H*d_v]
+    seqs         optional subset of sequence indices to evaluate
+
+    Steps per sequence b (positions per reading R2):
+      1. new tokens: c = W_DKV h, kr = RoPE(W_KR h, pos), pos = L-S_q .. L-1
+      2. q = W_Q h split per head into [q_nope ; q_rope]; q_rope <- RoPE(q_rope, pos)
+      3. non-absorbed attention over the cache (see attention_nonabsorbed)
+      4. out = W_O [o_1; ...; o_H]
+    Returns dict of per-sequence results keyed by stage name.
+    """
+    h_new = np.asarray(h_new, dtype=F64)
+    B, S_q, _ = h_new.shape
+    H = n_heads
+    d_c = W_DKV.shape[0]
+    d_r = W_KR.shape[0]
+    d_qk = W_Q.shape[0] // H
+    seqs = range(B) if seqs is None else seqs
+    res = {k: {} for k in ("q", "q_roped", "c_new", "kr_new", "o", "o_lat",
+                           "lse", "out")}
+    for b in seqs:
+        Lp = np.asarray(c_prior[b]).shape[0]
+        L = Lp + S_q
+        pos = np.arange(Lp, L)
+        c_new = project(h_new[b], W_DKV)                   # [S_q, d_c]
+        kr_new = rope(project(h_new[b], W_KR), pos, rope_base)
+        C = np.concatenate([np.asarray(c_prior[b], dtype=F64).reshape(Lp, d_c),
+                            c_new], axis=0)
+        KR = np.concatenate([rope(np.asarray(krpre_prior[b], dtype=F64)
+                                  .reshape(Lp, d_r), np.arange(Lp), rope_base),
+                             kr_new], axis=0)
+        q = project(h_new[b], W_Q).reshape(S_q, H, d_qk)
+        q_roped = q.copy()
+        q_roped[..., d_qk - d_r:] = rope(q[..., d_qk - d_r:], pos[:, None],
+                                         rope_base)
+        att = attention_nonabsorbed(q_roped, C, KR, W_UK, W_UV, scale)
+        out = project(att["o"].reshape(S_q, -1), W_O)
+        res["q"][b] = q
+        res["q_roped"][b] = q_roped
+        res["c_new"][b] = c_new
+        res["kr_new"][b] = kr_new
+        res["o"][b] = att["o"]
+        res["o_lat"][b] = att["o_lat"]
+        res["lse"][b] = att["lse"]
+        res["out"][b] = out
+    return res
+
+
+# ---------------------------------------------------------------------------
+# Paged cache append (deepforge page, §1 box: only c_t and the small RoPE key
+# are ever written to memory).  Layout: pool[page, slot, 0:d_c] = c,
+# pool[page, slot, d_c:d_c+d_r] = rotated RoPE key; token at position p of
+# sequence b lives in page page_table[b][p // page_size], slot p % page_size.
+# ---------------------------------------------------------------------------
+
+def cache_append(pool, c, kr, batch_idx, pos, page_table, page_size):
+    """Return a copy of ``pool`` with each new token's row written, one by one.
+
+    Works on any dtype (raw bf16 bit patterns as uint16 included); copies the
+    values unchanged.
+    """
+    out = np.array(pool, copy=True)
+    d_c = c.shape[1]
+    for t in range(c.shape[0]):
+        b = int(batch_idx[t])
+        p = int(pos[t])
+        page = int(page_table[b][p // page_size])
+        slot = p % page_size
+        out[page, slot, :d_c] = c[t]
+        out[page, slot, d_c:] = kr[t]
+    return out
+
+
+def combine_splits(o_parts, lse_parts):
+    """Merge per-split attention results by log-sum-exp weighting.
+
+    o_parts [S, ...D] (each split's normalised output), lse_parts [S, ...];
+    returns (o, lse) of attention over the union of the splits' tokens.
+    Splits whose lse is -inf (no tokens) carry zero weight.
+    """
+    o_parts = np.asarray(o_parts, dtype=F64)
+    lse_parts = np.asarray(lse_parts, dtype=F64)
+    m = lse_parts.max(axis=0)
+    w = np.exp(lse_parts - m)
+    z = w.sum(axis=0)
+    o = (w[..., None] * o_parts).sum(axis=0) / z[..., None]
+    return o, m + np.log(z)
