@@ -1,0 +1,192 @@
+/*
+ * mla.h -- C ABI of the B200 (sm_100a) MLA decode library (libmla_b200.so).
+ *
+ * One decode step of DeepSeek-V2's Multi-head Latent Attention, run on the
+ * compressed cache with the absorption trick.  Sources for what each call
+ * computes (page address and section as printed):
+ *
+ *   [DF-1]  deepforge.srivtx.xyz "DeepSeek-V2", §1 "Store a latent, rebuild
+ *           the keys and values" and the box "MLA: compress once,
+ *           reconstruct in attention": c_t = W_DKV h_t (512-dim) plus one
+ *           64-dim RoPE key are the only things cached per token per layer;
+ *           k = W_UK c, v = W_UV c; being linear, W_UK folds into the query
+ *           and W_UV into the output projection ("absorption").
+ *   [DF-0]  same page, §1 "The bottleneck at inference time": token t's
+ *           query is compared against the keys of all earlier tokens and
+ *           their values are mixed (softmax attention over the cache).
+ *   [CA-1]  crackai.dev "DeepSeek-V2", "How It Works": up-projections differ
+ *           per head; the decoupled RoPE keys carry position separately.
+ *
+ * Conventions shared by every call
+ *   - All pointers named "device" are CUDA device pointers owned by the
+ *     caller; the library never frees or retains them.  Pointers named
+ *     "host" are host memory.
+ *   - Element counts and strides are in ELEMENTS of the buffer's type.
+ *   - dtype MLA_F32: every floating buffer is float32 and all arithmetic is
+ *     fp32 (SIMT kernels).  dtype MLA_BF16: activations, weights, the query
+ *     buffer and the cache are bf16 (raw 16-bit), accumulation is fp32;
+ *     buffers documented as "fp32" stay fp32 in both modes.
+ *   - stream is a cudaStream_t (NULL = legacy default stream).  Every call
+ *     except mla_get_device_status only enqueues work; none synchronises.
+ *   - Host-detectable argument errors return MLA_ERR_INVALID_ARG or
+ *     MLA_ERR_UNSUPPORTED before anything is enqueued.  A launch failure
+ *     returns MLA_ERR_CUDA.  Errors found on the device (a page id outside
+ *     the pool, a bounded wait that ran out) set a per-device status word
+ *     that mla_get_device_status reads and clears; the offending access is
+ *     skipped, never performed.
+ *   - The library allocates no device memory except the 4-byte status word
+ *     per device; scratch space is passed in by the caller.
+ *   - Calls are stateless apart from a host-side cache of TMA descriptors;
+ *     calls on different streams may run concurrently.
+ */
+#ifndef MLA_B200_H
+#define MLA_B200_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  MLA_OK = 0,
+  MLA_ERR_INVALID_ARG = 1,   /* null pointer, bad size or stride */
+  MLA_ERR_UNSUPPORTED = 2,   /* shape the selected kernels do not cover */
+  MLA_ERR_CUDA = 3,          /* a CUDA runtime call failed */
+  MLA_ERR_TIMEOUT = 4,       /* device: a bounded wait ran out */
+  MLA_ERR_BOUNDS = 5         /* device: an index left its buffer */
+} mla_status;
+
+typedef enum { MLA_F32 = 0, MLA_BF16 = 1 } mla_dtype;
+
+/* Model dimensions of one MLA layer.  d_v is the value head width (= d_nope
+ * for DeepSeek-V2); page_size is the number of tokens per cache page. */
+typedef struct {
+  int n_heads;      /* H */
+  int d_nope;       /* per-head query/key width without RoPE (128) */
+  int d_latent;     /* d_c, latent width (512) */
+  int d_rope;       /* d_r, decoupled RoPE key width (64), even */
+  int d_v;          /* per-head value width (128) */
+  int d_model;      /* hidden size (5120) */
+  int page_size;    /* tokens per page (64) */
+  float scale;      /* softmax scale, 1/sqrt(d_nope + d_rope) */
+  float rope_base;  /* RoPE base (10000) */
+  mla_dtype dtype;
+} mla_dims;
+
+/* A0 -- dense projection of hidden states ([DF-1]: c_t = W_DKV h_t; the
+ * query and RoPE-key projections are the same operation).
+ *   y[r, o] = sum_i x[r, i] * w[o, i]      r < rows, o < out_f, i < in_f
+ * x: device [rows, in_f], w: device [out_f, in_f], y: device [rows, out_f],
+ * all row-major and contiguous, dtype of dims.  fp32 accumulation; bf16 y is
+ * rounded to nearest even.  rows >= 0 (0 is a no-op); in_f, out_f >= 1.
+ * bf16 needs in_f % 8 == 0 and 16-byte aligned x and w. */
+mla_status mla_project(const mla_dims* dims, const void* x, const void* w,
+                       void* y, int rows, int in_f, int out_f, void* stream);
+
+/* A1 -- fold W_UK into the query ([DF-1] absorption):
+ *   qbuf[t, i, c] = sum_n q[t, i, n] * w_uk[i, n, c],  n < d_nope, c < d_latent
+ * q: device, token t head i starts at q + t*q_stride_tok + i*(d_nope+d_rope)
+ *    (the first d_nope entries are read);
+ * w_uk: device [H, d_nope, d_latent] contiguous;
+ * qbuf: device [T, H, d_latent + d_rope] contiguous; only columns
+ *    [0, d_latent) are written (mla_rope fills the rest).
+ * bf16 needs q_stride_tok % 8 == 0, d_nope % 16 == 0, d_latent % 128 == 0. */
+mla_status mla_absorb_q(const mla_dims* dims, const void* q, int q_stride_tok,
+                        const void* w_uk, void* qbuf, int T, void* stream);
+
+/* A2 -- rotary position embedding of RoPE parts ([DF-1] decoupled RoPE key,
+ * [CA-1]).  For t < T, h < n_heads_x, k < d_rope/2 the pair
+ *   (x0, x1) = (x[t*xs_tok + h*xs_head + 2k], ... + 2k + 1)
+ * is rotated by the angle pos[t] * rope_base^(-2k/d_rope):
+ *   y[.. 2k] = x0*cos - x1*sin,   y[.. 2k+1] = x0*sin + x1*cos.
+ * The angle is formed and reduced in fp64, the rotation is done in fp32.
+ * x, y: device, dtype of dims, may alias exactly (in place).  pos: device
+ * int32 [T], each >= 0. */
+mla_status mla_rope(const mla_dims* dims, const void* x, int xs_tok,
+                    int xs_head, int n_heads_x, void* y, int ys_tok,
+                    int ys_head, const int32_t* pos, int T, void* stream);
+
+/* A3 -- append new tokens to the paged latent cache ([DF-1]: only c_t and
+ * the RoPE key are written to memory).  For each t < T:
+ *   page = page_table[batch_idx[t]*max_pages + pos[t]/page_size]
+ *   pool[page][pos[t] % page_size][0 : d_latent]          = c[t*cs_tok ...]
+ *   pool[page][pos[t] % page_size][d_latent : d_latent+d_rope] = kr[t*ks_tok ...]
+ * An exact copy of the element bits.  pool: device
+ * [n_pages, page_size, d_latent + d_rope]; page_table: device int32
+ * [B, max_pages]; batch_idx, pos: device int32 [T].  A page id outside
+ * [0, n_pages) or pos/page_size >= max_pages skips that token and raises
+ * MLA_ERR_BOUNDS in the device status. */
+mla_status mla_cache_append(const mla_dims* dims, const void* c, int cs_tok,
+                            const void* kr, int ks_tok,
+                            const int32_t* batch_idx, const int32_t* pos,
+                            const int32_t* page_table, int max_pages,
+                            void* pool, int n_pages, int T, void* stream);
+
+/* Workspace bytes mla_decode needs for B sequences of S_q query tokens and
+ * num_workers split workers (0 = the default mla_decode would pick). */
+size_t mla_decode_workspace_size(const mla_dims* dims, int B, int S_q,
+                                 int num_workers);
+
+/* A4 + A5 -- attention of every query against the latent cache, with the
+ * absorbed query ([DF-0], [DF-1]).  For sequence b with L = seq_lens[b]
+ * cached tokens (the S_q query tokens included, at positions L-S_q..L-1),
+ * query j and head i:
+ *   s_t  = scale * qbuf[b, j, i, :] . pool_row(b, t)   over all d_latent+d_rope
+ *   p    = softmax over t <= L - S_q + j
+ *   o_lat[b, j, i, :] = sum_t p_t * pool_row(b, t)[0 : d_latent]
+ *   lse[b, j, i]      = ln sum_t exp(s_t)
+ * pool_row(b, t) = pool[page_table[b*max_pages + t/page_size]][t % page_size].
+ * The token range of every sequence is split over num_workers workers
+ * (0 = one per pair of SMs) with equal token counts per worker; a
+ * log-sum-exp combine merges the pieces.
+ * qbuf: device [B, S_q, H, d_latent + d_rope]; seq_lens: device int32 [B]
+ * with S_q <= seq_lens[b] <= max_pages*page_size; o_lat: device fp32
+ * [B, S_q, H, d_latent]; lse: device fp32 [B, S_q, H]; workspace: device,
+ * >= mla_decode_workspace_size bytes, 256-byte aligned, contents ignored.
+ * bf16 requires d_latent == 512, d_rope == 64, page_size == 64, and
+ * S_q*H % 128 == 0; 1 <= S_q <= 2 in both modes. */
+mla_status mla_decode(const mla_dims* dims, const void* qbuf, const void* pool,
+                      int n_pages, const int32_t* page_table, int max_pages,
+                      const int32_t* seq_lens, int B, int S_q, int num_workers,
+                      void* workspace, size_t ws_bytes, float* o_lat,
+                      float* lse, void* stream);
+
+/* Scratch bytes mla_out_proj needs for T tokens. */
+size_t mla_out_proj_scratch_size(const mla_dims* dims, int T);
+
+/* A6 -- apply W_UV per head, then the output projection ([DF-1]: W_UV folds
+ * into the output side):
+ *   o[t, i, v]   = sum_c w_uv[i, v, c] * o_lat[t, i, c]
+ *   out[t, m]    = sum_{i,v} w_o[m, i*d_v + v] * o[t, i, v]
+ * o_lat: device fp32 [T, H, d_latent] (rounded to bf16 for the bf16 path);
+ * w_uv: device [H, d_v, d_latent]; w_o: device [d_model, H*d_v];
+ * scratch: device, >= mla_out_proj_scratch_size bytes, 256-byte aligned;
+ * out: device fp32 [T, d_model]. */
+mla_status mla_out_proj(const mla_dims* dims, const float* o_lat,
+                        const void* w_uv, const void* w_o, void* scratch,
+                        size_t scratch_bytes, float* out, int T, void* stream);
+
+/* Synchronises `stream`, then returns and clears the device status word of
+ * the current device (MLA_OK, MLA_ERR_TIMEOUT or MLA_ERR_BOUNDS; TIMEOUT
+ * wins if both were raised), or MLA_ERR_CUDA if the stream failed. */
+mla_status mla_get_device_status(void* stream);
+
+/* Static, human-readable text for a status code. */
+const char* mla_status_string(mla_status s);
+
+/* Self-test of the failure path: enqueues one kernel whose only wait is on
+ * an mbarrier that nothing completes, bounded to wait_ns nanoseconds; the
+ * kernel then raises MLA_ERR_TIMEOUT in the device status and returns.  No
+ * fault, trap or hang is involved. */
+mla_status mla_selftest_wait_timeout(unsigned long long wait_ns, void* stream);
+
+/* Number of kernel launches the library has enqueued since load (for
+ * benchmark bookkeeping; incremented on the host). */
+uint64_t mla_launch_count(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* MLA_B200_H */

@@ -1,0 +1,449 @@
+// api.cu -- the extern "C" entry points of libmla_b200.so (see include/mla.h).
+//
+// Host-side validation, TMA descriptor encoding, split planning and kernel
+// launches.  All device work is in the kernels included below; nothing here
+// computes on the host.
+#include <atomic>
+#include <cmath>
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+
+#include "../../include/mla.h"
+#include "common.cuh"
+#include "decode_tc.cuh"
+#include "gemm_tc.cuh"
+#include "simt.cuh"
+
+using namespace mla;
+
+namespace {
+
+std::atomic<uint64_t> g_launches{0};
+
+inline cudaStream_t as_stream(void* s) { return reinterpret_cast<cudaStream_t>(s); }
+
+inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+mla_status check_launch() {
+  g_launches.fetch_add(1, std::memory_order_relaxed);
+  return cudaGetLastError() == cudaSuccess ? MLA_OK : MLA_ERR_CUDA;
+}
+
+#define MLA_TRY(expr)                   \
+  do {                                  \
+    mla_status _s = (expr);             \
+    if (_s != MLA_OK) return _s;        \
+  } while (0)
+
+bool dims_ok(const mla_dims* d) {
+  return d != nullptr && d->n_heads > 0 && d->d_nope > 0 && d->d_latent > 0 && d->d_rope >= 0 &&
+         (d->d_rope % 2) == 0 && d->d_v > 0 && d->d_model > 0 && d->page_size > 0 &&
+         (d->dtype == MLA_F32 || d->dtype == MLA_BF16) && std::isfinite(d->scale);
+}
+
+int sm_count() {
+  int dev = 0, n = 0;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+  return n > 0 ? n : 148;
+}
+
+// ---------------------------------------------------------------------------
+// TMA descriptors (driver entry point fetched through the runtime)
+// ---------------------------------------------------------------------------
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  });
+  return fn;
+}
+
+// bf16 tensor of rank `rank` (<= 3), dims innermost first, byte strides of
+// dims 1.., 128-byte swizzle, zero fill out of bounds.
+bool make_tmap_bf16(CUtensorMap* m, const void* ptr, int rank, const uint64_t* dims,
+                    const uint64_t* strides_bytes, const uint32_t* box) {
+  EncodeTiledFn fn = encode_fn();
+  if (fn == nullptr) return false;
+  cuuint64_t d[5], s[4];
+  cuuint32_t bx[5], es[5];
+  for (int i = 0; i < rank; ++i) {
+    d[i] = dims[i];
+    bx[i] = box[i];
+    es[i] = 1;
+  }
+  for (int i = 0; i + 1 < rank; ++i) s[i] = strides_bytes[i];
+  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, rank, const_cast<void*>(ptr), d, s, bx, es,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+// ---------------------------------------------------------------------------
+// GEMM launchers
+// ---------------------------------------------------------------------------
+template <typename TI, typename TO>
+mla_status launch_simt_gemm(const SimtGemmArgs& g, cudaStream_t st) {
+  if (g.M <= 0 || g.N <= 0 || g.batch <= 0) return MLA_OK;
+  dim3 grid((g.M + 63) / 64, (g.N + 63) / 64, g.batch);
+  simt_gemm_kernel<TI, TO><<<grid, 256, 0, st>>>(g);
+  return check_launch();
+}
+
+struct TcGemmPlan {
+  int n_tile, n_tiles, stages, splits, k_chunks_per_split;
+  size_t smem;
+};
+
+TcGemmPlan plan_tc_gemm(int M, int N, int K, int batch, bool allow_split) {
+  TcGemmPlan p;
+  int n16 = ((N + 15) / 16) * 16;
+  p.n_tile = n16 < 256 ? n16 : 256;
+  p.n_tiles = (N + p.n_tile - 1) / p.n_tile;
+  const size_t stage_bytes = (size_t)kGemmBM * kGemmBK * 2 + (size_t)p.n_tile * kGemmBK * 2;
+  int st = (int)((96 * 1024) / stage_bytes);
+  p.stages = st < 2 ? 2 : (st > 8 ? 8 : st);
+  const int k_chunks = (K + kGemmBK - 1) / kGemmBK;
+  p.splits = 1;
+  if (allow_split) {
+    const long long ctas = (long long)((M + kGemmBM - 1) / kGemmBM) * p.n_tiles * batch;
+    const long long target = 2LL * sm_count();
+    while (ctas * p.splits < target && k_chunks / (p.splits + 1) >= 4) ++p.splits;
+  }
+  p.k_chunks_per_split = (k_chunks + p.splits - 1) / p.splits;
+  p.smem = stage_bytes * p.stages + 1024;
+  return p;
+}
+
+// A: [batch][M][K] K-major (a_mn = false) or [batch][K][M] (a_mn = true);
+// X: [batch][N][K] with row stride xs_n and batch stride xs_b (elements).
+// out element (b, n, m) at ob*b + on*n + om*m.
+mla_status launch_tc_gemm(const void* A, bool a_mn, long long as_b, const void* X, long long xs_n,
+                          long long xs_b, int M, int N, int K, int batch, void* out, long long ob,
+                          long long on, long long om, int out_kind, cudaStream_t st) {
+  if (M <= 0 || N <= 0 || batch <= 0) return MLA_OK;
+  if (!aligned16(A) || !aligned16(X) || (K % 8) != 0 || (xs_n % 8) != 0 || (xs_b % 8) != 0 ||
+      (as_b % 8) != 0)
+    return MLA_ERR_INVALID_ARG;
+  if (a_mn && (M % 8) != 0) return MLA_ERR_INVALID_ARG;
+  TcGemmPlan p = plan_tc_gemm(M, N, K, batch, out_kind == kOutF32Atomic);
+  CUtensorMap tA, tX;
+  {
+    uint64_t dims[3], strides[2];
+    uint32_t box[3];
+    if (a_mn) {
+      dims[0] = M; dims[1] = K; dims[2] = batch;
+      strides[0] = (uint64_t)M * 2; strides[1] = (uint64_t)as_b * 2;
+      box[0] = 64; box[1] = kGemmBK; box[2] = 1;
+    } else {
+      dims[0] = K; dims[1] = M; dims[2] = batch;
+      strides[0] = (uint64_t)K * 2; strides[1] = (uint64_t)as_b * 2;
+      box[0] = kGemmBK; box[1] = kGemmBM; box[2] = 1;
+    }
+    if (batch == 1) strides[1] = strides[0] * dims[1];
+    if (!make_tmap_bf16(&tA, A, 3, dims, strides, box)) return MLA_ERR_CUDA;
+  }
+  {
+    uint64_t dims[3] = {(uint64_t)K, (uint64_t)N, (uint64_t)batch};
+    uint64_t strides[2] = {(uint64_t)xs_n * 2, (uint64_t)xs_b * 2};
+    if (batch == 1) strides[1] = strides[0] * dims[1];
+    uint32_t box[3] = {(uint32_t)kGemmBK, (uint32_t)p.n_tile, 1};
+    if (!make_tmap_bf16(&tX, X, 3, dims, strides, box)) return MLA_ERR_CUDA;
+  }
+  GemmTcArgs g;
+  g.M = M; g.N = N; g.K = K;
+  g.n_tile = p.n_tile; g.n_tiles = p.n_tiles;
+  g.k_chunks_per_split = p.k_chunks_per_split;
+  g.stages = p.stages;
+  g.out = out; g.ob = ob; g.on = on; g.om = om;
+  dim3 grid((M + kGemmBM - 1) / kGemmBM, p.n_tiles * p.splits, batch);
+#define MLA_GEMM_LAUNCH(AMN, OUT)                                                              \
+  do {                                                                                         \
+    auto kfn = gemm_tc_kernel<AMN, OUT>;                                                       \
+    if (cudaFuncSetAttribute(kfn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)p.smem) != \
+        cudaSuccess)                                                                           \
+      return MLA_ERR_CUDA;                                                                     \
+    kfn<<<grid, 128, p.smem, st>>>(tA, tX, g);                                                 \
+  } while (0)
+  if (a_mn) {
+    if (out_kind == kOutBf16) MLA_GEMM_LAUNCH(true, kOutBf16);
+    else if (out_kind == kOutF32) MLA_GEMM_LAUNCH(true, kOutF32);
+    else MLA_GEMM_LAUNCH(true, kOutF32Atomic);
+  } else {
+    if (out_kind == kOutBf16) MLA_GEMM_LAUNCH(false, kOutBf16);
+    else if (out_kind == kOutF32) MLA_GEMM_LAUNCH(false, kOutF32);
+    else MLA_GEMM_LAUNCH(false, kOutF32Atomic);
+  }
+#undef MLA_GEMM_LAUNCH
+  return check_launch();
+}
+
+// ---------------------------------------------------------------------------
+// decode planning
+// ---------------------------------------------------------------------------
+constexpr int kBlockTokens = 128;
+
+bool use_tc_decode(const mla_dims* d, int S_q) {
+  return kDecodeTcReady && d->dtype == MLA_BF16 && d->d_latent == 512 && d->d_rope == 64 && d->page_size == 64 &&
+         ((S_q * d->n_heads) % 128) == 0;
+}
+
+struct DecodeLayout {
+  int R, rows_per_v, V, G;
+  size_t off_start, off_lse, off_o, total;
+};
+
+DecodeLayout decode_layout(const mla_dims* d, int B, int S_q, int num_workers) {
+  DecodeLayout L;
+  const bool tc = use_tc_decode(d, S_q);
+  L.R = tc ? (S_q * d->n_heads) / 128 : 1;
+  L.rows_per_v = (S_q * d->n_heads) / L.R;
+  L.V = B * L.R;
+  const int sms = sm_count();
+  L.G = num_workers > 0 ? num_workers : (tc ? sms / 2 : 2 * sms);
+  const size_t n_slots = (size_t)L.G + L.V;
+  auto up = [](size_t x) { return (x + 255) & ~(size_t)255; };
+  L.off_start = 0;
+  L.off_lse = up(sizeof(int32_t) * (L.V + 1));
+  L.off_o = L.off_lse + up(sizeof(float) * n_slots * L.rows_per_v);
+  L.total = L.off_o + up(sizeof(float) * n_slots * L.rows_per_v * d->d_latent);
+  return L;
+}
+
+}  // namespace
+
+// ===========================================================================
+// C ABI
+// ===========================================================================
+extern "C" {
+
+const char* mla_status_string(mla_status s) {
+  switch (s) {
+    case MLA_OK: return "ok";
+    case MLA_ERR_INVALID_ARG: return "invalid argument";
+    case MLA_ERR_UNSUPPORTED: return "unsupported shape for the selected kernels";
+    case MLA_ERR_CUDA: return "CUDA runtime error";
+    case MLA_ERR_TIMEOUT: return "device wait timed out";
+    case MLA_ERR_BOUNDS: return "device index out of bounds";
+  }
+  return "unknown status";
+}
+
+uint64_t mla_launch_count(void) { return g_launches.load(); }
+
+mla_status mla_get_device_status(void* stream) {
+  if (cudaStreamSynchronize(as_stream(stream)) != cudaSuccess) return MLA_ERR_CUDA;
+  unsigned v = 0, zero = 0;
+  if (cudaMemcpyFromSymbol(&v, g_status, sizeof(v)) != cudaSuccess) return MLA_ERR_CUDA;
+  if (v != 0 && cudaMemcpyToSymbol(g_status, &zero, sizeof(zero)) != cudaSuccess)
+    return MLA_ERR_CUDA;
+  if (v & kFlagTimeout) return MLA_ERR_TIMEOUT;
+  if (v & kFlagBounds) return MLA_ERR_BOUNDS;
+  return MLA_OK;
+}
+
+mla_status mla_selftest_wait_timeout(unsigned long long wait_ns, void* stream) {
+  wait_selftest_kernel<<<1, 32, 0, as_stream(stream)>>>(wait_ns);
+  return check_launch();
+}
+
+mla_status mla_project(const mla_dims* dims, const void* x, const void* w, void* y, int rows,
+                       int in_f, int out_f, void* stream) {
+  if (!dims_ok(dims) || rows < 0 || in_f < 1 || out_f < 1) return MLA_ERR_INVALID_ARG;
+  if (rows == 0) return MLA_OK;
+  if (!x || !w || !y) return MLA_ERR_INVALID_ARG;
+  cudaStream_t st = as_stream(stream);
+  if (dims->dtype == MLA_F32) {
+    SimtGemmArgs g{w, x, y, out_f, rows, in_f, 1, 0, in_f, 1, 0, in_f, 1, 0, out_f, 1, 0};
+    return launch_simt_gemm<float, float>(g, st);
+  }
+  return launch_tc_gemm(w, false, 0, x, in_f, 0, out_f, rows, in_f, 1, y, 0, out_f, 1, kOutBf16,
+                        st);
+}
+
+mla_status mla_absorb_q(const mla_dims* dims, const void* q, int q_stride_tok, const void* w_uk,
+                        void* qbuf, int T, void* stream) {
+  if (!dims_ok(dims) || T < 0) return MLA_ERR_INVALID_ARG;
+  if (T == 0) return MLA_OK;
+  if (!q || !w_uk || !qbuf) return MLA_ERR_INVALID_ARG;
+  const int H = dims->n_heads, dn = dims->d_nope, dc = dims->d_latent, dr = dims->d_rope;
+  const int dqk = dn + dr, D = dc + dr;
+  if (q_stride_tok < H * dqk) return MLA_ERR_INVALID_ARG;
+  cudaStream_t st = as_stream(stream);
+  if (dims->dtype == MLA_F32) {
+    SimtGemmArgs g{w_uk, q, qbuf, dc, T, dn, H,
+                   (long long)dn * dc, 1, dc,
+                   dqk, q_stride_tok, 1,
+                   D, (long long)H * D, 1, 0};
+    return launch_simt_gemm<float, float>(g, st);
+  }
+  if ((dn % 16) != 0 || (dc % 128) != 0 || (q_stride_tok % 8) != 0 || (dqk % 8) != 0)
+    return MLA_ERR_UNSUPPORTED;
+  // A = W_UK[i] read as [K = d_nope][M = d_latent] (MN-major); X = q_nope of head i.
+  return launch_tc_gemm(w_uk, true, (long long)dn * dc, q, q_stride_tok, dqk, dc, T, dn, H, qbuf,
+                        D, (long long)H * D, 1, kOutBf16, st);
+}
+
+mla_status mla_rope(const mla_dims* dims, const void* x, int xs_tok, int xs_head, int n_heads_x,
+                    void* y, int ys_tok, int ys_head, const int32_t* pos, int T, void* stream) {
+  if (!dims_ok(dims) || T < 0 || n_heads_x < 0) return MLA_ERR_INVALID_ARG;
+  if (T == 0 || n_heads_x == 0 || dims->d_rope == 0) return MLA_OK;
+  if (!x || !y || !pos) return MLA_ERR_INVALID_ARG;
+  const long long n = (long long)T * n_heads_x * (dims->d_rope / 2);
+  const int blk = 256;
+  const long long grid = (n + blk - 1) / blk;
+  cudaStream_t st = as_stream(stream);
+  if (dims->dtype == MLA_F32)
+    rope_kernel<float><<<(unsigned)grid, blk, 0, st>>>(
+        static_cast<const float*>(x), xs_tok, xs_head, n_heads_x, static_cast<float*>(y), ys_tok,
+        ys_head, pos, T, dims->d_rope, (double)dims->rope_base);
+  else
+    rope_kernel<__nv_bfloat16><<<(unsigned)grid, blk, 0, st>>>(
+        static_cast<const __nv_bfloat16*>(x), xs_tok, xs_head, n_heads_x,
+        static_cast<__nv_bfloat16*>(y), ys_tok, ys_head, pos, T, dims->d_rope,
+        (double)dims->rope_base);
+  return check_launch();
+}
+
+mla_status mla_cache_append(const mla_dims* dims, const void* c, int cs_tok, const void* kr,
+                            int ks_tok, const int32_t* batch_idx, const int32_t* pos,
+                            const int32_t* page_table, int max_pages, void* pool, int n_pages,
+                            int T, void* stream) {
+  if (!dims_ok(dims) || T < 0 || max_pages < 1 || n_pages < 1) return MLA_ERR_INVALID_ARG;
+  if (T == 0) return MLA_OK;
+  if (!c || !batch_idx || !pos || !page_table || !pool || (dims->d_rope > 0 && !kr))
+    return MLA_ERR_INVALID_ARG;
+  cudaStream_t st = as_stream(stream);
+  if (dims->dtype == MLA_F32)
+    append_kernel<uint32_t><<<T, 128, 0, st>>>(
+        static_cast<const uint32_t*>(c), cs_tok, static_cast<const uint32_t*>(kr), ks_tok,
+        batch_idx, pos, page_table, max_pages, static_cast<uint32_t*>(pool), n_pages,
+        dims->page_size, dims->d_latent, dims->d_rope);
+  else
+    append_kernel<uint16_t><<<T, 128, 0, st>>>(
+        static_cast<const uint16_t*>(c), cs_tok, static_cast<const uint16_t*>(kr), ks_tok,
+        batch_idx, pos, page_table, max_pages, static_cast<uint16_t*>(pool), n_pages,
+        dims->page_size, dims->d_latent, dims->d_rope);
+  return check_launch();
+}
+
+size_t mla_decode_workspace_size(const mla_dims* dims, int B, int S_q, int num_workers) {
+  if (!dims_ok(dims) || B < 0 || S_q < 1 || num_workers < 0) return 0;
+  return decode_layout(dims, B, S_q, num_workers).total;
+}
+
+mla_status mla_decode(const mla_dims* dims, const void* qbuf, const void* pool, int n_pages,
+                      const int32_t* page_table, int max_pages, const int32_t* seq_lens, int B,
+                      int S_q, int num_workers, void* workspace, size_t ws_bytes, float* o_lat,
+                      float* lse, void* stream) {
+  if (!dims_ok(dims) || B < 0 || S_q < 1 || S_q > 2 || num_workers < 0 || n_pages < 1 ||
+      max_pages < 1)
+    return MLA_ERR_INVALID_ARG;
+  if (B == 0) return MLA_OK;
+  if (!qbuf || !pool || !page_table || !seq_lens || !workspace || !o_lat || !lse)
+    return MLA_ERR_INVALID_ARG;
+  if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return MLA_ERR_INVALID_ARG;
+  if ((dims->d_latent % 4) != 0 || dims->d_latent > 512) return MLA_ERR_UNSUPPORTED;
+  const DecodeLayout L = decode_layout(dims, B, S_q, num_workers);
+  if (ws_bytes < L.total) return MLA_ERR_INVALID_ARG;
+  cudaStream_t st = as_stream(stream);
+  char* ws = static_cast<char*>(workspace);
+  int32_t* start = reinterpret_cast<int32_t*>(ws + L.off_start);
+  float* ws_lse = reinterpret_cast<float*>(ws + L.off_lse);
+  float* ws_o = reinterpret_cast<float*>(ws + L.off_o);
+  const int max_tokens = max_pages * dims->page_size;
+  plan_kernel<<<1, 1024, 0, st>>>(seq_lens, B, L.R, S_q, max_tokens, kBlockTokens, start);
+  MLA_TRY(check_launch());
+  const int H = dims->n_heads, dc = dims->d_latent, dr = dims->d_rope;
+  if (use_tc_decode(dims, S_q)) {
+    if (!aligned16(qbuf) || !aligned16(pool)) return MLA_ERR_INVALID_ARG;
+    MLA_TRY(launch_decode_tc(qbuf, pool, n_pages, page_table, max_pages, seq_lens, B, S_q, H,
+                             dims->scale, L.G, start, ws_lse, ws_o, st));
+    g_launches.fetch_add(1, std::memory_order_relaxed);
+  } else {
+    dim3 grid(L.G, (L.rows_per_v + 7) / 8);
+    const int kc = (dc + 31) / 32;
+#define MLA_SIMT_DECODE(T, KC)                                                                 \
+  decode_simt_kernel<T, KC><<<grid, 256, 0, st>>>(                                             \
+      static_cast<const T*>(qbuf), static_cast<const T*>(pool), n_pages, page_table, max_pages, \
+      seq_lens, B, S_q, H, dc, dr, dims->page_size, dims->scale, L.G, kBlockTokens, start,      \
+      ws_lse, ws_o)
+    if (dims->dtype == MLA_F32) {
+      if (kc <= 2) MLA_SIMT_DECODE(float, 2);
+      else if (kc <= 4) MLA_SIMT_DECODE(float, 4);
+      else if (kc <= 8) MLA_SIMT_DECODE(float, 8);
+      else MLA_SIMT_DECODE(float, 16);
+    } else {
+      if (kc <= 2) MLA_SIMT_DECODE(__nv_bfloat16, 2);
+      else if (kc <= 4) MLA_SIMT_DECODE(__nv_bfloat16, 4);
+      else if (kc <= 8) MLA_SIMT_DECODE(__nv_bfloat16, 8);
+      else MLA_SIMT_DECODE(__nv_bfloat16, 16);
+    }
+#undef MLA_SIMT_DECODE
+    MLA_TRY(check_launch());
+  }
+  dim3 cgrid(L.V, (L.rows_per_v + 7) / 8);
+  combine_kernel<<<cgrid, 256, 0, st>>>(ws_lse, ws_o, start, L.V, L.R, L.G, L.rows_per_v, dc,
+                                        o_lat, lse);
+  return check_launch();
+}
+
+size_t mla_out_proj_scratch_size(const mla_dims* dims, int T) {
+  if (!dims_ok(dims) || T < 0) return 0;
+  auto up = [](size_t x) { return (x + 255) & ~(size_t)255; };
+  const size_t H = dims->n_heads;
+  if (dims->dtype == MLA_F32) return up((size_t)T * H * dims->d_v * 4);
+  return up((size_t)T * H * dims->d_latent * 2) + up((size_t)T * H * dims->d_v * 2);
+}
+
+mla_status mla_out_proj(const mla_dims* dims, const float* o_lat, const void* w_uv,
+                        const void* w_o, void* scratch, size_t scratch_bytes, float* out, int T,
+                        void* stream) {
+  if (!dims_ok(dims) || T < 0) return MLA_ERR_INVALID_ARG;
+  if (T == 0) return MLA_OK;
+  if (!o_lat || !w_uv || !w_o || !scratch || !out) return MLA_ERR_INVALID_ARG;
+  if (scratch_bytes < mla_out_proj_scratch_size(dims, T)) return MLA_ERR_INVALID_ARG;
+  if ((reinterpret_cast<uintptr_t>(scratch) & 255u) != 0) return MLA_ERR_INVALID_ARG;
+  const int H = dims->n_heads, dc = dims->d_latent, dv = dims->d_v, dm = dims->d_model;
+  cudaStream_t st = as_stream(stream);
+  if (dims->dtype == MLA_F32) {
+    float* o = static_cast<float*>(scratch);
+    SimtGemmArgs g1{w_uv, o_lat, o, dv, T, dc, H,
+                    (long long)dv * dc, dc, 1,
+                    dc, (long long)H * dc, 1,
+                    dv, (long long)H * dv, 1, 0};
+    MLA_TRY((launch_simt_gemm<float, float>(g1, st)));
+    SimtGemmArgs g2{w_o, o, out, dm, T, H * dv, 1, 0, (long long)H * dv, 1, 0, (long long)H * dv,
+                    1, 0, dm, 1, 0};
+    return launch_simt_gemm<float, float>(g2, st);
+  }
+  auto up = [](size_t x) { return (x + 255) & ~(size_t)255; };
+  __nv_bfloat16* olb = static_cast<__nv_bfloat16*>(scratch);
+  __nv_bfloat16* o = reinterpret_cast<__nv_bfloat16*>(static_cast<char*>(scratch) +
+                                                      up((size_t)T * H * dc * 2));
+  const long long n = (long long)T * H * dc;
+  cast_f32_bf16_kernel<<<(unsigned)((n / 4 + 255) / 256 + 1), 256, 0, st>>>(o_lat, olb, n);
+  MLA_TRY(check_launch());
+  // o[t, i, :] = W_UV[i] o_lat[t, i, :]
+  MLA_TRY(launch_tc_gemm(w_uv, false, (long long)dv * dc, olb, (long long)H * dc, dc, dv, T, dc, H,
+                         o, dv, (long long)H * dv, 1, kOutBf16, st));
+  // out[t, :] = W_O o[t, :]
+  if (cudaMemsetAsync(out, 0, sizeof(float) * (size_t)T * dm, st) != cudaSuccess)
+    return MLA_ERR_CUDA;
+  return launch_tc_gemm(w_o, false, 0, o, (long long)H * dv, 0, dm, T, H * dv, 1, out, 0, dm, 1,
+                        kOutF32Atomic, st);
+}
+
+}  // extern "C"

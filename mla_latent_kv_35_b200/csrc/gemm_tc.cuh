@@ -1,0 +1,187 @@
+// gemm_tc.cuh -- weight-streaming bf16 GEMM on the 5th-generation tensor
+// cores (tcgen05, TMEM accumulator, TMA-fed 128-byte-swizzled operands).
+//
+//   out[b][n][m] (+)= sum_k W[b][m][k] * X[b][n][k]
+//
+// The weight matrix is the MMA's A operand (M = output features, 128 per
+// CTA) and the few activation rows are the B operand (N = tokens, padded to
+// a multiple of 16, at most 256 per CTA): at decode the token count is far
+// below 128, so putting the weights on M keeps the MMA at full height.
+// A may be K-major ([M][K], the usual [out, in] weight) or MN-major ([K][M],
+// e.g. W_UK[i] read as its transpose).  X is always K-major.  Split-K over
+// grid.y accumulates fp32 outputs with atomics.
+//
+// Warp roles (128 threads): warp 0 lane 0 issues TMA loads into an
+// S-stage ring; warp 1 allocates TMEM and its lane 0 issues the MMAs; after
+// the last MMA all four warps read the accumulator (TMEM lane = output row)
+// and store it.
+#pragma once
+
+#include "common.cuh"
+
+namespace mla {
+
+enum GemmOut : int { kOutBf16 = 0, kOutF32 = 1, kOutF32Atomic = 2 };
+
+struct GemmTcArgs {
+  int M, N, K;           // per batch entry
+  int n_tile;            // BN, multiple of 16, <= 256
+  int n_tiles;           // ceil(N / BN)
+  int k_chunks_per_split;
+  int stages;
+  void* out;
+  long long ob, on, om;  // output strides in elements
+};
+
+constexpr int kGemmBM = 128;
+constexpr int kGemmBK = 64;  // 64 bf16 = one 128-byte swizzle row
+
+template <bool kAmn, int kOut>
+__global__ void __launch_bounds__(128, 1) gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA,
+                                                         const __grid_constant__ CUtensorMap tmX,
+                                                         GemmTcArgs g) {
+  extern __shared__ uint8_t smem_raw[];
+  __shared__ __align__(8) uint64_t full_bar[8];
+  __shared__ __align__(8) uint64_t empty_bar[8];
+  __shared__ __align__(8) uint64_t acc_bar;
+  __shared__ uint32_t tmem_base_sh;
+  __shared__ int abort_flag;
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int m0 = blockIdx.x * kGemmBM;
+  const int n_tile_idx = blockIdx.y % g.n_tiles;
+  const int split = blockIdx.y / g.n_tiles;
+  const int n0 = n_tile_idx * g.n_tile;
+  const int b = blockIdx.z;
+  const int BN = g.n_tile;
+  const int S = g.stages;
+  const int k_chunks_total = (g.K + kGemmBK - 1) / kGemmBK;
+  const int kc0 = split * g.k_chunks_per_split;
+  const int kc1 = min(k_chunks_total, kc0 + g.k_chunks_per_split);
+  const int nk = max(0, kc1 - kc0);
+
+  const uint32_t a_bytes = kGemmBM * kGemmBK * 2;  // 16 KB
+  const uint32_t x_bytes = BN * kGemmBK * 2;
+  const uint32_t stage_bytes = a_bytes + x_bytes;
+  const uint32_t smem_base = (smem_u32(smem_raw) + 1023u) & ~1023u;
+
+  if (threadIdx.x == 0) {
+    abort_flag = 0;
+    for (int s = 0; s < S; ++s) {
+      mbar_init(smem_u32(&full_bar[s]), 1);
+      mbar_init(smem_u32(&empty_bar[s]), 1);
+    }
+    mbar_init(smem_u32(&acc_bar), 1);
+    fence_mbar_init();
+    tma_prefetch_desc(&tmA);
+    tma_prefetch_desc(&tmX);
+  }
+  uint32_t tmem_cols = 32;
+  while ((int)tmem_cols < BN) tmem_cols <<= 1;
+  if (warp == 1) {
+    tmem_alloc<1>(smem_u32(&tmem_base_sh), tmem_cols);
+    tmem_relinquish<1>();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = tmem_base_sh;
+  volatile int* abort_p = &abort_flag;
+
+  if (warp == 0 && lane == 0 && nk > 0) {
+    // ---------------- TMA producer ----------------
+    int issued = 0;
+    for (int i = 0; i < nk; ++i) {
+      const int s = i % S;
+      if (!mbar_wait(smem_u32(&empty_bar[s]), ((i / S) & 1) ^ 1, abort_p)) break;
+      const uint32_t fb = smem_u32(&full_bar[s]);
+      const uint32_t sa = smem_base + s * stage_bytes;
+      mbar_expect_tx(fb, stage_bytes);
+      const int k = (kc0 + i) * kGemmBK;
+      if constexpr (kAmn) {
+        tma_load_3d(sa, &tmA, m0, k, b, fb);
+        tma_load_3d(sa + a_bytes / 2, &tmA, m0 + 64, k, b, fb);
+      } else {
+        tma_load_3d(sa, &tmA, k, m0, b, fb);
+      }
+      tma_load_3d(sa + a_bytes, &tmX, k, n0, b, fb);
+      ++issued;
+    }
+    if (*abort_p) {
+      // let copies still in flight land before the CTA can exit
+      for (int i = max(0, issued - S); i < issued; ++i)
+        mbar_wait(smem_u32(&full_bar[i % S]), (i / S) & 1, nullptr);
+    }
+  } else if (warp == 1 && lane == 0 && nk > 0) {
+    // ---------------- MMA issuer ----------------
+    const uint32_t idesc = idesc_bf16_f32(kGemmBM, BN, kAmn, false);
+    bool ok = true;
+    for (int i = 0; i < nk; ++i) {
+      const int s = i % S;
+      if (!mbar_wait(smem_u32(&full_bar[s]), (i / S) & 1, abort_p)) { ok = false; break; }
+      tc_fence_after();
+      const uint32_t sa = smem_base + s * stage_bytes;
+      const uint32_t sx = sa + a_bytes;
+#pragma unroll
+      for (int kk = 0; kk < kGemmBK / 16; ++kk) {
+        uint64_t ad;
+        if constexpr (kAmn)
+          ad = sw128_desc(sa + kk * 2048, 8192, 1024);  // 16 K-rows of 128 B per step
+        else
+          ad = sw128_desc(sa + kk * 32, 16, 1024);      // 16 K-elements = 32 B per step
+        const uint64_t xd = sw128_desc(sx + kk * 32, 16, 1024);
+        mma_bf16_ss<1>(tmem, ad, xd, idesc, (i > 0 || kk > 0) ? 1u : 0u);
+      }
+      mma_commit_1(smem_u32(&empty_bar[s]));
+    }
+    if (ok) mma_commit_1(smem_u32(&acc_bar));
+  }
+  __syncwarp();
+
+  // ---------------- epilogue: all 4 warps ----------------
+  bool have = nk > 0 && mbar_wait(smem_u32(&acc_bar), 0, abort_p);
+  if (have) {
+    tc_fence_after();
+    const int m = m0 + warp * 32 + lane;
+    for (int c0 = 0; c0 < BN; c0 += 32) {
+      uint32_t r[32];
+      tmem_ld32(tmem + ((uint32_t)(warp * 32) << 16) + c0, r);
+      tmem_wait_ld();
+      if (m < g.M) {
+#pragma unroll
+        for (int i = 0; i < 32; ++i) {
+          const int n = n0 + c0 + i;
+          if (c0 + i < BN && n < g.N) {
+            const long long o = (long long)b * g.ob + (long long)n * g.on + (long long)m * g.om;
+            const float v = __uint_as_float(r[i]);
+            if constexpr (kOut == kOutBf16)
+              static_cast<__nv_bfloat16*>(g.out)[o] = __float2bfloat16_rn(v);
+            else if constexpr (kOut == kOutF32)
+              static_cast<float*>(g.out)[o] = v;
+            else
+              atomicAdd(static_cast<float*>(g.out) + o, v);
+          }
+        }
+      }
+    }
+  } else if (nk == 0 && kOut != kOutF32Atomic) {
+    // empty K range: the product is zero
+    const int m = m0 + warp * 32 + lane;
+    if (m < g.M)
+      for (int i = 0; i < BN; ++i) {
+        const int n = n0 + i;
+        if (n < g.N) {
+          const long long o = (long long)b * g.ob + (long long)n * g.on + (long long)m * g.om;
+          if constexpr (kOut == kOutBf16)
+            static_cast<__nv_bfloat16*>(g.out)[o] = __float2bfloat16_rn(0.f);
+          else
+            static_cast<float*>(g.out)[o] = 0.f;
+        }
+      }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) tmem_dealloc<1>(tmem, tmem_cols);
+}
+
+}  // namespace mla

@@ -1,0 +1,360 @@
+// simt.cuh -- CUDA-core kernels: the fp32 path of every step, plus the
+// elementwise steps (RoPE, cache append, casts), the split planner and the
+// log-sum-exp combine that the bf16 path shares.
+#pragma once
+
+#include "common.cuh"
+
+namespace mla {
+
+// ---------------------------------------------------------------------------
+// Batched strided GEMM on CUDA cores (fp32 accumulate).
+//   out[b*ob + n*on + m*om] (+)= sum_k A[b*ab + m*am + k*ak] * X[b*xb + n*xn + k*xk]
+// 64x64 output tile per 256-thread block, 4x4 per thread, k-tiles of 16.
+// ---------------------------------------------------------------------------
+struct SimtGemmArgs {
+  const void* A;
+  const void* X;
+  void* out;
+  int M, N, K, batch;
+  long long ab, am, ak, xb, xn, xk, ob, on, om;
+  int atomic_out;  // fp32 output only: accumulate with atomicAdd
+};
+
+template <typename TI, typename TO>
+__global__ void __launch_bounds__(256) simt_gemm_kernel(SimtGemmArgs g) {
+  __shared__ float As[16][65];
+  __shared__ float Xs[16][65];
+  const TI* A = static_cast<const TI*>(g.A);
+  const TI* X = static_cast<const TI*>(g.X);
+  TO* out = static_cast<TO*>(g.out);
+  const int b = blockIdx.z;
+  const int m0 = blockIdx.x * 64, n0 = blockIdx.y * 64;
+  const int tx = threadIdx.x % 16, ty = threadIdx.x / 16;
+  float acc[4][4] = {};
+  for (int k0 = 0; k0 < g.K; k0 += 16) {
+    for (int e = threadIdx.x; e < 16 * 64; e += 256) {
+      int kk = e / 64, mm = e % 64;
+      int k = k0 + kk;
+      int m = m0 + mm, n = n0 + mm;
+      As[kk][mm] = (k < g.K && m < g.M) ? to_f32(A[b * g.ab + m * g.am + k * g.ak]) : 0.f;
+      Xs[kk][mm] = (k < g.K && n < g.N) ? to_f32(X[b * g.xb + n * g.xn + k * g.xk]) : 0.f;
+    }
+    __syncthreads();
+#pragma unroll
+    for (int kk = 0; kk < 16; ++kk) {
+      float a[4], x[4];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) a[i] = As[kk][tx + 16 * i];
+#pragma unroll
+      for (int j = 0; j < 4; ++j) x[j] = Xs[kk][ty + 16 * j];
+#pragma unroll
+      for (int i = 0; i < 4; ++i)
+#pragma unroll
+        for (int j = 0; j < 4; ++j) acc[i][j] = fmaf(a[i], x[j], acc[i][j]);
+    }
+    __syncthreads();
+  }
+#pragma unroll
+  for (int i = 0; i < 4; ++i)
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      int m = m0 + tx + 16 * i, n = n0 + ty + 16 * j;
+      if (m < g.M && n < g.N) {
+        long long o = b * g.ob + n * g.on + m * g.om;
+        if constexpr (sizeof(TO) == 4) {
+          if (g.atomic_out)
+            atomicAdd(reinterpret_cast<float*>(out) + o, acc[i][j]);
+          else
+            out[o] = from_f32<TO>(acc[i][j]);
+        } else {
+          out[o] = from_f32<TO>(acc[i][j]);
+        }
+      }
+    }
+}
+
+// ---------------------------------------------------------------------------
+// RoPE: rotate consecutive pairs by pos * base^(-2k/d); angle in fp64.
+// ---------------------------------------------------------------------------
+template <typename T>
+__global__ void rope_kernel(const T* x, long long xs_tok, long long xs_head, int nh, T* y,
+                            long long ys_tok, long long ys_head, const int32_t* pos, int Tn,
+                            int d_rope, double base) {
+  const int half = d_rope / 2;
+  long long idx = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+  long long total = (long long)Tn * nh * half;
+  if (idx >= total) return;
+  const int k = (int)(idx % half);
+  const int h = (int)((idx / half) % nh);
+  const int t = (int)(idx / ((long long)half * nh));
+  const double theta = pow(base, -2.0 * (double)k / (double)d_rope);
+  const double ang = (double)pos[t] * theta;
+  // reduce to [-pi, pi] in fp64 before taking sine and cosine
+  const double two_pi = 6.283185307179586476925286766559;
+  const double red = ang - two_pi * rint(ang / two_pi);
+  double sn, cs;
+  sincos(red, &sn, &cs);
+  const float c = (float)cs, s = (float)sn;
+  const T* px = x + t * xs_tok + h * xs_head + 2 * k;
+  T* py = y + t * ys_tok + h * ys_head + 2 * k;
+  const float x0 = to_f32(px[0]), x1 = to_f32(px[1]);
+  py[0] = from_f32<T>(x0 * c - x1 * s);
+  py[1] = from_f32<T>(x0 * s + x1 * c);
+}
+
+// ---------------------------------------------------------------------------
+// Cache append: exact copy of each new token's latent and RoPE key into its
+// page slot.  Element size E bytes (2 for bf16, 4 for fp32).
+// ---------------------------------------------------------------------------
+template <typename E>
+__global__ void append_kernel(const E* c, long long cs_tok, const E* kr, long long ks_tok,
+                              const int32_t* batch_idx, const int32_t* pos,
+                              const int32_t* page_table, int max_pages, E* pool, int n_pages,
+                              int page_size, int d_c, int d_r) {
+  const int t = blockIdx.x;
+  const int b = batch_idx[t];
+  const int p = pos[t];
+  const int lp = p / page_size;
+  if (p < 0 || b < 0 || lp >= max_pages) {
+    if (threadIdx.x == 0) raise_flag(kFlagBounds);
+    return;
+  }
+  const int page = page_table[(long long)b * max_pages + lp];
+  if (page < 0 || page >= n_pages) {
+    if (threadIdx.x == 0) raise_flag(kFlagBounds);
+    return;
+  }
+  const int D = d_c + d_r;
+  E* row = pool + ((long long)page * page_size + (p % page_size)) * D;
+  for (int e = threadIdx.x; e < D; e += blockDim.x)
+    row[e] = e < d_c ? c[t * cs_tok + e] : kr[t * ks_tok + (e - d_c)];
+}
+
+__global__ void cast_f32_bf16_kernel(const float* x, __nv_bfloat16* y, long long n) {
+  long long i = ((long long)blockIdx.x * blockDim.x + threadIdx.x) * 4;
+  if (i + 3 < n) {
+    float4 v = *reinterpret_cast<const float4*>(x + i);
+    uint2 o;
+    o.x = pack_bf16x2(v.x, v.y);
+    o.y = pack_bf16x2(v.z, v.w);
+    *reinterpret_cast<uint2*>(y + i) = o;
+  } else {
+    for (; i < n; ++i) y[i] = __float2bfloat16_rn(x[i]);
+  }
+}
+
+// ---------------------------------------------------------------------------
+// Split planning.  Virtual sequence v = b*R + r (R row blocks per sequence)
+// has nb_v = ceil(L_b / BLK) token blocks.  start[v] = sum_{u<v} nb_u and
+// start[V] = total.  Worker k of G owns blocks [lo_k, lo_{k+1}) of the
+// concatenation, lo_k = floor(k * total / G).  The piece of worker k in v
+// writes partial slot k + v (unique: pieces form a monotone staircase).
+// ---------------------------------------------------------------------------
+__global__ void plan_kernel(const int32_t* seq_lens, int B, int R, int S_q, int max_tokens,
+                            int BLK, int32_t* start) {
+  __shared__ int32_t warp_sums[32];
+  __shared__ int32_t carry;
+  if (threadIdx.x == 0) carry = 0;
+  __syncthreads();
+  const int V = B * R;
+  for (int base = 0; base < V; base += blockDim.x) {
+    const int v = base + threadIdx.x;
+    int nb = 0;
+    if (v < V) {
+      const int L = seq_lens[v / R];
+      if (L < S_q || L > max_tokens) {
+        if (v % R == 0) raise_flag(kFlagBounds);
+      } else {
+        nb = (L + BLK - 1) / BLK;
+      }
+    }
+    // inclusive warp scan
+    int x = nb;
+    const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      int y = __shfl_up_sync(0xffffffffu, x, o);
+      if (lane >= o) x += y;
+    }
+    if (lane == 31) warp_sums[w] = x;
+    __syncthreads();
+    if (w == 0) {
+      int s = lane < (int)(blockDim.x >> 5) ? warp_sums[lane] : 0;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        int y = __shfl_up_sync(0xffffffffu, s, o);
+        if (lane >= o) s += y;
+      }
+      warp_sums[lane] = s;  // inclusive prefix over warps
+    }
+    __syncthreads();
+    const int excl = carry + (w > 0 ? warp_sums[w - 1] : 0) + x - nb;
+    if (v < V) start[v] = excl;
+    __syncthreads();
+    if (threadIdx.x == blockDim.x - 1) carry = excl + nb;
+    __syncthreads();
+  }
+  if (threadIdx.x == 0) start[V] = carry;
+}
+
+__device__ __forceinline__ int worker_lo(int k, int total, int G) {
+  return (int)(((long long)k * total) / G);
+}
+// worker owning global block x (0 <= x < total)
+__device__ __forceinline__ int worker_of(int x, int total, int G) {
+  return (int)((((long long)x + 1) * G - 1) / total);
+}
+// first v with start[v+1] > x, i.e. the virtual sequence holding block x
+__device__ __forceinline__ int seq_of_block(const int32_t* start, int V, int x) {
+  int lo = 0, hi = V - 1;
+  while (lo < hi) {
+    int mid = (lo + hi) >> 1;
+    if (start[mid + 1] > x) hi = mid; else lo = mid + 1;
+  }
+  return lo;
+}
+
+// ---------------------------------------------------------------------------
+// SIMT split-KV decode: one warp per query row, 8 rows per block.  Grid
+// (G workers, ceil(rows_per_v / 8)).  Writes normalised partial outputs and
+// natural-log lse per piece into slot k + v.  R = 1 here (v = b).
+// ---------------------------------------------------------------------------
+template <typename T, int kMaxC>
+__global__ void __launch_bounds__(256) decode_simt_kernel(
+    const T* qbuf, const T* pool, int n_pages, const int32_t* page_table, int max_pages,
+    const int32_t* seq_lens, int B, int S_q, int H, int d_c, int d_r, int page_size, float scale,
+    int G, int BLK, const int32_t* start, float* ws_lse, float* ws_o) {
+  const int k = blockIdx.x;
+  const int lane = threadIdx.x & 31;
+  const int rows = S_q * H;
+  const int r = blockIdx.y * 8 + (threadIdx.x >> 5);
+  if (r >= rows) return;
+  const int total = start[B];
+  if (total == 0) return;
+  const int lo = worker_lo(k, total, G), hi = worker_lo(k + 1, total, G);
+  if (lo >= hi) return;
+  const int D = d_c + d_r;
+  const int j = r / H;
+  int v = seq_of_block(start, B, lo);
+  for (; v < B && start[v] < hi; ++v) {
+    const int x0 = max(lo, start[v]) - start[v];
+    const int x1 = min(hi, start[v + 1]) - start[v];
+    if (x1 <= x0) continue;
+    const int L = seq_lens[v];
+    const int limit = L - S_q + j + 1;  // visible tokens t < limit
+    const int t0 = x0 * BLK, t1 = min(min(x1 * BLK, L), limit);
+    const T* q = qbuf + ((long long)v * rows + r) * D;
+    float m = -INFINITY, l = 0.f;
+    float o[kMaxC];
+#pragma unroll
+    for (int u = 0; u < kMaxC; ++u) o[u] = 0.f;
+    for (int t = t0; t < t1; ++t) {
+      const int page = page_table[(long long)v * max_pages + t / page_size];
+      if (page < 0 || page >= n_pages) {
+        if (lane == 0) raise_flag(kFlagBounds);
+        continue;
+      }
+      const T* row = pool + ((long long)page * page_size + t % page_size) * D;
+      float s = 0.f;
+      for (int e = lane; e < D; e += 32) s = fmaf(to_f32(q[e]), to_f32(row[e]), s);
+#pragma unroll
+      for (int off = 16; off > 0; off >>= 1) s += __shfl_xor_sync(0xffffffffu, s, off);
+      s *= scale;
+      const float m_new = fmaxf(m, s);
+      const float alpha = __expf(m - m_new);
+      const float p = __expf(s - m_new);
+      l = l * alpha + p;
+#pragma unroll
+      for (int u = 0; u < kMaxC; ++u) {
+        const int c = lane + 32 * u;
+        if (c < d_c) o[u] = o[u] * alpha + p * to_f32(row[c]);
+      }
+      m = m_new;
+    }
+    const long long slot = (long long)k + v;
+    const float inv = l > 0.f ? 1.f / l : 0.f;
+#pragma unroll
+    for (int u = 0; u < kMaxC; ++u) {
+      const int c = lane + 32 * u;
+      if (c < d_c) ws_o[(slot * rows + r) * d_c + c] = o[u] * inv;
+    }
+    if (lane == 0) ws_lse[slot * rows + r] = l > 0.f ? m + logf(l) : -INFINITY;
+  }
+}
+
+// ---------------------------------------------------------------------------
+// Log-sum-exp combine of the pieces of every virtual sequence.
+//   o = sum_k w_k o_k / sum_k w_k, w_k = exp(lse_k - max lse), lse = max + ln sum w
+// Grid (V, ceil(rows_per_v / 8)), one warp per row.
+// ---------------------------------------------------------------------------
+__global__ void __launch_bounds__(256) combine_kernel(const float* ws_lse, const float* ws_o,
+                                                      const int32_t* start, int V, int R, int G,
+                                                      int rows_per_v, int d_c, float* o_lat,
+                                                      float* lse) {
+  const int v = blockIdx.x;
+  const int r = blockIdx.y * 8 + (threadIdx.x >> 5);
+  const int lane = threadIdx.x & 31;
+  if (r >= rows_per_v) return;
+  const int total = start[V];
+  const long long out_row = (long long)(v / R) * R * rows_per_v + (long long)(v % R) * rows_per_v + r;
+  float* dst = o_lat + out_row * d_c;
+  if (start[v + 1] == start[v]) {
+    for (int c = lane; c < d_c; c += 32) dst[c] = 0.f;
+    if (lane == 0) lse[out_row] = -INFINITY;
+    return;
+  }
+  const int k0 = worker_of(start[v], total, G);
+  const int k1 = worker_of(start[v + 1] - 1, total, G);
+  // workers with an empty range (only when G > total) wrote no slot
+#define MLA_LIVE(k) (worker_lo((k) + 1, total, G) > worker_lo((k), total, G))
+  float mx = -INFINITY;
+  for (int k = k0; k <= k1; ++k)
+    if (MLA_LIVE(k)) mx = fmaxf(mx, ws_lse[((long long)k + v) * rows_per_v + r]);
+  if (mx == -INFINITY) {
+    for (int c = lane; c < d_c; c += 32) dst[c] = 0.f;
+    if (lane == 0) lse[out_row] = -INFINITY;
+    return;
+  }
+  float z = 0.f;
+  for (int k = k0; k <= k1; ++k)
+    if (MLA_LIVE(k)) z += __expf(ws_lse[((long long)k + v) * rows_per_v + r] - mx);
+  const float inv_z = 1.f / z;
+  for (int c4 = lane * 4; c4 < d_c; c4 += 128) {
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int k = k0; k <= k1; ++k) {
+      if (!MLA_LIVE(k)) continue;
+      const long long slot = (long long)k + v;
+      const float w = __expf(ws_lse[slot * rows_per_v + r] - mx) * inv_z;
+      const float4 x = *reinterpret_cast<const float4*>(ws_o + (slot * rows_per_v + r) * d_c + c4);
+      acc.x = fmaf(w, x.x, acc.x);
+      acc.y = fmaf(w, x.y, acc.y);
+      acc.z = fmaf(w, x.z, acc.z);
+      acc.w = fmaf(w, x.w, acc.w);
+    }
+    *reinterpret_cast<float4*>(dst + c4) = acc;
+  }
+  if (lane == 0) lse[out_row] = mx + logf(z);
+#undef MLA_LIVE
+}
+
+// A bounded wait that nothing completes: exercises the timeout path.
+__global__ void wait_selftest_kernel(unsigned long long wait_ns) {
+  __shared__ __align__(8) uint64_t bar;
+  if (threadIdx.x == 0) {
+    mbar_init(smem_u32(&bar), 1);
+    fence_mbar_init();
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    const uint64_t t0 = globaltimer();
+    while (!mbar_try_wait(smem_u32(&bar), 0)) {
+      if (globaltimer() - t0 > wait_ns) {
+        raise_flag(kFlagTimeout);
+        break;
+      }
+    }
+  }
+}
+
+}  // namespace mla

@@ -1,0 +1,159 @@
+"""One MLA decode layer driven through the C ABI (device buffers + call order).
+
+``MLADecodeLayer.step`` enqueues the whole hot path on the current stream:
+
+  A0  mla_project       y = [W_Q; W_DKV; W_KR] h           (one GEMM)
+  A2  mla_rope          q_rope -> qbuf[..., d_c:],  k_rope rotated in place
+  A3  mla_cache_append  [c ; k_rope] of the new tokens -> paged pool
+  A1  mla_absorb_q      q_nope . W_UK -> qbuf[..., :d_c]
+  A4+A5 mla_decode      split-KV attention on the latent cache + LSE combine
+  A6  mla_out_proj      W_UV per head, then W_O
+
+Torch only provides device memory and the stream; every step runs in the
+library's kernels.
+"""
+
+from __future__ import annotations
+
+import numpy as np
+import torch
+
+from . import binding as _b
+from .binding import MLADims
+
+
+def _to_dev(x: np.ndarray, dtype, device):
+    return torch.from_numpy(np.ascontiguousarray(x)).to(device=device, dtype=dtype)
+
+
+class MLADecodeLayer:
+    """Weights and cache of one MLA layer on one GPU."""
+
+    def __init__(self, dims: MLADims, weights: dict, device="cuda"):
+        self.dims = dims
+        self.device = torch.device(device)
+        dt = dims.torch_dtype
+        H, dn, dr, dc = dims.n_heads, dims.d_nope, dims.d_rope, dims.d_latent
+        self.dqk = dn + dr
+        self.D = dc + dr
+        self.Y = H * self.dqk + self.D      # row width of the A0 output
+        w_a0 = np.concatenate([weights["W_Q"], weights["W_DKV"], weights["W_KR"]], 0)
+        self.W_A0 = _to_dev(w_a0, dt, self.device)
+        self.W_UK = _to_dev(weights["W_UK"], dt, self.device)
+        self.W_UV = _to_dev(weights["W_UV"], dt, self.device)
+        self.W_O = _to_dev(weights["W_O"], dt, self.device)
+        self._bufs = {}
+        self.pool = None
+
+    # ------------------------------------------------------------------
+    # cache
+    # ------------------------------------------------------------------
+    def set_cache(self, pool, page_table, seq_lens):
+        """pool [n_pages, page_size, D] (dims dtype), page_table int32
+        [B, max_pages], seq_lens int32 [B] (context after this step's append)."""
+        self.pool = pool
+        self.page_table = page_table
+        self.seq_lens = seq_lens
+        self.n_pages = pool.shape[0]
+        self.max_pages = page_table.shape[1]
+
+    def prefill_from_hidden(self, h_ctx_list):
+        """Fill each sequence's prior tokens from hidden states: project with
+        [W_DKV; W_KR], rotate the RoPE keys at positions 0.., append."""
+        d = self.dims
+        H = d.n_heads
+        w_ckv = self.W_A0[H * self.dqk:]
+        for b, h in enumerate(h_ctx_list):
+            n = h.shape[0]
+            if n == 0:
+                continue
+            hd = _to_dev(h, d.torch_dtype, self.device)
+            y = torch.empty((n, self.D), dtype=d.torch_dtype, device=self.device)
+            _b.mla_project(d, hd, w_ckv, y, n, d.d_model, self.D)
+            pos = torch.arange(n, dtype=torch.int32, device=self.device)
+            kr = y[:, d.d_latent:]
+            _b.mla_rope(d, kr, self.D, 0, 1, kr, self.D, 0, pos, n)
+            bi = torch.full((n,), b, dtype=torch.int32, device=self.device)
+            _b.mla_cache_append(d, y, self.D, kr, self.D, bi, pos, self.page_table,
+                                self.max_pages, self.pool, self.n_pages, n)
+
+    # ------------------------------------------------------------------
+    # step buffers
+    # ------------------------------------------------------------------
+    def buffers(self, B: int, S_q: int, num_workers: int = 0):
+        key = (B, S_q, num_workers)
+        if key not in self._bufs:
+            d = self.dims
+            T = B * S_q
+            dev, dt = self.device, d.torch_dtype
+            ws = _b.mla_decode_workspace_size(d, B, S_q, num_workers)
+            sc = _b.mla_out_proj_scratch_size(d, T)
+            self._bufs[key] = dict(
+                y=torch.empty((T, self.Y), dtype=dt, device=dev),
+                qbuf=torch.empty((T, d.n_heads, self.D), dtype=dt, device=dev),
+                o_lat=torch.empty((T, d.n_heads, d.d_latent), dtype=torch.float32, device=dev),
+                lse=torch.empty((T, d.n_heads), dtype=torch.float32, device=dev),
+                out=torch.empty((T, d.d_model), dtype=torch.float32, device=dev),
+                ws=torch.empty((max(ws, 256),), dtype=torch.uint8, device=dev),
+                scratch=torch.empty((max(sc, 256),), dtype=torch.uint8, device=dev),
+            )
+        return self._bufs[key]
+
+    # ------------------------------------------------------------------
+    # the hot path
+    # ------------------------------------------------------------------
+    def step(self, h, batch_idx, pos, B: int, S_q: int, num_workers: int = 0):
+        """h [T, d_model] device (dims dtype), batch_idx/pos int32 [T] device,
+        T = B*S_q tokens b-major.  Returns the dict of step buffers."""
+        d = self.dims
+        H, dn, dc, dr = d.n_heads, d.d_nope, d.d_latent, d.d_rope
+        T = B * S_q
+        bf = self.buffers(B, S_q, num_workers)
+        y, qbuf = bf["y"], bf["qbuf"]
+        Y, D, dqk = self.Y, self.D, self.dqk
+        _b.mla_project(d, h, self.W_A0, y, T, d.d_model, Y)                        # A0
+        off_c = H * dqk
+        _b.mla_rope(d, y[:, dn:], Y, dqk, H, qbuf[:, :, dc:], H * D, D, pos, T)   # A2 q
+        kr = y[:, off_c + dc:]
+        _b.mla_rope(d, kr, Y, 0, 1, kr, Y, 0, pos, T)                              # A2 k
+        _b.mla_cache_append(d, y[:, off_c:], Y, kr, Y, batch_idx, pos,             # A3
+                            self.page_table, self.max_pages, self.pool, self.n_pages, T)
+        _b.mla_absorb_q(d, y, Y, self.W_UK, qbuf, T)                                # A1
+        _b.mla_decode(d, qbuf, self.pool, self.n_pages, self.page_table,            # A4+A5
+                      self.max_pages, self.seq_lens, B, S_q, num_workers, bf["ws"],
+                      bf["o_lat"], bf["lse"])
+        _b.mla_out_proj(d, bf["o_lat"], self.W_UV, self.W_O, bf["scratch"],         # A6
+                        bf["out"], T)
+        return bf
+
+
+def build_pool_host(w, page_table, n_pages, prior_bits, canary=0xFFFF):
+    """Host image of the paged pool for workload ``w``: prior rows of each
+    sequence scattered into its pages, every other slot set to ``canary``.
+
+    prior_bits: list of [Lp_b, D] uint16 (bf16) or float32 arrays.
+    """
+    D = w.D
+    if w.dtype == "bf16":
+        pool = np.full((n_pages, w.page_size, D), canary, dtype=np.uint16)
+    else:
+        pool = np.full((n_pages, w.page_size, D), np.nan, dtype=np.float32)
+    for b, rows in enumerate(prior_bits):
+        Lp = rows.shape[0]
+        npg = -(-Lp // w.page_size)
+        if npg == 0:
+            continue
+        full = Lp // w.page_size
+        pages = page_table[b, :npg]
+        if full:
+            pool[pages[:full]] = rows[:full * w.page_size].reshape(full, w.page_size, D)
+        rem = Lp - full * w.page_size
+        if rem:
+            pool[pages[full], :rem] = rows[full * w.page_size:]
+    return pool
+
+
+def pool_to_device(pool_host: np.ndarray, dtype: str, device="cuda"):
+    if dtype == "bf16":
+        return torch.from_numpy(pool_host.view(np.int16)).to(device).view(torch.bfloat16)
+    return torch.from_numpy(pool_host).to(device)

@@ -199,6 +199,13 @@ def draw_prior(w: Workload, b: int):
     return _quant(w, c), _quant(w, kr)
 
 
+def draw_prior_bits(w: Workload, b: int) -> np.ndarray:
+    """Sequence b's prior cache rows [Lp, d_c + d_r] as bf16 bit patterns
+    (uint16), same values as draw_prior."""
+    c, kr = draw_prior(w, b)
+    return bf16_bits(np.concatenate([c, kr], axis=1))
+
+
 def draw_prior_all(w: Workload, seqs=None, threads: int = 8):
     """draw_prior for many sequences, in parallel threads."""
     seqs = list(range(w.B)) if seqs is None else list(seqs)

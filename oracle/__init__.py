@@ -11,6 +11,9 @@ from .mla_oracle import (  # noqa: F401
     project,
     attention_nonabsorbed,
     attention_absorbed,
+    absorb_query,
+    latent_attention,
+    out_proj,
     decode_step,
     cache_append,
     combine_splits,

@@ -175,6 +175,55 @@ def attention_nonabsorbed(q, C, KR, W_UK, W_UV, scale):
     return {"o": o, "o_lat": o_lat, "lse": lse, "p": probs}
 
 
+def absorb_query(q_nope, W_UK):
+    """Fold W_UK into the query: q_lat[..., i, :] = W_UK[i]^T q_nope[..., i, :].
+
+    q_nope [..., H, d_n], W_UK [H, d_n, d_c] -> [..., H, d_c].  With
+    k_{i,t} = W_UK[i] c_t, q_nope . k = q_lat . c_t (linearity).
+    """
+    q_nope = np.asarray(q_nope, dtype=F64)
+    W = np.asarray(W_UK, dtype=F64)
+    out = np.zeros(q_nope.shape[:-1] + (W.shape[2],))
+    for i in range(W.shape[0]):
+        out[..., i, :] = q_nope[..., i, :] @ W[i]
+    return out
+
+
+def latent_attention(q_abs, C, KR, scale):
+    """Attention run directly on the cache with an absorbed query.
+
+    q_abs [S_q, H, d_c + d_r] = [q_lat ; roped q_rope] per head, C [L, d_c],
+    KR [L, d_r].  Score s_t = scale * (q_lat . c_t + q_rope . KR_t), causal as
+    in attention_nonabsorbed.  Returns o_lat [S_q, H, d_c] = sum_t p_t c_t and
+    lse [S_q, H].
+    """
+    q_abs = np.asarray(q_abs, dtype=F64)
+    C = np.asarray(C, dtype=F64)
+    KR = np.asarray(KR, dtype=F64)
+    S_q, H, _ = q_abs.shape
+    L, d_c = C.shape
+    o_lat = np.zeros((S_q, H, d_c))
+    lse = np.zeros((S_q, H))
+    for j in range(S_q):
+        vis = L - S_q + j + 1
+        for i in range(H):
+            s = scale * (C[:vis] @ q_abs[j, i, :d_c] + KR[:vis] @ q_abs[j, i, d_c:])
+            _, o_lat[j, i], lse[j, i] = _softmax_attend(s, C[:vis])
+    return {"o_lat": o_lat, "lse": lse}
+
+
+def out_proj(o_lat, W_UV, W_O):
+    """Output side with W_UV folded in: o_i = W_UV[i] o_lat_i, then
+    out = W_O [o_1; ...; o_H].  o_lat [T, H, d_c] -> (o [T, H, d_v], out [T, d_model])."""
+    o_lat = np.asarray(o_lat, dtype=F64)
+    W = np.asarray(W_UV, dtype=F64)
+    o = np.zeros(o_lat.shape[:-1] + (W.shape[1],))
+    for i in range(W.shape[0]):
+        o[..., i, :] = o_lat[..., i, :] @ W[i].T
+    out = project(o.reshape(o.shape[0], -1), W_O)
+    return o, out
+
+
 def attention_absorbed(q, C, KR, W_UK, W_UV, scale):
     """Absorbed formulation of the same attention (identity check only).
 
@@ -183,25 +232,13 @@ def attention_absorbed(q, C, KR, W_UK, W_UV, scale):
     o_i = W_UV[i] (sum_t p_t c_t).
     """
     q = np.asarray(q, dtype=F64)
-    C = np.asarray(C, dtype=F64)
-    KR = np.asarray(KR, dtype=F64)
-    S_q, H, _ = q.shape
     d_n = W_UK.shape[1]
-    L = C.shape[0]
-    o = np.zeros((S_q, H, W_UV.shape[1]))
-    o_lat = np.zeros((S_q, H, C.shape[1]))
-    lse = np.zeros((S_q, H))
-    q_lat = np.zeros((S_q, H, C.shape[1]))
-    for i in range(H):
-        Wk = np.asarray(W_UK[i], dtype=F64)
-        Wv = np.asarray(W_UV[i], dtype=F64)
-        for j in range(S_q):
-            vis = L - S_q + j + 1
-            q_lat[j, i] = Wk.T @ q[j, i, :d_n]
-            s = scale * (C[:vis] @ q_lat[j, i] + KR[:vis] @ q[j, i, d_n:])
-            p, o_lat[j, i], lse[j, i] = _softmax_attend(s, C[:vis])
-            o[j, i] = Wv @ o_lat[j, i]
-    return {"o": o, "o_lat": o_lat, "lse": lse, "q_lat": q_lat}
+    q_lat = absorb_query(q[..., :d_n], W_UK)
+    att = latent_attention(np.concatenate([q_lat, q[..., d_n:]], axis=-1), C, KR, scale)
+    o = np.zeros(att["o_lat"].shape[:-1] + (W_UV.shape[1],))
+    for i in range(W_UV.shape[0]):
+        o[:, i] = att["o_lat"][:, i] @ np.asarray(W_UV[i], dtype=F64).T
+    return {"o": o, "o_lat": att["o_lat"], "lse": att["lse"], "q_lat": q_lat}
 
 
 # ---------------------------------------------------------------------------
@@ -209,7 +246,8 @@ def attention_absorbed(q, C, KR, W_UK, W_UV, scale):
 # ---------------------------------------------------------------------------
 
 def decode_step(h_new, c_prior, krpre_prior, W_Q, W_DKV, W_KR, W_UK, W_UV,
-                W_O, scale, rope_base, n_heads, seqs=None):
+                W_O, scale, rope_base, n_heads, seqs=None,
+                prior_kr_rotated=False, heads=None, formulation="nonabsorbed"):
     """One MLA decode step for a batch, non-absorbed, fp64.
 
     h_new        [B, S_q, d_model]   hidden states of the new tokens
@@ -219,6 +257,13 @@ def decode_step(h_new, c_prior, krpre_prior, W_Q, W_DKV, W_KR, W_UK, W_UV,
     W_Q [H*(d_n+d_r), d_model], W_DKV [d_c, d_model], W_KR [d_r, d_model],
     W_UK [H, d_n, d_c], W_UV [H, d_v, d_c], W_O [d_model, H*d_v]
     seqs         optional subset of sequence indices to evaluate
+    prior_kr_rotated  the prior RoPE keys are given as cached, i.e. already
+                 rotated (workloads that draw the cache directly)
+    heads        optional subset of heads for the attention (the output
+                 projection needs every head and is then skipped)
+    formulation  "nonabsorbed" (default, the reference) or "absorbed" (the
+                 pinned-equal absorbed formulation, far cheaper at long
+                 context because it never rebuilds keys and values)
 
     Steps per sequence b (positions per reading R2):
       1. new tokens: c = W_DKV h, kr = RoPE(W_KR h, pos), pos = L-S_q .. L-1
@@ -244,15 +289,20 @@ def decode_step(h_new, c_prior, krpre_prior, W_Q, W_DKV, W_KR, W_UK, W_UV,
         kr_new = rope(project(h_new[b], W_KR), pos, rope_base)
         C = np.concatenate([np.asarray(c_prior[b], dtype=F64).reshape(Lp, d_c),
                             c_new], axis=0)
-        KR = np.concatenate([rope(np.asarray(krpre_prior[b], dtype=F64)
-                                  .reshape(Lp, d_r), np.arange(Lp), rope_base),
-                             kr_new], axis=0)
+        kr_prior = np.asarray(krpre_prior[b], dtype=F64).reshape(Lp, d_r)
+        if not prior_kr_rotated:
+            kr_prior = rope(kr_prior, np.arange(Lp), rope_base)
+        KR = np.concatenate([kr_prior, kr_new], axis=0)
         q = project(h_new[b], W_Q).reshape(S_q, H, d_qk)
         q_roped = q.copy()
         q_roped[..., d_qk - d_r:] = rope(q[..., d_qk - d_r:], pos[:, None],
                                          rope_base)
-        att = attention_nonabsorbed(q_roped, C, KR, W_UK, W_UV, scale)
-        out = project(att["o"].reshape(S_q, -1), W_O)
+        hs = list(range(H)) if heads is None else list(heads)
+        attn = attention_nonabsorbed if formulation == "nonabsorbed" \
+            else attention_absorbed
+        att = attn(q_roped[:, hs], C, KR, np.asarray(W_UK)[hs],
+                   np.asarray(W_UV)[hs], scale)
+        out = project(att["o"].reshape(S_q, -1), W_O) if heads is None else None
         res["q"][b] = q
         res["q_roped"][b] = q_roped
         res["c_new"][b] = c_new

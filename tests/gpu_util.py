@@ -1,0 +1,66 @@
+"""Shared helpers of the GPU parity tests (tolerances, conversions)."""
+
+import numpy as np
+import torch
+
+from mla_latent_kv_35_b200 import binding as B
+from mla_latent_kv_35_b200 import build as _build
+from mla_latent_kv_35_b200 import workloads as wl
+
+DEV = "cuda"
+
+# bf16 cache and weights with fp32 accumulation: max-abs 2e-2, mean-abs 2e-3;
+# fp32 path: 1e-4 max-abs.  Relative L2 error is reported and bounded too
+# (outputs shrink like L^-1/2 with N(0,1) data, so absolute bounds alone are
+# loose at long context).
+TOL = {"bf16": dict(max_abs=2e-2, mean_abs=2e-3, rel_l2=1e-2),
+       "f32": dict(max_abs=1e-4, mean_abs=1e-5, rel_l2=1e-4)}
+
+
+def ensure_lib():
+    _build.build()
+    return B.lib()
+
+
+def dims(dtype="bf16", H=128, dn=128, dc=512, dr=64, dm=5120, page=64):
+    return B.MLADims(H, dn, dc, dr, dn, dm, page, (dn + dr) ** -0.5, 10000.0, dtype)
+
+
+def to_dev(x, dtype):
+    t = torch.from_numpy(np.ascontiguousarray(x, dtype=np.float32))
+    return t.to(DEV, torch.bfloat16 if dtype == "bf16" else torch.float32)
+
+
+def to_np(t):
+    return t.detach().float().cpu().numpy().astype(np.float64)
+
+
+def q(x, dtype):
+    """Round host values to what the device stores (bf16 RNE or fp32)."""
+    x = np.asarray(x, dtype=np.float32)
+    return wl.bf16_to_f32(wl.bf16_bits(x)) if dtype == "bf16" else x
+
+
+def check(got, ref, dtype, what="", tol=None):
+    got = np.asarray(got, dtype=np.float64)
+    ref = np.asarray(ref, dtype=np.float64)
+    assert got.shape == ref.shape, (what, got.shape, ref.shape)
+    t = dict(TOL[dtype])
+    if tol:
+        t.update(tol)
+    finite = np.isfinite(ref)
+    assert (np.isfinite(got) == finite).all(), f"{what}: non-finite mismatch"
+    d = np.abs(got[finite] - ref[finite])
+    mx = float(d.max()) if d.size else 0.0
+    mean = float(d.mean()) if d.size else 0.0
+    nrm = float(np.linalg.norm(ref[finite]))
+    rel = float(np.linalg.norm(d) / nrm) if nrm > 0 else 0.0
+    msg = f"{what}: max_abs={mx:.3e} mean_abs={mean:.3e} rel_l2={rel:.3e}"
+    assert mx <= t["max_abs"], msg
+    assert mean <= t["mean_abs"], msg
+    assert rel <= t["rel_l2"], msg
+    return mx, mean, rel
+
+
+def status():
+    return B.mla_get_device_status()

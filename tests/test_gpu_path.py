@@ -1,0 +1,134 @@
+"""Whole decode step (A0-A6) on the GPU against the oracle, per workload.
+
+tiny: every sequence, non-absorbed oracle, fp32 tolerance.
+bf16 workloads at full size, in the launch configuration the benchmark
+times: sampled sequences.  For each sampled sequence a few heads go through
+the non-absorbed oracle (explicit per-head keys and values) and all heads
+through the oracle's absorbed formulation (pinned equal to it to 1e-10),
+which also gives the reference for the output projection.
+"""
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from mla_latent_kv_35_b200 import workloads as wl
+from mla_latent_kv_35_b200.binding import MLADims
+from mla_latent_kv_35_b200.engine import MLADecodeLayer, build_pool_host, pool_to_device
+from gpu_util import DEV, check, ensure_lib, status, to_np
+
+gpu = pytest.mark.gpu
+
+
+def _setup(w):
+    ensure_lib()
+    W = wl.draw_weights(w)
+    d = MLADims.of(w)
+    layer = MLADecodeLayer(d, W, DEV)
+    table, n_pages = wl.page_layout(w)
+    if w.prior_from_h:
+        prior = [np.zeros((0, w.D), np.float32) for _ in range(w.B)]
+    elif w.dtype == "bf16":
+        from concurrent.futures import ThreadPoolExecutor
+        with ThreadPoolExecutor(8) as ex:
+            prior = list(ex.map(lambda b: wl.draw_prior_bits(w, b), range(w.B)))
+    else:
+        prior = [np.concatenate(wl.draw_prior(w, b), 1) for b in range(w.B)]
+    pool = pool_to_device(build_pool_host(w, table, n_pages, prior), w.dtype, DEV)
+    del prior
+    layer.set_cache(pool, torch.from_numpy(table).to(DEV),
+                    torch.tensor(w.ctx, dtype=torch.int32, device=DEV))
+    h_ctx = None
+    if w.prior_from_h:
+        h_ctx = [wl.draw_h_ctx(w, b) for b in range(w.B)]
+        layer.prefill_from_hidden(h_ctx)
+    h = wl.draw_h_new(w)
+    bi, pos = wl.positions(w)
+    hd = torch.from_numpy(h.reshape(w.T, w.d_model)).to(DEV, d.torch_dtype)
+    bf = layer.step(hd, torch.from_numpy(bi).to(DEV), torch.from_numpy(pos).to(DEV), w.B,
+                    w.S_q)
+    torch.cuda.synchronize()
+    assert status() == 0
+    return W, layer, bf, h, h_ctx, table
+
+
+@gpu
+def test_tiny_full_path_fp32():
+    w = wl.workload("tiny")
+    W, layer, bf, h, h_ctx, table = _setup(w)
+    c_prior = [oracle.project(x, W["W_DKV"]) for x in h_ctx]
+    kr_prior = [oracle.project(x, W["W_KR"]) for x in h_ctx]
+    res = oracle.decode_step(h, c_prior, kr_prior, W["W_Q"], W["W_DKV"], W["W_KR"], W["W_UK"],
+                             W["W_UV"], W["W_O"], w.scale, w.rope_base, w.H)
+    H, dqk, dc = w.H, w.d_nope + w.d_rope, w.d_latent
+    y = to_np(bf["y"])
+    qbuf = to_np(bf["qbuf"])
+    o_lat = to_np(bf["o_lat"])
+    lse = to_np(bf["lse"])
+    out = to_np(bf["out"])
+    pool = to_np(layer.pool)
+    for b in range(w.B):
+        check(y[b, :H * dqk].reshape(H, dqk), res["q"][b][0], "f32", "A0 q")
+        check(qbuf[b, :, dc:], res["q_roped"][b][0, :, w.d_nope:], "f32", "A2 q_rope")
+        L = w.ctx[b]
+        row = pool[table[b, (L - 1) // 64], (L - 1) % 64]
+        check(row[:dc], res["c_new"][b][0], "f32", "A3 c")
+        check(row[dc:], res["kr_new"][b][0], "f32", "A3 k_rope")
+        check(o_lat[b], res["o_lat"][b][0], "f32", "A4 o_lat")
+        check(lse[b], res["lse"][b][0], "f32", "A4 lse")
+        check(out[b], res["out"][b][0], "f32", "A6 out")
+
+
+def _check_bf16_workload(name, sample, nonabs_heads=(0, 77, 127)):
+    w = wl.workload(name)
+    W, layer, bf, h, _, table = _setup(w)
+    o_lat = to_np(bf["o_lat"]).reshape(w.B, w.S_q, w.H, w.d_latent)
+    lse = to_np(bf["lse"]).reshape(w.B, w.S_q, w.H)
+    out = to_np(bf["out"]).reshape(w.B, w.S_q, w.d_model)
+    pool = layer.pool.view(torch.int16)
+    for b in sample:
+        c, kr = wl.draw_prior(w, b)
+        args = (h[b:b + 1], [c], [kr], W["W_Q"], W["W_DKV"], W["W_KR"], W["W_UK"], W["W_UV"],
+                W["W_O"], w.scale, w.rope_base, w.H)
+        ab = oracle.decode_step(*args, prior_kr_rotated=True, formulation="absorbed")
+        na = oracle.decode_step(*args, prior_kr_rotated=True, heads=list(nonabs_heads))
+        check(o_lat[b], ab["o_lat"][0], "bf16", f"{name} b={b} o_lat (all heads)")
+        check(lse[b], ab["lse"][0], "bf16", f"{name} b={b} lse")
+        check(out[b], ab["out"][0], "bf16", f"{name} b={b} out")
+        check(o_lat[b][:, list(nonabs_heads)], na["o_lat"][0], "bf16",
+              f"{name} b={b} o_lat vs non-absorbed")
+        check(lse[b][:, list(nonabs_heads)], na["lse"][0], "bf16",
+              f"{name} b={b} lse vs non-absorbed")
+        # the appended rows hold the new tokens' latent and rotated RoPE key
+        L = w.ctx[b]
+        for j in range(w.S_q):
+            p = L - w.S_q + j
+            row = pool[int(table[b, p // 64]), p % 64].cpu().numpy().view(np.uint16)
+            rowf = wl.bf16_to_f32(row).astype(np.float64)
+            check(rowf[:w.d_latent], ab["c_new"][0][j], "bf16", "A3 c_new")
+            check(rowf[w.d_latent:], ab["kr_new"][0][j], "bf16", "A3 kr_new")
+
+
+@gpu
+def test_dsv2_full_path():
+    _check_bf16_workload("dsv2", sample=[0, 9, 15])
+
+
+@gpu
+def test_ragged_full_path():
+    w = wl.workload("ragged")
+    lens = np.array(w.ctx)
+    sample = [int(np.argmin(lens)), int(np.argmax(lens)), 5]
+    _check_bf16_workload("ragged", sample=sample)
+
+
+@gpu
+def test_batch128_full_path():
+    _check_bf16_workload("batch128", sample=[0, 127], nonabs_heads=(3, 100))
+
+
+@gpu
+@pytest.mark.parametrize("name", ["long1", "long4"])
+def test_long_context_full_path(name):
+    _check_bf16_workload(name, sample=[0] if name == "long1" else [0, 3], nonabs_heads=(64,))

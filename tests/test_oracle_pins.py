@@ -354,3 +354,14 @@ def test_planted_mistakes_are_caught(monkeypatch):
     x = np.array([0.3, -1.2])
     wrong = oracle.rope(x, -5, 10000.0)
     assert np.abs(wrong - _rope_complex(x, 5, 10000.0)).max() > 1e-3
+
+
+def test_out_proj_matches_nonabsorbed_output():
+    """out_proj(o_lat) equals W_O applied to the explicit per-head outputs."""
+    rng = np.random.default_rng(13)
+    P = _rand_problem(rng, S_q=1, H=3, L=11)
+    res = oracle.attention_nonabsorbed(**P)
+    W_O = rng.standard_normal((7, 3 * 5))
+    o, out = oracle.out_proj(res["o_lat"], P["W_UV"], W_O)
+    np.testing.assert_allclose(o, res["o"], atol=1e-12)
+    np.testing.assert_allclose(out, res["o"].reshape(1, -1) @ W_O.T, atol=1e-12)
