@@ -1,0 +1,396 @@
+"""Benchmark of one MLA decode step (A0-A6) on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME]
+                    [--impl reference]
+
+A step is one pass of the whole hot path over one batch: projection (A0),
+RoPE (A2), cache append (A3), query absorption (A1), split-KV decode on the
+paged latent cache with LSE combine (A4+A5) and the output projection (A6),
+enqueued through the C ABI on one stream.  Inputs are seeded synthetic data of
+the DeepSeek-V2 attention shapes (workloads.py); the default workload is
+`batch128` (B=128, 128 heads, latent 512 + RoPE 64, context 32768 in 64-token
+pages scattered by a seeded permutation): its 4.83 GB cache is far larger
+than the 126 MB L2, so no flush is needed between steps.
+
+Prints ONE JSON line (rank 0).  `value` is decode tokens per second of the
+whole step (B*S_q query tokens per step, summed over ranks); `roofline`
+describes the decode call (split kernel + combine); `e2e` repeats the
+measurement through the same public API with host buffers (inputs copied in
+from pinned memory and the output copied back inside the timed region).
+With --gpus N > 1 every rank runs its own batch (independent sequences, no
+data-path collective: weak scaling).
+"""
+
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+
+
+def _peaks():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            p = json.load(f)
+        return float(p["hbm_gbs"]), float(p["bf16_tflops"]), "measured"
+    except Exception:
+        return 6650.0, 1590.0, "fallback"
+
+
+def _workload_bytes(w):
+    """Algorithmic bytes and FLOPs of the decode call (A4+A5) per step."""
+    D = w.D
+    vis = []
+    for L in w.ctx:
+        for j in range(w.S_q):
+            vis.append(L - w.S_q + j + 1)
+    cache = sum(w.ctx) * D * 2
+    q = w.T * w.H * D * 2
+    out = w.T * w.H * (w.d_latent + 1) * 4
+    flops = 2 * w.H * (D + w.d_latent) * sum(vis)
+    return cache + q + out, flops, cache
+
+
+class ClockSampler:
+    """nvidia-smi samples of SM clock and throttle reasons while running."""
+
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index):
+        self.idx = gpu_index
+        self.proc = None
+        self.lines = []
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.idx), f"--query-gpu={self.Q}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.t = threading.Thread(target=self._read, daemon=True)
+            self.t.start()
+        except Exception:
+            self.proc = None
+        return self
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def __exit__(self, *a):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except Exception:
+                self.proc.kill()
+
+    def summary(self):
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            f = [x.strip() for x in ln.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                mx = float(f[2])
+            except ValueError:
+                continue
+            for n, v in zip(names, f[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+def _traffic_for(kernel_src_paths):
+    """ncu DRAM bytes per decode call recorded in profiles/, if the kernel
+    source is unchanged since the capture (else None)."""
+    path = os.path.join(ROOT, "profiles", "decode_tc_traffic.json")
+    try:
+        with open(path) as f:
+            rec = json.load(f)
+    except Exception:
+        return None
+    h = hashlib.sha256()
+    for p in kernel_src_paths:
+        with open(p, "rb") as f:
+            h.update(f.read())
+    if rec.get("source_sha256") != h.hexdigest():
+        return None
+    return rec.get("dram_bytes_per_call")
+
+
+# ---------------------------------------------------------------------------
+# CPU oracle arm
+# ---------------------------------------------------------------------------
+def _oracle_sample(w, budget_s=25.0):
+    """Time the oracle's decode step on whole sequences of the workload until
+    about budget_s seconds of CPU work; returns (tokens/s, sample text, cores)."""
+    import oracle
+    from mla_latent_kv_35_b200 import workloads as wl
+    W = wl.draw_weights(w)
+    h = wl.draw_h_new(w)
+    cores = len(os.sched_getaffinity(0))
+    t_total, toks, seqs = 0.0, 0, 0
+    for b in range(w.B):
+        c, kr = wl.draw_prior(w, b)
+        t0 = time.perf_counter()
+        oracle.decode_step(h[b:b + 1], [c], [kr], W["W_Q"], W["W_DKV"], W["W_KR"], W["W_UK"],
+                           W["W_UV"], W["W_O"], w.scale, w.rope_base, w.H,
+                           prior_kr_rotated=True)
+        t_total += time.perf_counter() - t0
+        toks += w.S_q
+        seqs += 1
+        if t_total >= budget_s:
+            break
+    sample = (f"{seqs} of {w.B} sequences of {w.name} (context {w.ctx[0]}), all {w.H} heads, "
+              f"fp64 non-absorbed oracle, {t_total:.1f} s")
+    return toks / t_total, sample, cores, t_total
+
+
+def run_reference(args, w):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    tps = []
+    sample = ""
+    cores = len(os.sched_getaffinity(0))
+    budget = max(5.0, 60.0 / max(1, args.steps + args.warmup))
+    for i in range(args.warmup + args.steps):
+        v, sample, cores, _ = _oracle_sample(w, budget_s=budget)
+        if i >= args.warmup:
+            tps.append(v)
+    value = statistics.mean(tps)
+    line = {
+        "impl": "reference",
+        "metric": "MLA decode tokens/s (one attention layer, whole step A0-A6)",
+        "value": value, "unit": "tokens/s", "n_gpus": args.gpus, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": 1000.0 * w.T / value,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic",
+        "config": {"workload": w.name, "batch": w.B, "heads": w.H, "context": w.ctx[0],
+                   "S_q": w.S_q, "latent": w.d_latent, "rope": w.d_rope},
+        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+# ---------------------------------------------------------------------------
+# GPU arm
+# ---------------------------------------------------------------------------
+def run_gpu(args, w):
+    import torch
+    import torch.distributed as dist
+    from mla_latent_kv_35_b200 import binding as B
+    from mla_latent_kv_35_b200 import build as _build
+    from mla_latent_kv_35_b200 import workloads as wl
+    from mla_latent_kv_35_b200.engine import (MLADecodeLayer, build_pool_host,
+                                               build_pool_host_drawn, pool_to_device)
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=600),
+                                device_id=dev)
+    if rank == 0:
+        _build.build()
+    if world > 1:
+        dist.barrier()
+    B.lib()
+
+    d = B.MLADims.of(w)
+    W = wl.draw_weights(w)
+    layer = MLADecodeLayer(d, W, dev)
+    table, n_pages = wl.page_layout(w)
+    if w.prior_from_h:
+        host = build_pool_host(w, table, n_pages, [np.zeros((0, w.D), np.float32)] * w.B)
+    else:
+        host = build_pool_host_drawn(w, table, n_pages)
+    pool = pool_to_device(host, w.dtype, dev)
+    del host
+    layer.set_cache(pool, torch.from_numpy(table).to(dev),
+                    torch.tensor(w.ctx, dtype=torch.int32, device=dev))
+    if w.prior_from_h:
+        layer.prefill_from_hidden([wl.draw_h_ctx(w, b) for b in range(w.B)])
+    h_np = wl.draw_h_new(w).reshape(w.T, w.d_model)
+    bi_np, pos_np = wl.positions(w)
+    h = torch.from_numpy(h_np).to(dev, d.torch_dtype)
+    bi = torch.from_numpy(bi_np).to(dev)
+    pos = torch.from_numpy(pos_np).to(dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def step(ev=None):
+        if ev is not None:
+            ev[0].record(stream)
+        layer.step(h, bi, pos, w.B, w.S_q)
+        if ev is not None:
+            ev[1].record(stream)
+
+    # the decode call alone, with events on the launching stream
+    bf = layer.buffers(w.B, w.S_q)
+
+    def decode_only():
+        B.mla_decode(d, bf["qbuf"], layer.pool, layer.n_pages, layer.page_table,
+                     layer.max_pages, layer.seq_lens, w.B, w.S_q, 0, bf["ws"], bf["o_lat"],
+                     bf["lse"])
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize(dev)
+    st = B.mla_get_device_status()
+    if st != 0:
+        raise RuntimeError(f"device status after warm-up: {B.mla_status_string(st)}")
+
+    def timed(fn, K):
+        evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+               for _ in range(K)]
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize(dev)
+        l0 = B.mla_launch_count()
+        t0 = time.perf_counter()
+        for e in evs:
+            e[0].record(stream)
+            fn()
+            e[1].record(stream)
+        torch.cuda.synchronize(dev)
+        wall = time.perf_counter() - t0
+        launches = B.mla_launch_count() - l0
+        if world > 1:
+            dist.barrier()
+        ms = [a.elapsed_time(b) for a, b in evs]
+        return ms, wall, launches
+
+    with ClockSampler(local) as clk:
+        step_ms, wall, launches = timed(step, args.steps)
+        dec_ms, _, dec_launches = timed(decode_only, max(args.steps, 5))
+    clocks = clk.summary()
+    st = B.mla_get_device_status()
+    if st != 0:
+        raise RuntimeError(f"device status after timing: {B.mla_status_string(st)}")
+
+    # end to end through the public API with host buffers
+    h_host = torch.from_numpy(h_np).to(d.torch_dtype).pin_memory()
+    bi_host = torch.from_numpy(bi_np).pin_memory()
+    pos_host = torch.from_numpy(pos_np).pin_memory()
+    out_host = torch.empty((w.T, w.d_model), dtype=torch.float32).pin_memory()
+
+    def e2e_step():
+        h.copy_(h_host, non_blocking=True)
+        bi.copy_(bi_host, non_blocking=True)
+        pos.copy_(pos_host, non_blocking=True)
+        b = layer.step(h, bi, pos, w.B, w.S_q)
+        out_host.copy_(b["out"], non_blocking=True)
+
+    for _ in range(2):
+        e2e_step()
+    e2e_ms, _, _ = timed(e2e_step, args.steps)
+    h2d = h_host.numel() * h_host.element_size() + bi_host.numel() * 4 + pos_host.numel() * 4
+    d2h = out_host.numel() * 4
+
+    # max over ranks
+    t_step = sum(step_ms) / len(step_ms)
+    t_dec = sum(dec_ms) / len(dec_ms)
+    t_e2e = sum(e2e_ms) / len(e2e_ms)
+    if world > 1:
+        tt = torch.tensor([t_step, t_dec, t_e2e], device=dev)
+        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+        t_step, t_dec, t_e2e = tt.tolist()
+
+    hbm_peak, tf_peak, peak_kind = _peaks()
+    alg_bytes, flops, cache_bytes = _workload_bytes(w)
+    achieved = alg_bytes / (t_dec * 1e-3) / 1e9
+    roof_t = max(alg_bytes / (hbm_peak * 1e9), flops / (tf_peak * 1e12))
+    csrc = os.path.join(ROOT, "mla_latent_kv_35_b200", "csrc")
+    traffic = _traffic_for([os.path.join(csrc, "decode_tc.cuh")])
+    tokens = w.T * world
+    line = {
+        "metric": "MLA decode tokens/s (one attention layer, whole step A0-A6)",
+        "value": tokens / (t_step * 1e-3),
+        "unit": "tokens/s",
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": t_step,
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "bf16" if w.dtype == "bf16" else "f32",
+        "data": "synthetic",
+        "config": {"workload": w.name, "batch_per_gpu": w.B, "heads": w.H,
+                   "context": w.ctx[0] if len(set(w.ctx)) == 1 else "ragged",
+                   "S_q": w.S_q, "latent": w.d_latent, "rope": w.d_rope,
+                   "page": w.page_size, "d_model": w.d_model,
+                   "l2": "inputs larger than L2 (cache %.2f GB), no flush" % (cache_bytes / 1e9),
+                   "parallelism": f"replicas x{world}" if world > 1 else "single GPU"},
+        "decode": {"ms": t_dec, "tokens_per_s": tokens / (t_dec * 1e-3),
+                   "cache_gb_per_s": cache_bytes / (t_dec * 1e-3) / 1e9,
+                   "tflops": flops / (t_dec * 1e-3) / 1e12,
+                   "roofline_ms": roof_t * 1e3, "frac_of_roofline": roof_t / (t_dec * 1e-3)},
+        "roofline": {"kernel": "mla_decode (decode_tc_kernel + combine)", "bound": "hbm",
+                     "achieved": achieved, "peak": hbm_peak, "unit": "GB/s",
+                     "frac": achieved / hbm_peak, "peak_source": peak_kind,
+                     "alg_bytes_per_launch": alg_bytes, "traffic": traffic},
+        "e2e": {"value": tokens / (t_e2e * 1e-3), "unit": "tokens/s", "ms_per_step": t_e2e,
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+        "gpu_launches": launches,
+        "clocks": clocks,
+        "wall_s_timed": wall,
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        v, sample, cores, _ = _oracle_sample(w, budget_s=20.0)
+        line["cpu_baseline"] = {"value": v, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+                                "sample": sample}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--workload", default="batch128")
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+    from mla_latent_kv_35_b200 import workloads as wl
+    w = wl.workload(args.workload)
+    if args.impl == "reference":
+        run_reference(args, w)
+    else:
+        run_gpu(args, w)
+
+
+if __name__ == "__main__":
+    main()

@@ -369,8 +369,9 @@ mla_status mla_decode(const mla_dims* dims, const void* qbuf, const void* pool, 
   const int H = dims->n_heads, dc = dims->d_latent, dr = dims->d_rope;
   if (use_tc_decode(dims, S_q)) {
     if (!aligned16(qbuf) || !aligned16(pool)) return MLA_ERR_INVALID_ARG;
-    MLA_TRY(launch_decode_tc(qbuf, pool, n_pages, page_table, max_pages, seq_lens, B, S_q, H,
-                             dims->scale, L.G, start, ws_lse, ws_o, st));
+    MLA_TRY(launch_decode_tc_impl(make_tmap_bf16, qbuf, pool, n_pages, page_table, max_pages,
+                                  seq_lens, B, S_q, H, dims->scale, L.G, start, ws_lse, ws_o,
+                                  st));
     g_launches.fetch_add(1, std::memory_order_relaxed);
   } else {
     dim3 grid(L.G, (L.rows_per_v + 7) / 8);

@@ -153,6 +153,38 @@ def build_pool_host(w, page_table, n_pages, prior_bits, canary=0xFFFF):
     return pool
 
 
+def build_pool_host_drawn(w, page_table, n_pages, canary=0xFFFF, threads=8):
+    """Like build_pool_host, drawing each sequence's prior rows from the
+    seeded generator inside worker threads (no full copy of the priors)."""
+    from concurrent.futures import ThreadPoolExecutor
+
+    from . import workloads as wl
+    D = w.D
+    if w.dtype == "bf16":
+        pool = np.full((n_pages, w.page_size, D), canary, dtype=np.uint16)
+    else:
+        pool = np.full((n_pages, w.page_size, D), np.nan, dtype=np.float32)
+
+    def fill(b):
+        if w.dtype == "bf16":
+            rows = wl.draw_prior_bits(w, b)
+        else:
+            rows = np.concatenate(wl.draw_prior(w, b), 1)
+        Lp = rows.shape[0]
+        full = Lp // w.page_size
+        npg = -(-Lp // w.page_size)
+        pages = page_table[b, :npg]
+        if full:
+            pool[pages[:full]] = rows[:full * w.page_size].reshape(full, w.page_size, D)
+        rem = Lp - full * w.page_size
+        if rem:
+            pool[pages[full], :rem] = rows[full * w.page_size:]
+
+    with ThreadPoolExecutor(threads) as ex:
+        list(ex.map(fill, range(w.B)))
+    return pool
+
+
 def pool_to_device(pool_host: np.ndarray, dtype: str, device="cuda"):
     if dtype == "bf16":
         return torch.from_numpy(pool_host.view(np.int16)).to(device).view(torch.bfloat16)
