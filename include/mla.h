@@ -173,6 +173,14 @@ mla_status mla_out_proj(const mla_dims* dims, const float* o_lat,
  * wins if both were raised), or MLA_ERR_CUDA if the stream failed. */
 mla_status mla_get_device_status(void* stream);
 
+/* Where the first bounded wait that ran out on the current device gave up
+ * since the last call: out4 = {site, info, parity, CTA index}, all zero if
+ * none did.  Sites: 1-10 split-decode kernel (1 producer slot free, 2 query
+ * slice free, 3 MMA operands landed, 4 P ready, 5 O free, 6 query landed,
+ * 7 S ready, 8-10 PV done), 21-23 GEMM.  Reads and clears the record
+ * (synchronous copy; call after mla_get_device_status). */
+mla_status mla_get_wait_diag(uint32_t* out4);
+
 /* Static, human-readable text for a status code. */
 const char* mla_status_string(mla_status s);
 

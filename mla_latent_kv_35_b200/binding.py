@@ -25,7 +25,7 @@ STATUS = {0: "MLA_OK", 1: "MLA_ERR_INVALID_ARG", 2: "MLA_ERR_UNSUPPORTED",
 EXPORTS = ("mla_project", "mla_absorb_q", "mla_rope", "mla_cache_append",
            "mla_decode_workspace_size", "mla_decode", "mla_out_proj_scratch_size",
            "mla_out_proj", "mla_get_device_status", "mla_status_string",
-           "mla_launch_count", "mla_selftest_wait_timeout")
+           "mla_launch_count", "mla_selftest_wait_timeout", "mla_get_wait_diag")
 
 
 class MLAError(RuntimeError):
@@ -89,6 +89,7 @@ _SIGS = {
     "mla_status_string": ([_I], ctypes.c_char_p),
     "mla_launch_count": ([], ctypes.c_uint64),
     "mla_selftest_wait_timeout": ([ctypes.c_ulonglong, _P], _I),
+    "mla_get_wait_diag": ([ctypes.POINTER(ctypes.c_uint32)], _I),
 }
 
 
@@ -187,6 +188,13 @@ def mla_out_proj(dims: MLADims, o_lat, w_uv, w_o, scratch, out, T: int):
 def mla_get_device_status() -> int:
     """Synchronise the current stream; return and clear the device status."""
     return int(lib().mla_get_device_status(_stream()))
+
+
+def mla_get_wait_diag():
+    """(site, info, parity, cta) of the first bounded wait that gave up."""
+    out = (ctypes.c_uint32 * 4)()
+    _check("mla_get_wait_diag", lib().mla_get_wait_diag(out))
+    return tuple(int(x) for x in out)
 
 
 def mla_status_string(code: int) -> str:

@@ -254,6 +254,15 @@ mla_status mla_get_device_status(void* stream) {
   return MLA_OK;
 }
 
+mla_status mla_get_wait_diag(uint32_t* out4) {
+  if (out4 == nullptr) return MLA_ERR_INVALID_ARG;
+  unsigned v[4] = {0, 0, 0, 0}, z[4] = {0, 0, 0, 0};
+  if (cudaMemcpyFromSymbol(v, g_wait_diag, sizeof(v)) != cudaSuccess) return MLA_ERR_CUDA;
+  if (cudaMemcpyToSymbol(g_wait_diag, z, sizeof(z)) != cudaSuccess) return MLA_ERR_CUDA;
+  for (int i = 0; i < 4; ++i) out4[i] = v[i];
+  return MLA_OK;
+}
+
 mla_status mla_selftest_wait_timeout(unsigned long long wait_ns, void* stream) {
   wait_selftest_kernel<<<1, 32, 0, as_stream(stream)>>>(wait_ns);
   return check_launch();

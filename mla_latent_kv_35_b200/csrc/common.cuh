@@ -25,6 +25,18 @@ __device__ unsigned int g_status;
 
 __device__ __forceinline__ void raise_flag(unsigned f) { atomicOr(&g_status, f); }
 
+// Where the first bounded wait that ran out gave up: {site, info, parity,
+// block index}.  Read and cleared through mla_get_wait_diag.
+__device__ unsigned int g_wait_diag[4];
+
+__device__ __forceinline__ void record_timeout(unsigned site, unsigned info, unsigned parity) {
+  if (atomicCAS(&g_wait_diag[0], 0u, site) == 0u) {
+    g_wait_diag[1] = info;
+    g_wait_diag[2] = parity;
+    g_wait_diag[3] = blockIdx.x;
+  }
+}
+
 // Bounded waits give up after this many nanoseconds of %globaltimer.
 #ifndef MLA_WAIT_NS
 #define MLA_WAIT_NS 1000000000ull
@@ -82,7 +94,8 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
 // Wait for phase `parity` of the barrier to complete.  Gives up after
 // MLA_WAIT_NS (raising kFlagTimeout and setting *abort) or as soon as another
 // thread of the CTA has set *abort.  Returns false when it gave up.
-__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int* abort) {
+__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int* abort,
+                                          unsigned site = 0, unsigned info = 0) {
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = globaltimer();
   for (uint32_t it = 1;; ++it) {
@@ -91,6 +104,7 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatil
       if (abort != nullptr && *abort) return false;
       if (globaltimer() - t0 > MLA_WAIT_NS) {
         raise_flag(kFlagTimeout);
+        record_timeout(site == 0 ? 0xFFu : site, info, parity);
         if (abort != nullptr) *abort = 1;
         return false;
       }

@@ -212,7 +212,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(dtc::kThreads, 1)
     int pv_pend_b = -1, pv_pend_L = 0, pv_pend_x = 0;  // pending PV block
     auto load_stage = [&](int page, int slot0, int cc0, int nchunks) -> bool {
       const int s = it % kStages;
-      if (!mbar_wait(smem_u32(&empty_bar[s]), ((it / kStages) & 1) ^ 1, abort_p)) return false;
+      if (!mbar_wait(smem_u32(&empty_bar[s]), ((it / kStages) & 1) ^ 1, abort_p, 1, it)) return false;
       const uint32_t fb = leader_full0 + s * 8;
       mbar_expect_tx_cluster(fb, nchunks * 8192);
       const uint32_t dst = sRing + s * kStageBytes;
@@ -234,7 +234,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(dtc::kThreads, 1)
       const int b = v / P.R, rb = v % P.R;
       const int L = P.seq_lens[b];
       // Q slice of this piece (needs the previous piece's QK MMAs finished)
-      if (piece > 0 && !mbar_wait(smem_u32(&q_empty), (piece - 1) & 1, abort_p)) { ok = false; break; }
+      if (piece > 0 && !mbar_wait(smem_u32(&q_empty), (piece - 1) & 1, abort_p, 2, piece)) { ok = false; break; }
       mbar_expect_tx_cluster(leader_qfull, kQBytes);
       const int row0 = b * rows_seq + rb * 128 + 64 * (int)rank;
       for (int c = 0; c < 9; ++c) tma_load_2d_pair(sQ + c * 8192, &tmQ, c * 64, row0, leader_qfull);
@@ -270,13 +270,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(dtc::kThreads, 1)
     int pend_piece = 0;
     auto consume = [&](int& s) -> bool {
       s = it % kStages;
-      if (!mbar_wait(smem_u32(&full_bar[s]), (it / kStages) & 1, abort_p)) return false;
+      if (!mbar_wait(smem_u32(&full_bar[s]), (it / kStages) & 1, abort_p, 3, it)) return false;
       tc_fence_after();
       return true;
     };
     auto issue_pv = [&](int jb, bool first, int pc) -> bool {
-      if (!mbar_wait(smem_u32(&p_full[jb & 1]), (jb >> 1) & 1, abort_p)) return false;
-      if (first && pc > 0 && !mbar_wait(smem_u32(&o_empty), (pc - 1) & 1, abort_p)) return false;
+      if (!mbar_wait(smem_u32(&p_full[jb & 1]), (jb >> 1) & 1, abort_p, 4, jb)) return false;
+      if (first && pc > 0 && !mbar_wait(smem_u32(&o_empty), (pc - 1) & 1, abort_p, 5, pc)) return false;
       tc_fence_after();
       const uint32_t pbuf = sP + (jb & 1) * kPBytes;
       for (int n = 0; n < 2; ++n)
@@ -297,7 +297,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(dtc::kThreads, 1)
       return true;
     };
     while (ok && pi.next(v, x0, x1)) {
-      if (!mbar_wait(smem_u32(&q_full), piece & 1, abort_p)) { ok = false; break; }
+      if (!mbar_wait(smem_u32(&q_full), piece & 1, abort_p, 6, piece)) { ok = false; break; }
       tc_fence_after();
       for (int x = x0; x < x1 && ok; ++x, ++j) {
         // QK(j) into S[j & 1]
@@ -344,7 +344,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(dtc::kThreads, 1)
       float m = -INFINITY, l = 0.f;
       bool o_started = false;
       for (int x = x0; x < x1; ++x, ++j) {
-        bool fail = !mbar_wait(smem_u32(&s_full[j & 1]), (j >> 1) & 1, abort_p);
+        bool fail = !mbar_wait(smem_u32(&s_full[j & 1]), (j >> 1) & 1, abort_p, 7, j);
         if (named_bar_or(1, 128, fail || *abort_p)) { dead = true; break; }
         tc_fence_after();
         uint32_t s_raw[64];
@@ -373,7 +373,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(dtc::kThreads, 1)
           const float alpha = (m == -INFINITY) ? 0.f : exp2f(m - m_blk);
           if (o_started) {
             // O holds PV up to block j-1: wait for it, then rescale in TMEM
-            if (mbar_wait(smem_u32(&pv_done[(j - 1) & 1]), ((j - 1) >> 1) & 1, abort_p)) {
+            if (mbar_wait(smem_u32(&pv_done[(j - 1) & 1]), ((j - 1) >> 1) & 1, abort_p, 8, j)) {
               tc_fence_after();
               for (int n = 0; n < 2; ++n)
                 for (int cc = 0; cc < 4; ++cc) {
@@ -393,7 +393,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(dtc::kThreads, 1)
           m = m_blk;
         }
         // P buffer (j & 1) was last read by PV(j - 2)
-        if (j >= 2) mbar_wait(smem_u32(&pv_done[j & 1]), ((j - 2) >> 1) & 1, abort_p);
+        if (j >= 2) mbar_wait(smem_u32(&pv_done[j & 1]), ((j - 2) >> 1) & 1, abort_p, 9, j);
         float lsum = 0.f;
         const uint32_t prow = sP + (j & 1) * kPBytes + half * 8192 + h * 128;
 #pragma unroll
@@ -424,7 +424,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(dtc::kThreads, 1)
       if (dead) break;
       // ---------------- epilogue of the piece ----------------
       const int jl = j - 1;
-      bool fail = !mbar_wait(smem_u32(&pv_done[jl & 1]), (jl >> 1) & 1, abort_p);
+      bool fail = !mbar_wait(smem_u32(&pv_done[jl & 1]), (jl >> 1) & 1, abort_p, 10, jl);
       if (named_bar_or(1, 128, fail || *abort_p)) { dead = true; break; }
       tc_fence_after();
       red_sum[half][h] = l;

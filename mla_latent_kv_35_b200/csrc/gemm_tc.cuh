@@ -93,7 +93,7 @@ __global__ void __launch_bounds__(128, 1) gemm_tc_kernel(const __grid_constant__
     int issued = 0;
     for (int i = 0; i < nk; ++i) {
       const int s = i % S;
-      if (!mbar_wait(smem_u32(&empty_bar[s]), ((i / S) & 1) ^ 1, abort_p)) break;
+      if (!mbar_wait(smem_u32(&empty_bar[s]), ((i / S) & 1) ^ 1, abort_p, 21, i)) break;
       const uint32_t fb = smem_u32(&full_bar[s]);
       const uint32_t sa = smem_base + s * stage_bytes;
       mbar_expect_tx(fb, stage_bytes);
@@ -118,7 +118,7 @@ __global__ void __launch_bounds__(128, 1) gemm_tc_kernel(const __grid_constant__
     bool ok = true;
     for (int i = 0; i < nk; ++i) {
       const int s = i % S;
-      if (!mbar_wait(smem_u32(&full_bar[s]), (i / S) & 1, abort_p)) { ok = false; break; }
+      if (!mbar_wait(smem_u32(&full_bar[s]), (i / S) & 1, abort_p, 22, i)) { ok = false; break; }
       tc_fence_after();
       const uint32_t sa = smem_base + s * stage_bytes;
       const uint32_t sx = sa + a_bytes;
@@ -139,7 +139,7 @@ __global__ void __launch_bounds__(128, 1) gemm_tc_kernel(const __grid_constant__
   __syncwarp();
 
   // ---------------- epilogue: all 4 warps ----------------
-  bool have = nk > 0 && mbar_wait(smem_u32(&acc_bar), 0, abort_p);
+  bool have = nk > 0 && mbar_wait(smem_u32(&acc_bar), 0, abort_p, 23, 0);
   if (have) {
     tc_fence_after();
     const int m = m0 + warp * 32 + lane;
