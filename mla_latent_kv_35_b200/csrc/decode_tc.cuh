@@ -272,6 +272,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(dtc::kThreads, 1)
       s = it % kStages;
       if (!mbar_wait(smem_u32(&full_bar[s]), (it / kStages) & 1, abort_p, 3, it)) return false;
       tc_fence_after();
+      ++it;
       return true;
     };
     auto issue_pv = [&](int jb, bool first, int pc) -> bool {
