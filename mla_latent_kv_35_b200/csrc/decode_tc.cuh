@@ -370,26 +370,33 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(dtc::kThreads, 1)
         named_bar_sync(1, 128);
         mx = fmaxf(mx, red_max[j & 1][half ^ 1][h]);
         const float m_blk = mx * P.scale_log2;
-        if (m_blk > m + kRescaleLog2 || (m == -INFINITY && m_blk > -INFINITY)) {
-          const float alpha = (m == -INFINITY) ? 0.f : exp2f(m - m_blk);
-          if (o_started) {
-            // O holds PV up to block j-1: wait for it, then rescale in TMEM
-            if (mbar_wait(smem_u32(&pv_done[(j - 1) & 1]), ((j - 1) >> 1) & 1, abort_p, 8, j)) {
-              tc_fence_after();
-              for (int n = 0; n < 2; ++n)
-                for (int cc = 0; cc < 4; ++cc) {
-                  uint32_t r[32];
-                  const uint32_t oa = tmem + lane_addr + kTmemO + 128 * n + 32 * cc;
-                  tmem_ld32(oa, r);
-                  tmem_wait_ld();
+        // Lazy rescale: a row moves its running max only when the block max
+        // exceeds it by more than 2^kRescaleLog2.  The decision is per row,
+        // but TMEM loads/stores are warp-collective, so a warp rescales when
+        // any of its rows needs it, with alpha = 1 for the other rows.
+        const bool need = m_blk > m + kRescaleLog2 || (m == -INFINITY && m_blk > -INFINITY);
+        const float alpha = !need ? 1.f : (m == -INFINITY ? 0.f : exp2f(m - m_blk));
+        if (o_started && __any_sync(0xffffffffu, need)) {
+          // O holds PV up to block j-1: wait for it, then rescale in TMEM
+          const bool ok = mbar_wait(smem_u32(&pv_done[(j - 1) & 1]), ((j - 1) >> 1) & 1,
+                                    abort_p, 8, j);
+          if (__all_sync(0xffffffffu, ok)) {
+            tc_fence_after();
+            for (int n = 0; n < 2; ++n)
+              for (int cc = 0; cc < 4; ++cc) {
+                uint32_t r[32];
+                const uint32_t oa = tmem + lane_addr + kTmemO + 128 * n + 32 * cc;
+                tmem_ld32(oa, r);
+                tmem_wait_ld();
 #pragma unroll
-                  for (int i = 0; i < 32; ++i)
-                    r[i] = __float_as_uint(__uint_as_float(r[i]) * alpha);
-                  tmem_st32(oa, r);
-                }
-              tmem_wait_st();
-            }
+                for (int i = 0; i < 32; ++i)
+                  r[i] = __float_as_uint(__uint_as_float(r[i]) * alpha);
+                tmem_st32(oa, r);
+              }
+            tmem_wait_st();
           }
+        }
+        if (need) {
           l *= alpha;
           m = m_blk;
         }

@@ -139,7 +139,9 @@ __global__ void __launch_bounds__(128, 1) gemm_tc_kernel(const __grid_constant__
   __syncwarp();
 
   // ---------------- epilogue: all 4 warps ----------------
-  bool have = nk > 0 && mbar_wait(smem_u32(&acc_bar), 0, abort_p, 23, 0);
+  // TMEM loads are warp-collective: every thread takes the same branch
+  const bool have =
+      __syncthreads_and(nk > 0 && mbar_wait(smem_u32(&acc_bar), 0, abort_p, 23, 0)) != 0;
   if (have) {
     tc_fence_after();
     const int m = m0 + warp * 32 + lane;
