@@ -276,12 +276,18 @@ def test_decode_split_invariance(peaky):
     base_o, base_l = _run_decode(d, c, 1, workers=1)
     for b in range(3):
         ref = _decode_ref(d, c, b)
-        check(base_o[b], ref["o_lat"], "bf16", f"workers=1 b={b}")
+        # P is rounded to bf16 (2^-9 relative) before PV, so the absolute error
+        # bound scales with the output magnitude; the planted needle makes
+        # outputs O(10) in the peaky variant
+        mag = max(1.0, float(np.abs(ref["o_lat"]).max()))
+        check(base_o[b], ref["o_lat"], "bf16", f"workers=1 b={b}",
+              tol=dict(max_abs=2e-2 * mag, mean_abs=2e-3 * mag))
         check(base_l[b], ref["lse"], "bf16", f"lse workers=1 b={b}")
+    mag = max(1.0, float(np.abs(base_o).max()))
     for workers in (2, 7, 300, 0):
         o, l = _run_decode(d, c, 1, workers=workers)
-        check(o, base_o, "bf16", f"workers={workers}", tol=dict(max_abs=2e-3, mean_abs=1e-4,
-                                                               rel_l2=2e-3))
+        check(o, base_o, "bf16", f"workers={workers}",
+              tol=dict(max_abs=4e-3 * mag, mean_abs=2e-4 * mag, rel_l2=2e-3))
         check(l, base_l, "bf16", f"lse workers={workers}", tol=dict(max_abs=1e-3))
 
 
