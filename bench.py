@@ -381,11 +381,17 @@ def main():
     ap.add_argument("--workload", default="batch128")
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--batch", type=int, default=0,
+                    help="use only the first N sequences of the workload")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
     from mla_latent_kv_35_b200 import workloads as wl
     w = wl.workload(args.workload)
+    if args.batch:
+        # same shapes with fewer sequences (small profiling case)
+        from dataclasses import replace
+        w = replace(w, B=args.batch, ctx=w.ctx[:args.batch], name=f"{w.name}[B={args.batch}]")
     if args.impl == "reference":
         run_reference(args, w)
     else:
