@@ -153,6 +153,34 @@ mla_status mla_decode(const mla_dims* dims, const void* qbuf, const void* pool,
                       void* workspace, size_t ws_bytes, float* o_lat,
                       float* lse, void* stream);
 
+/* A4 + A5 without caller-provided scratch.  The pages have no counterpart
+ * for this call; it exists for callers that cannot allocate device memory:
+ * code running under a host framework that owns every byte of device memory
+ * through its own allocator (so a library must not allocate behind its
+ * back), or latency-critical loops where cudaMalloc/cudaFree, which can
+ * synchronise the device, are not allowed.
+ *
+ * Same arguments and results as mla_decode minus workspace/ws_bytes.  The
+ * workspace lives in a fixed 64 MiB array in the library's device memory
+ * (MLA_NOALLOC_SCRATCH_BYTES), which every GPU that loads the library holds
+ * until the process exits.  A call whose mla_decode_workspace_size(dims, B,
+ * S_q, num_workers) exceeds it returns MLA_ERR_UNSUPPORTED before launching
+ * anything (the tensor-core path needs about 257 KiB per (worker + 128 query
+ * rows of one sequence), e.g. 53 MiB for 128 sequences with the default 74
+ * workers).  The first call on each device looks up the array's device
+ * address (cudaGetSymbolAddress) with that device current; make that first
+ * call before any stream capture.  Nothing in the array needs to start at
+ * zero; it keeps the last call's contents.  All calls on a device share the
+ * one array, so calls whose kernels overlap on the GPU (different streams
+ * without ordering) race on it.  The call itself allocates nothing. */
+#define MLA_NOALLOC_SCRATCH_BYTES (64u << 20)
+mla_status mla_decode_noalloc(const mla_dims* dims, const void* qbuf,
+                              const void* pool, int n_pages,
+                              const int32_t* page_table, int max_pages,
+                              const int32_t* seq_lens, int B, int S_q,
+                              int num_workers, float* o_lat, float* lse,
+                              void* stream);
+
 /* Scratch bytes mla_out_proj needs for T tokens. */
 size_t mla_out_proj_scratch_size(const mla_dims* dims, int T);
 

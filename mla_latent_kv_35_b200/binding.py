@@ -25,7 +25,8 @@ STATUS = {0: "MLA_OK", 1: "MLA_ERR_INVALID_ARG", 2: "MLA_ERR_UNSUPPORTED",
 EXPORTS = ("mla_project", "mla_absorb_q", "mla_rope", "mla_cache_append",
            "mla_decode_workspace_size", "mla_decode", "mla_out_proj_scratch_size",
            "mla_out_proj", "mla_get_device_status", "mla_status_string",
-           "mla_launch_count", "mla_selftest_wait_timeout", "mla_get_wait_diag")
+           "mla_launch_count", "mla_selftest_wait_timeout", "mla_get_wait_diag",
+           "mla_decode_noalloc")
 
 
 class MLAError(RuntimeError):
@@ -90,6 +91,8 @@ _SIGS = {
     "mla_launch_count": ([], ctypes.c_uint64),
     "mla_selftest_wait_timeout": ([ctypes.c_ulonglong, _P], _I),
     "mla_get_wait_diag": ([ctypes.POINTER(ctypes.c_uint32)], _I),
+    "mla_decode_noalloc": ([ctypes.POINTER(Dims), _P, _P, _I, _P, _I, _P, _I, _I, _I, _P, _P,
+                            _P], _I),
 }
 
 
@@ -171,6 +174,20 @@ def mla_decode(dims: MLADims, qbuf, pool, n_pages, page_table, max_pages, seq_le
         ctypes.byref(dims.c()), _ptr(qbuf), _ptr(pool), n_pages, _ptr(page_table), max_pages,
         _ptr(seq_lens), B, S_q, num_workers, _ptr(workspace), ws_bytes, _ptr(o_lat), _ptr(lse),
         _stream()))
+
+
+NOALLOC_SCRATCH_BYTES = 64 << 20
+
+
+def mla_decode_noalloc(dims: MLADims, qbuf, pool, n_pages, page_table, max_pages, seq_lens,
+                       B, S_q, num_workers, o_lat, lse):
+    """mla_decode with the library's built-in scratch instead of a workspace
+    (for callers that cannot allocate device memory; calls share the scratch
+    and must not overlap on the GPU)."""
+    _dev(qbuf, pool, page_table, seq_lens, o_lat, lse)
+    _check("mla_decode_noalloc", lib().mla_decode_noalloc(
+        ctypes.byref(dims.c()), _ptr(qbuf), _ptr(pool), n_pages, _ptr(page_table), max_pages,
+        _ptr(seq_lens), B, S_q, num_workers, _ptr(o_lat), _ptr(lse), _stream()))
 
 
 def mla_out_proj_scratch_size(dims: MLADims, T: int) -> int:

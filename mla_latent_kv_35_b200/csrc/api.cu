@@ -457,3 +457,53 @@ mla_status mla_out_proj(const mla_dims* dims, const float* o_lat, const void* w_
 }
 
 }  // extern "C"
+
+// ===========================================================================
+// Allocation-free decode: the workspace is a fixed array in this library's
+// device memory instead of caller-provided scratch (see mla_decode_noalloc in
+// include/mla.h for who needs this and the sharing rules).
+// ===========================================================================
+static __device__ __align__(256) unsigned char g_noalloc_scratch[MLA_NOALLOC_SCRATCH_BYTES];
+
+namespace {
+
+constexpr int kMaxDevices = 64;
+std::mutex g_noalloc_mu;
+void* g_noalloc_addr[kMaxDevices] = {};
+
+// Device address of g_noalloc_scratch on the current device.  In host code
+// the array's name only stands in for the symbol, so the address is looked
+// up once per device (with that device current) and cached.
+mla_status noalloc_scratch_address(void** out) {
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess) return MLA_ERR_CUDA;
+  if (dev < 0 || dev >= kMaxDevices) return MLA_ERR_UNSUPPORTED;
+  std::lock_guard<std::mutex> lock(g_noalloc_mu);
+  if (g_noalloc_addr[dev] == nullptr) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || p == nullptr)
+      return MLA_ERR_CUDA;
+    g_noalloc_addr[dev] = p;
+  }
+  *out = g_noalloc_addr[dev];
+  return MLA_OK;
+}
+
+}  // namespace
+
+extern "C" mla_status mla_decode_noalloc(const mla_dims* dims, const void* qbuf,
+                                         const void* pool, int n_pages,
+                                         const int32_t* page_table, int max_pages,
+                                         const int32_t* seq_lens, int B, int S_q,
+                                         int num_workers, float* o_lat, float* lse,
+                                         void* stream) {
+  if (!dims_ok(dims) || B < 0 || S_q < 1 || S_q > 2 || num_workers < 0)
+    return MLA_ERR_INVALID_ARG;
+  if (B == 0) return MLA_OK;
+  const size_t need = mla_decode_workspace_size(dims, B, S_q, num_workers);
+  if (need == 0 || need > (size_t)MLA_NOALLOC_SCRATCH_BYTES) return MLA_ERR_UNSUPPORTED;
+  void* ws = nullptr;
+  MLA_TRY(noalloc_scratch_address(&ws));
+  return mla_decode(dims, qbuf, pool, n_pages, page_table, max_pages, seq_lens, B, S_q,
+                    num_workers, ws, (size_t)MLA_NOALLOC_SCRATCH_BYTES, o_lat, lse, stream);
+}
