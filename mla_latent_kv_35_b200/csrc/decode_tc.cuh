@@ -5,15 +5,15 @@
 // keys and values" and "The bottleneck at inference time"): with W_UK folded
 // into the query, every head's score against cached token t is
 // q_abs . [c_t ; k_rope_t] over the 576 cached numbers, and the latent output
-// is sum_t softmax(s)_t c_t.  The cache row is read once and serves both as
-// the key (all 576 columns) and as the value (the first 512).
+// is sum_t softmax(s)_t c_t.  The cache row serves both as the key (all 576
+// columns) and as the value (the first 512).
 //
 // Work decomposition
 //   * A cluster of two CTAs (one per SM of a TPC) owns 128 query rows
 //     (S_q*H rows of one sequence, 128 at a time) and a contiguous run of
 //     128-token blocks.  CTA r holds rows [64r, 64r+64): its Q slice (72 KB)
 //     stays in shared memory for the whole piece.
-//   * QK: one pair MMA (cta_group::2, M = 128 rows, N = 128 tokens, K = 576).
+//   * QK: pair MMAs (cta_group::2, M = 128 rows, N = 128 tokens, K = 576).
 //     CTA r supplies the B half of page r of the block.  Each SM gets its 64
 //     rows x 128 tokens in TMEM folded onto 128 lanes x 64 columns: lane l<64
 //     holds row l, tokens 0..63; lane l>=64 holds row l-64, tokens 64..127.
@@ -22,6 +22,9 @@
 //     [256n + 128r, +128) of all 128 tokens (MN-major B read straight from
 //     the cache tile) and its own 64 rows of P (bf16, K-major).  O therefore
 //     takes 256 TMEM columns per SM; S is double buffered in 2 x 64 more.
+//   * QK tiles and PV tiles travel through two separate TMA rings with their
+//     own producer warps, so PV tiles waiting for P never hold back the QK
+//     loads of later blocks.
 //   * Each 128-thread softmax warpgroup reads its SM's S, exchanges row
 //     maxima between the two lanes that share a row, keeps a lazily rescaled
 //     running max (O is only rescaled in TMEM when the max grows by more than
@@ -52,14 +55,16 @@ constexpr int kDC = 512;           // latent width
 constexpr int kD = 576;            // cached numbers per token
 constexpr int kPage = 64;          // tokens per page
 constexpr int kBlk = 128;          // tokens per block (two pages)
-constexpr int kStages = 7;         // ring stages of 16 KB
-constexpr int kStageBytes = 16384;
-constexpr int kQBytes = 9 * 8192;  // 64 rows x 576 cols bf16
-constexpr int kPBytes = 16384;     // 64 rows x 128 tokens bf16
+constexpr int kQkStages = 9;       // QK ring: one 64-token x 64-column chunk each
+constexpr int kPvStages = 4;       // PV ring: two such chunks (128 latent columns)
+constexpr int kChunk = 8192;
+constexpr int kQBytes = 9 * kChunk;  // 64 rows x 576 cols bf16
+constexpr int kPBytes = 2 * kChunk;  // 64 rows x 128 tokens bf16
 constexpr uint32_t kOffQ = 0;
 constexpr uint32_t kOffP = kOffQ + kQBytes;
-constexpr uint32_t kOffRing = kOffP + 2 * kPBytes;
-constexpr uint32_t kSmemBytes = kOffRing + kStages * kStageBytes + 1024;  // + alignment
+constexpr uint32_t kOffQk = kOffP + kPBytes;
+constexpr uint32_t kOffPv = kOffQk + kQkStages * kChunk;
+constexpr uint32_t kSmemBytes = kOffPv + kPvStages * 2 * kChunk + 1024;  // + alignment
 constexpr int kThreads = 256;
 constexpr int kSoftmaxWarp0 = 4;
 constexpr uint32_t kTmemCols = 512;
@@ -122,19 +127,20 @@ struct PieceIter {
   }
 };
 
-// Page of token block x, half p (0/1) of sequence b: returns the pool page
-// (or -1 when the page lies past the context) and the slot shift for a
-// partial page (rows before it load as zeros).
+// Page of token block x, half p (0/1) of sequence b: the pool page and the
+// first slot to load.  A partial page starts at a negative slot (the rows
+// before the page load as zeros); a page past the context, or a page id
+// outside the pool (raising MLA_ERR_BOUNDS), loads entirely out of bounds.
 __device__ __forceinline__ void page_of(const DecodeTcParams& P, int b, int L, int x, int p,
                                         int& page, int& slot0) {
   const int first = x * dtc::kBlk + p * dtc::kPage;
   const int valid = min(L - first, dtc::kPage);
   if (valid <= 0) {
     page = 0;
-    slot0 = dtc::kPage;  // entirely out of bounds -> zeros
+    slot0 = dtc::kPage;
     return;
   }
-  int pg = P.page_table[(long long)b * P.max_pages + first / dtc::kPage];
+  const int pg = P.page_table[(long long)b * P.max_pages + first / dtc::kPage];
   if (pg < 0 || pg >= P.n_pages) {
     raise_flag(kFlagBounds);
     page = 0;
@@ -142,7 +148,7 @@ __device__ __forceinline__ void page_of(const DecodeTcParams& P, int b, int L, i
     return;
   }
   page = pg;
-  slot0 = valid - dtc::kPage;  // 0 for a full page, negative for a partial one
+  slot0 = valid - dtc::kPage;
 }
 
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(dtc::kThreads, 1)
@@ -150,10 +156,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(dtc::kThreads, 1)
                      const __grid_constant__ CUtensorMap tmKV, const DecodeTcParams P) {
   using namespace dtc;
   extern __shared__ uint8_t smem_raw[];
-  __shared__ __align__(8) uint64_t full_bar[kStages];
-  __shared__ __align__(8) uint64_t empty_bar[kStages];
-  __shared__ __align__(8) uint64_t q_full, q_empty, o_empty;
-  __shared__ __align__(8) uint64_t s_full[2], p_full[2], pv_done[2];
+  __shared__ __align__(8) uint64_t qk_full[kQkStages], qk_empty[kQkStages];
+  __shared__ __align__(8) uint64_t pv_full[kPvStages], pv_empty[kPvStages];
+  __shared__ __align__(8) uint64_t q_full, q_empty, o_empty, p_full, pv_done;
+  __shared__ __align__(8) uint64_t s_full[2];
   __shared__ float red_max[2][2][64];
   __shared__ float red_sum[2][64];
   __shared__ uint32_t tmem_base_sh;
@@ -163,22 +169,28 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(dtc::kThreads, 1)
   const uint32_t rank = cluster_ctarank();
   const int worker = blockIdx.x >> 1;
   const uint32_t base = (smem_u32(smem_raw) + 1023u) & ~1023u;
-  const uint32_t sQ = base + kOffQ, sP = base + kOffP, sRing = base + kOffRing;
+  const uint32_t sQ = base + kOffQ, sP = base + kOffP;
+  const uint32_t sQk = base + kOffQk, sPv = base + kOffPv;
 
   if (threadIdx.x == 0) {
     abort_flag = 0;
-    for (int s = 0; s < kStages; ++s) {
-      mbar_init(smem_u32(&full_bar[s]), 2);
-      mbar_init(smem_u32(&empty_bar[s]), 1);
+    for (int s = 0; s < kQkStages; ++s) {
+      // full barriers: the leader's producer arrives once with the bytes of
+      // both CTAs; the peer's copies only complete transactions on it
+      mbar_init(smem_u32(&qk_full[s]), 1);
+      mbar_init(smem_u32(&qk_empty[s]), 1);  // MMA commit (multicast)
     }
-    mbar_init(smem_u32(&q_full), 2);
+    for (int s = 0; s < kPvStages; ++s) {
+      mbar_init(smem_u32(&pv_full[s]), 1);
+      mbar_init(smem_u32(&pv_empty[s]), 1);
+    }
+    mbar_init(smem_u32(&q_full), 1);
     mbar_init(smem_u32(&q_empty), 1);
-    mbar_init(smem_u32(&o_empty), 8);
-    for (int b = 0; b < 2; ++b) {
-      mbar_init(smem_u32(&s_full[b]), 1);
-      mbar_init(smem_u32(&p_full[b]), 8);
-      mbar_init(smem_u32(&pv_done[b]), 1);
-    }
+    mbar_init(smem_u32(&o_empty), 8);        // 4 softmax warps x 2 CTAs
+    mbar_init(smem_u32(&p_full), 8);
+    mbar_init(smem_u32(&pv_done), 1);
+    mbar_init(smem_u32(&s_full[0]), 1);
+    mbar_init(smem_u32(&s_full[1]), 1);
     fence_mbar_init();
     tma_prefetch_desc(&tmQ);
     tma_prefetch_desc(&tmKV);
@@ -200,101 +212,117 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(dtc::kThreads, 1)
   const int rows_seq = P.S_q * P.H;
 
   if (warp == 0 && lane == 0) {
-    // =====================  TMA producer (both CTAs)  =====================
-    const uint32_t leader_full0 = mapa_shared(smem_u32(&full_bar[0]), 0);
-    const uint32_t leader_qfull = mapa_shared(smem_u32(&q_full), 0);
-    uint32_t it = 0;  // ring position
+    // =================  QK producer: Q slices and QK chunks  =================
+    const uint32_t lead_full0 = mapa_shared(smem_u32(&qk_full[0]), 0);
+    const uint32_t lead_qfull = mapa_shared(smem_u32(&q_full), 0);
+    uint32_t it = 0;
     PieceIter pi;
     pi.init(P.start, V, lo, hi);
     int v, x0, x1, piece = 0;
     bool ok = true;
-    // schedule: per block j: QK(j) stages; PV(j-1) stages after QK(j)
-    int pv_pend_b = -1, pv_pend_L = 0, pv_pend_x = 0;  // pending PV block
-    auto load_stage = [&](int page, int slot0, int cc0, int nchunks) -> bool {
-      const int s = it % kStages;
-      if (!mbar_wait(smem_u32(&empty_bar[s]), ((it / kStages) & 1) ^ 1, abort_p, 1, it)) return false;
-      const uint32_t fb = leader_full0 + s * 8;
-      mbar_expect_tx_cluster(fb, nchunks * 8192);
-      const uint32_t dst = sRing + s * kStageBytes;
-      for (int c = 0; c < nchunks; ++c)
-        tma_load_3d_pair(dst + c * 8192, &tmKV, (cc0 + c) * 64, slot0, page, fb);
-      ++it;
-      return true;
-    };
-    auto load_pv = [&](int b, int L, int x) -> bool {
-      for (int n = 0; n < 2; ++n)
-        for (int p = 0; p < 2; ++p) {
-          int page, slot0;
-          page_of(P, b, L, x, p, page, slot0);
-          if (!load_stage(page, slot0, 4 * n + 2 * (int)rank, 2)) return false;
-        }
-      return true;
-    };
     while (ok && pi.next(v, x0, x1)) {
       const int b = v / P.R, rb = v % P.R;
       const int L = P.seq_lens[b];
-      // Q slice of this piece (needs the previous piece's QK MMAs finished)
-      if (piece > 0 && !mbar_wait(smem_u32(&q_empty), (piece - 1) & 1, abort_p, 2, piece)) { ok = false; break; }
-      mbar_expect_tx_cluster(leader_qfull, kQBytes);
+      // the Q slice is free once the previous piece's QK MMAs completed
+      if (piece > 0 && !mbar_wait(smem_u32(&q_empty), (piece - 1) & 1, abort_p, 2, piece)) {
+        ok = false;
+        break;
+      }
+      if (rank == 0) mbar_expect_tx(smem_u32(&q_full), 2 * kQBytes);
       const int row0 = b * rows_seq + rb * 128 + 64 * (int)rank;
-      for (int c = 0; c < 9; ++c) tma_load_2d_pair(sQ + c * 8192, &tmQ, c * 64, row0, leader_qfull);
+      for (int c = 0; c < 9; ++c)
+        tma_load_2d_pair(sQ + c * kChunk, &tmQ, c * 64, row0, lead_qfull);
       for (int x = x0; x < x1 && ok; ++x) {
         int page, slot0;
         page_of(P, b, L, x, (int)rank, page, slot0);
-        for (int c = 0; c < 4 && ok; ++c) ok = load_stage(page, slot0, 2 * c, 2);
-        if (ok) ok = load_stage(page, slot0, 8, 1);
-        if (ok && pv_pend_b >= 0) ok = load_pv(pv_pend_b, pv_pend_L, pv_pend_x);
-        pv_pend_b = b; pv_pend_L = L; pv_pend_x = x;
+        for (int c = 0; c < 9; ++c, ++it) {
+          const int s = it % kQkStages;
+          if (!mbar_wait(smem_u32(&qk_empty[s]), ((it / kQkStages) & 1) ^ 1, abort_p, 1, it)) {
+            ok = false;
+            break;
+          }
+          const uint32_t fb = lead_full0 + s * 8;
+          if (rank == 0) mbar_expect_tx(smem_u32(&qk_full[s]), 2 * kChunk);
+          tma_load_3d_pair(sQk + s * kChunk, &tmKV, c * 64, slot0, page, fb);
+        }
       }
       ++piece;
     }
-    if (ok && pv_pend_b >= 0) ok = load_pv(pv_pend_b, pv_pend_L, pv_pend_x);
     if (!ok) {
       // give copies already issued time to land before the CTA can exit
       const uint64_t t0 = globaltimer();
       while (globaltimer() - t0 < 50000ull) {
       }
     }
+  } else if (warp == 2 && lane == 0) {
+    // =================  PV producer: this CTA's latent half of both pages  =====
+    const uint32_t lead_full0 = mapa_shared(smem_u32(&pv_full[0]), 0);
+    uint32_t it = 0;
+    PieceIter pi;
+    pi.init(P.start, V, lo, hi);
+    int v, x0, x1;
+    bool ok = true;
+    while (ok && pi.next(v, x0, x1)) {
+      const int b = v / P.R;
+      const int L = P.seq_lens[b];
+      for (int x = x0; x < x1 && ok; ++x)
+        for (int n = 0; n < 2 && ok; ++n)
+          for (int p = 0; p < 2; ++p, ++it) {
+            int page, slot0;
+            page_of(P, b, L, x, p, page, slot0);
+            const int s = it % kPvStages;
+            if (!mbar_wait(smem_u32(&pv_empty[s]), ((it / kPvStages) & 1) ^ 1, abort_p, 11, it)) {
+              ok = false;
+              break;
+            }
+            const uint32_t fb = lead_full0 + s * 8;
+            if (rank == 0) mbar_expect_tx(smem_u32(&pv_full[s]), 4 * kChunk);
+            const int cc = 4 * n + 2 * (int)rank;
+            const uint32_t dst = sPv + s * 2 * kChunk;
+            tma_load_3d_pair(dst, &tmKV, cc * 64, slot0, page, fb);
+            tma_load_3d_pair(dst + kChunk, &tmKV, (cc + 1) * 64, slot0, page, fb);
+          }
+    }
+    if (!ok) {
+      const uint64_t t0 = globaltimer();
+      while (globaltimer() - t0 < 50000ull) {
+      }
+    }
   } else if (warp == 1 && lane == 0 && rank == 0) {
-    // =====================  MMA issuer (leader CTA)  =====================
+    // =================  MMA issuer (leader CTA)  =================
     const uint32_t idesc_qk = idesc_bf16_f32(128, 128, false, false);
     const uint32_t idesc_pv = idesc_bf16_f32(128, 256, false, true);
-    uint32_t it = 0;
-    int j = 0;  // global block counter of this worker
+    uint32_t itq = 0, itv = 0;
+    int j = 0;  // block counter of this worker
     PieceIter pi;
     pi.init(P.start, V, lo, hi);
     int v, x0, x1, piece = 0;
     bool ok = true;
-    int pend = -1;            // global index of the block whose PV is pending
-    bool pend_first = false;  // that block is the first of its piece
+    int pend = -1;            // block whose PV is pending
+    bool pend_first = false;  // ... is the first block of its piece
     int pend_piece = 0;
-    auto consume = [&](int& s) -> bool {
-      s = it % kStages;
-      if (!mbar_wait(smem_u32(&full_bar[s]), (it / kStages) & 1, abort_p, 3, it)) return false;
-      tc_fence_after();
-      ++it;
-      return true;
-    };
     auto issue_pv = [&](int jb, bool first, int pc) -> bool {
-      if (!mbar_wait(smem_u32(&p_full[jb & 1]), (jb >> 1) & 1, abort_p, 4, jb)) return false;
-      if (first && pc > 0 && !mbar_wait(smem_u32(&o_empty), (pc - 1) & 1, abort_p, 5, pc)) return false;
+      if (!mbar_wait(smem_u32(&p_full), jb & 1, abort_p, 4, jb)) return false;
+      if (first && pc > 0 && !mbar_wait(smem_u32(&o_empty), (pc - 1) & 1, abort_p, 5, pc))
+        return false;
       tc_fence_after();
-      const uint32_t pbuf = sP + (jb & 1) * kPBytes;
       for (int n = 0; n < 2; ++n)
-        for (int p = 0; p < 2; ++p) {
-          int s;
-          if (!consume(s)) return false;
-          const uint32_t st = sRing + s * kStageBytes;
+        for (int p = 0; p < 2; ++p, ++itv) {
+          const int s = itv % kPvStages;
+          if (!mbar_wait(smem_u32(&pv_full[s]), (itv / kPvStages) & 1, abort_p, 12, itv))
+            return false;
+          tc_fence_after();
+          const uint32_t st = sPv + s * 2 * kChunk;
 #pragma unroll
           for (int kk = 0; kk < 4; ++kk) {
-            const uint64_t ad = sw128_desc(pbuf + p * 8192 + kk * 32, 16, 1024);
-            const uint64_t bd = sw128_desc(st + kk * 2048, 8192, 1024);
+            const uint64_t ad = sw128_desc(sP + p * kChunk + kk * 32, 16, 1024);
+            const uint64_t bd = sw128_desc(st + kk * 2048, kChunk, 1024);
             const uint32_t acc = (first && p == 0 && kk == 0) ? 0u : 1u;
             mma_bf16_ss<2>(tmem + kTmemO + 128 * n, ad, bd, idesc_pv, acc);
           }
-          mma_commit_2_mc(smem_u32(&empty_bar[s]), 3);
+          mma_commit_2_mc(smem_u32(&pv_empty[s]), 3);
         }
-      mma_commit_2_mc(smem_u32(&pv_done[jb & 1]), 3);
+      mma_commit_2_mc(smem_u32(&pv_done), 3);
       return true;
     };
     while (ok && pi.next(v, x0, x1)) {
@@ -303,18 +331,21 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(dtc::kThreads, 1)
       for (int x = x0; x < x1 && ok; ++x, ++j) {
         // QK(j) into S[j & 1]
         const uint32_t sd = tmem + kTmemS + 64 * (j & 1);
-        for (int c = 0; c < 5 && ok; ++c) {
-          int s;
-          if (!consume(s)) { ok = false; break; }
-          const uint32_t st = sRing + s * kStageBytes;
-          const int nk = (c < 4) ? 8 : 4;
-          for (int kk = 0; kk < nk; ++kk) {
-            const int col = c * 2 + kk / 4;  // 64-column chunk of the 576
-            const uint64_t ad = sw128_desc(sQ + col * 8192 + (kk & 3) * 32, 16, 1024);
-            const uint64_t bd = sw128_desc(st + (kk / 4) * 8192 + (kk & 3) * 32, 16, 1024);
+        for (int c = 0; c < 9; ++c, ++itq) {
+          const int s = itq % kQkStages;
+          if (!mbar_wait(smem_u32(&qk_full[s]), (itq / kQkStages) & 1, abort_p, 3, itq)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t st = sQk + s * kChunk;
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk) {
+            const uint64_t ad = sw128_desc(sQ + c * kChunk + kk * 32, 16, 1024);
+            const uint64_t bd = sw128_desc(st + kk * 32, 16, 1024);
             mma_bf16_ss<2>(sd, ad, bd, idesc_qk, (c | kk) ? 1u : 0u);
           }
-          mma_commit_2_mc(smem_u32(&empty_bar[s]), 3);
+          mma_commit_2_mc(smem_u32(&qk_empty[s]), 3);
         }
         if (!ok) break;
         mma_commit_2_mc(smem_u32(&s_full[j & 1]), 3);
@@ -326,12 +357,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(dtc::kThreads, 1)
     }
     if (ok && pend >= 0) issue_pv(pend, pend_first, pend_piece);
   } else if (warp >= kSoftmaxWarp0) {
-    // =====================  softmax + epilogue (both CTAs)  =====================
+    // =================  softmax + epilogue (both CTAs)  =================
     const int tid = threadIdx.x - kSoftmaxWarp0 * 32;  // = TMEM lane
     const int h = tid & 63, half = tid >> 6;
     const uint32_t lane_addr = (uint32_t)(32 * (warp - kSoftmaxWarp0)) << 16;
-    const uint32_t leader_pfull0 = mapa_shared(smem_u32(&p_full[0]), 0);
-    const uint32_t leader_oempty = mapa_shared(smem_u32(&o_empty), 0);
+    const uint32_t lead_pfull = mapa_shared(smem_u32(&p_full), 0);
+    const uint32_t lead_oempty = mapa_shared(smem_u32(&o_empty), 0);
+    const uint32_t prow = sP + half * kChunk + h * 128;
     PieceIter pi;
     pi.init(P.start, V, lo, hi);
     int v, x0, x1;
@@ -345,42 +377,58 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(dtc::kThreads, 1)
       float m = -INFINITY, l = 0.f;
       bool o_started = false;
       for (int x = x0; x < x1; ++x, ++j) {
-        bool fail = !mbar_wait(smem_u32(&s_full[j & 1]), (j >> 1) & 1, abort_p, 7, j);
-        if (named_bar_or(1, 128, fail || *abort_p)) { dead = true; break; }
-        tc_fence_after();
+        const bool got = mbar_wait(smem_u32(&s_full[j & 1]), (j >> 1) & 1, abort_p, 7, j);
         uint32_t s_raw[64];
-        {
-          uint32_t (&a)[32] = *reinterpret_cast<uint32_t(*)[32]>(&s_raw[0]);
-          uint32_t (&c)[32] = *reinterpret_cast<uint32_t(*)[32]>(&s_raw[32]);
-          const uint32_t sa = tmem + lane_addr + kTmemS + 64 * (j & 1);
-          tmem_ld32(sa, a);
-          tmem_ld32(sa + 32, c);
-          tmem_wait_ld();
-        }
+        float mx = -INFINITY;
         // token t of this lane's page: first + c - shift, valid if c >= shift
         const int first = x * kBlk + half * kPage;
         const int valid = min(L - first, kPage);
         const int shift = valid > 0 ? kPage - valid : kPage;
         const int cmax = limit - first + shift;  // columns c < cmax are visible
-        float mx = -INFINITY;
+        if (__all_sync(0xffffffffu, got)) {
+          tc_fence_after();
+          uint32_t (&a)[32] = *reinterpret_cast<uint32_t(*)[32]>(&s_raw[0]);
+          uint32_t (&c2)[32] = *reinterpret_cast<uint32_t(*)[32]>(&s_raw[32]);
+          const uint32_t sa = tmem + lane_addr + kTmemS + 64 * (j & 1);
+          tmem_ld32(sa, a);
+          tmem_ld32(sa + 32, c2);
+          tmem_wait_ld();
 #pragma unroll
-        for (int c = 0; c < 64; ++c)
-          if (c >= shift && c < cmax) mx = fmaxf(mx, __uint_as_float(s_raw[c]));
+          for (int c = 0; c < 64; ++c)
+            if (c >= shift && c < cmax) mx = fmaxf(mx, __uint_as_float(s_raw[c]));
+        }
         red_max[j & 1][half][h] = mx;
-        named_bar_sync(1, 128);
+        // one barrier: partner's max visible, and everyone agrees to go on
+        if (named_bar_or(1, 128, !got || *abort_p)) { dead = true; break; }
         mx = fmaxf(mx, red_max[j & 1][half ^ 1][h]);
         const float m_blk = mx * P.scale_log2;
         // Lazy rescale: a row moves its running max only when the block max
-        // exceeds it by more than 2^kRescaleLog2.  The decision is per row,
-        // but TMEM loads/stores are warp-collective, so a warp rescales when
-        // any of its rows needs it, with alpha = 1 for the other rows.
+        // exceeds it by more than 2^kRescaleLog2.  TMEM loads/stores are
+        // warp-collective, so a warp rescales when any of its rows needs it,
+        // with alpha = 1 for the other rows.
         const bool need = m_blk > m + kRescaleLog2 || (m == -INFINITY && m_blk > -INFINITY);
-        const float alpha = !need ? 1.f : (m == -INFINITY ? 0.f : exp2f(m - m_blk));
-        if (o_started && __any_sync(0xffffffffu, need)) {
-          // O holds PV up to block j-1: wait for it, then rescale in TMEM
-          const bool ok = mbar_wait(smem_u32(&pv_done[(j - 1) & 1]), ((j - 1) >> 1) & 1,
-                                    abort_p, 8, j);
-          if (__all_sync(0xffffffffu, ok)) {
+        const float alpha = !need ? 1.f : (m == -INFINITY ? 0.f : ex2_approx(m - m_blk));
+        const float m_use = need ? m_blk : m;
+        uint32_t pk[32];
+        float lsum = 0.f;
+#pragma unroll
+        for (int e = 0; e < 32; ++e) {
+          const int c0 = 2 * e;
+          const float p0 = (c0 >= shift && c0 < cmax)
+                               ? ex2_approx(fmaf(__uint_as_float(s_raw[c0]), P.scale_log2, -m_use))
+                               : 0.f;
+          const float p1 = (c0 + 1 >= shift && c0 + 1 < cmax)
+                               ? ex2_approx(fmaf(__uint_as_float(s_raw[c0 + 1]), P.scale_log2,
+                                                 -m_use))
+                               : 0.f;
+          lsum += p0 + p1;
+          pk[e] = pack_bf16x2(p0, p1);
+        }
+        // PV(j-1) must be done before P is overwritten and before O is rescaled
+        bool ok = true;
+        if (j > 0) ok = mbar_wait(smem_u32(&pv_done), (j - 1) & 1, abort_p, 8, j);
+        if (__all_sync(0xffffffffu, ok)) {
+          if (o_started && __any_sync(0xffffffffu, need)) {
             tc_fence_after();
             for (int n = 0; n < 2; ++n)
               for (int cc = 0; cc < 4; ++cc) {
@@ -395,50 +443,31 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(dtc::kThreads, 1)
               }
             tmem_wait_st();
           }
-        }
-        if (need) {
-          l *= alpha;
-          m = m_blk;
-        }
-        // P buffer (j & 1) was last read by PV(j - 2)
-        if (j >= 2) mbar_wait(smem_u32(&pv_done[j & 1]), ((j - 2) >> 1) & 1, abort_p, 9, j);
-        float lsum = 0.f;
-        const uint32_t prow = sP + (j & 1) * kPBytes + half * 8192 + h * 128;
 #pragma unroll
-        for (int u = 0; u < 8; ++u) {
-          uint32_t pk[4];
-#pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            const int c0 = u * 8 + e * 2;
-            float p0 = (c0 >= shift && c0 < cmax)
-                           ? exp2f(fmaf(__uint_as_float(s_raw[c0]), P.scale_log2, -m)) : 0.f;
-            float p1 = (c0 + 1 >= shift && c0 + 1 < cmax)
-                           ? exp2f(fmaf(__uint_as_float(s_raw[c0 + 1]), P.scale_log2, -m)) : 0.f;
-            lsum += p0 + p1;
-            pk[e] = pack_bf16x2(p0, p1);
+          for (int u = 0; u < 8; ++u) {
+            const uint32_t addr = prow + ((u ^ (h & 7)) << 4);
+            asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr),
+                         "r"(pk[4 * u]), "r"(pk[4 * u + 1]), "r"(pk[4 * u + 2]),
+                         "r"(pk[4 * u + 3])
+                         : "memory");
           }
-          const uint32_t addr = prow + ((u ^ (h & 7)) << 4);
-          asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(pk[0]),
-                       "r"(pk[1]), "r"(pk[2]), "r"(pk[3])
-                       : "memory");
         }
-        l += lsum;
+        l = need ? l * alpha + lsum : l + lsum;
+        m = m_use;
         fence_proxy_async_smem();
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive_cluster(leader_pfull0 + (j & 1) * 8);
+        if (lane == 0) mbar_arrive_cluster(lead_pfull);
         o_started = true;
       }
       if (dead) break;
       // ---------------- epilogue of the piece ----------------
       const int jl = j - 1;
-      bool fail = !mbar_wait(smem_u32(&pv_done[jl & 1]), (jl >> 1) & 1, abort_p, 10, jl);
-      if (named_bar_or(1, 128, fail || *abort_p)) { dead = true; break; }
-      tc_fence_after();
+      const bool got = mbar_wait(smem_u32(&pv_done), jl & 1, abort_p, 10, jl);
       red_sum[half][h] = l;
-      named_bar_sync(1, 128);
+      if (named_bar_or(1, 128, !got || *abort_p)) { dead = true; break; }
+      tc_fence_after();
       const float lt = l + red_sum[half ^ 1][h];
-      named_bar_sync(1, 128);  // red_sum reused by the next piece
       const float inv = lt > 0.f ? 1.f / lt : 0.f;
       const long long slot = (long long)worker + v;
       const long long row = slot * 128 + 64 * (int)rank + h;
@@ -457,9 +486,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(dtc::kThreads, 1)
         }
       if (half == 0)
         P.ws_lse[row] = lt > 0.f ? (m + log2f(lt)) * 0.69314718055994531f : -INFINITY;
+      named_bar_sync(1, 128);  // red_sum is rewritten by the next piece
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive_cluster(leader_oempty);
+      if (lane == 0) mbar_arrive_cluster(lead_oempty);
     }
   }
 
