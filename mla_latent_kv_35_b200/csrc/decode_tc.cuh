@@ -55,16 +55,19 @@ constexpr int kDC = 512;           // latent width
 constexpr int kD = 576;            // cached numbers per token
 constexpr int kPage = 64;          // tokens per page
 constexpr int kBlk = 128;          // tokens per block (two pages)
-constexpr int kQkStages = 9;       // QK ring: one 64-token x 64-column chunk each
-constexpr int kPvStages = 4;       // PV ring: two such chunks (128 latent columns)
-constexpr int kChunk = 8192;
+constexpr int kChunk = 8192;       // 64 tokens x 64 columns bf16, one swizzled operand tile
+constexpr int kQkChunks = 3;       // chunks per QK stage (one TMA box)
+constexpr int kQkStages = 3;       // QK ring: 3 stages x 3 chunks = one page per block
+constexpr int kQkStageBytes = kQkChunks * kChunk;
+constexpr int kPvStages = 2;       // PV ring: one page's latent half (4 chunks) per stage
+constexpr int kPvStageBytes = 4 * kChunk;
 constexpr int kQBytes = 9 * kChunk;  // 64 rows x 576 cols bf16
 constexpr int kPBytes = 2 * kChunk;  // 64 rows x 128 tokens bf16
 constexpr uint32_t kOffQ = 0;
 constexpr uint32_t kOffP = kOffQ + kQBytes;
 constexpr uint32_t kOffQk = kOffP + kPBytes;
-constexpr uint32_t kOffPv = kOffQk + kQkStages * kChunk;
-constexpr uint32_t kSmemBytes = kOffPv + kPvStages * 2 * kChunk + 1024;  // + alignment
+constexpr uint32_t kOffPv = kOffQk + kQkStages * kQkStageBytes;
+constexpr uint32_t kSmemBytes = kOffPv + kPvStages * kPvStageBytes + 1024;  // + alignment
 constexpr int kThreads = 256;
 constexpr int kSoftmaxWarp0 = 4;
 constexpr uint32_t kTmemCols = 512;
@@ -153,7 +156,8 @@ __device__ __forceinline__ void page_of(const DecodeTcParams& P, int b, int L, i
 
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(dtc::kThreads, 1)
     decode_tc_kernel(const __grid_constant__ CUtensorMap tmQ,
-                     const __grid_constant__ CUtensorMap tmKV, const DecodeTcParams P) {
+                     const __grid_constant__ CUtensorMap tmQK,
+                     const __grid_constant__ CUtensorMap tmPV, const DecodeTcParams P) {
   using namespace dtc;
   extern __shared__ uint8_t smem_raw[];
   __shared__ __align__(8) uint64_t qk_full[kQkStages], qk_empty[kQkStages];
@@ -193,7 +197,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(dtc::kThreads, 1)
     mbar_init(smem_u32(&s_full[1]), 1);
     fence_mbar_init();
     tma_prefetch_desc(&tmQ);
-    tma_prefetch_desc(&tmKV);
+    tma_prefetch_desc(&tmQK);
+    tma_prefetch_desc(&tmPV);
   }
   if (warp == 1) {
     tmem_alloc<2>(smem_u32(&tmem_base_sh), kTmemCols);
@@ -235,15 +240,16 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(dtc::kThreads, 1)
       for (int x = x0; x < x1 && ok; ++x) {
         int page, slot0;
         page_of(P, b, L, x, (int)rank, page, slot0);
-        for (int c = 0; c < 9; ++c, ++it) {
+        // one box = chunks [3k, 3k+3) of the page (64 slots x 64 columns each)
+        for (int k = 0; k < 9 / kQkChunks; ++k, ++it) {
           const int s = it % kQkStages;
           if (!mbar_wait(smem_u32(&qk_empty[s]), ((it / kQkStages) & 1) ^ 1, abort_p, 1, it)) {
             ok = false;
             break;
           }
           const uint32_t fb = lead_full0 + s * 8;
-          if (rank == 0) mbar_expect_tx(smem_u32(&qk_full[s]), 2 * kChunk);
-          tma_load_3d_pair(sQk + s * kChunk, &tmKV, c * 64, slot0, page, fb);
+          if (rank == 0) mbar_expect_tx(smem_u32(&qk_full[s]), 2 * kQkStageBytes);
+          tma_load_4d_pair(sQk + s * kQkStageBytes, &tmQK, 0, slot0, kQkChunks * k, page, fb);
         }
       }
       ++piece;
@@ -266,22 +272,20 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(dtc::kThreads, 1)
       const int b = v / P.R;
       const int L = P.seq_lens[b];
       for (int x = x0; x < x1 && ok; ++x)
-        for (int n = 0; n < 2 && ok; ++n)
-          for (int p = 0; p < 2; ++p, ++it) {
-            int page, slot0;
-            page_of(P, b, L, x, p, page, slot0);
-            const int s = it % kPvStages;
-            if (!mbar_wait(smem_u32(&pv_empty[s]), ((it / kPvStages) & 1) ^ 1, abort_p, 11, it)) {
-              ok = false;
-              break;
-            }
-            const uint32_t fb = lead_full0 + s * 8;
-            if (rank == 0) mbar_expect_tx(smem_u32(&pv_full[s]), 4 * kChunk);
-            const int cc = 4 * n + 2 * (int)rank;
-            const uint32_t dst = sPv + s * 2 * kChunk;
-            tma_load_3d_pair(dst, &tmKV, cc * 64, slot0, page, fb);
-            tma_load_3d_pair(dst + kChunk, &tmKV, (cc + 1) * 64, slot0, page, fb);
+        for (int p = 0; p < 2; ++p, ++it) {
+          int page, slot0;
+          page_of(P, b, L, x, p, page, slot0);
+          const int s = it % kPvStages;
+          if (!mbar_wait(smem_u32(&pv_empty[s]), ((it / kPvStages) & 1) ^ 1, abort_p, 11, it)) {
+            ok = false;
+            break;
           }
+          const uint32_t fb = lead_full0 + s * 8;
+          if (rank == 0) mbar_expect_tx(smem_u32(&pv_full[s]), 2 * kPvStageBytes);
+          // one box = latent chunks {4n + 2r, 4n + 2r + 1} for n = 0, 1 of page p,
+          // landing as [n][chunk][slot][64 columns]
+          tma_load_5d_pair(sPv + s * kPvStageBytes, &tmPV, 0, slot0, 2 * (int)rank, 0, page, fb);
+        }
     }
     if (!ok) {
       const uint64_t t0 = globaltimer();
@@ -306,22 +310,23 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(dtc::kThreads, 1)
       if (first && pc > 0 && !mbar_wait(smem_u32(&o_empty), (pc - 1) & 1, abort_p, 5, pc))
         return false;
       tc_fence_after();
-      for (int n = 0; n < 2; ++n)
-        for (int p = 0; p < 2; ++p, ++itv) {
-          const int s = itv % kPvStages;
-          if (!mbar_wait(smem_u32(&pv_full[s]), (itv / kPvStages) & 1, abort_p, 12, itv))
-            return false;
-          tc_fence_after();
-          const uint32_t st = sPv + s * 2 * kChunk;
+      for (int p = 0; p < 2; ++p, ++itv) {
+        const int s = itv % kPvStages;
+        if (!mbar_wait(smem_u32(&pv_full[s]), (itv / kPvStages) & 1, abort_p, 12, itv))
+          return false;
+        tc_fence_after();
+        const uint32_t st = sPv + s * kPvStageBytes;
+        for (int n = 0; n < 2; ++n) {
 #pragma unroll
           for (int kk = 0; kk < 4; ++kk) {
             const uint64_t ad = sw128_desc(sP + p * kChunk + kk * 32, 16, 1024);
-            const uint64_t bd = sw128_desc(st + kk * 2048, kChunk, 1024);
+            const uint64_t bd = sw128_desc(st + n * 2 * kChunk + kk * 2048, kChunk, 1024);
             const uint32_t acc = (first && p == 0 && kk == 0) ? 0u : 1u;
             mma_bf16_ss<2>(tmem + kTmemO + 128 * n, ad, bd, idesc_pv, acc);
           }
-          mma_commit_2_mc(smem_u32(&pv_empty[s]), 3);
         }
+        mma_commit_2_mc(smem_u32(&pv_empty[s]), 3);
+      }
       mma_commit_2_mc(smem_u32(&pv_done), 3);
       return true;
     };
@@ -331,19 +336,22 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(dtc::kThreads, 1)
       for (int x = x0; x < x1 && ok; ++x, ++j) {
         // QK(j) into S[j & 1]
         const uint32_t sd = tmem + kTmemS + 64 * (j & 1);
-        for (int c = 0; c < 9; ++c, ++itq) {
+        for (int k = 0; k < 9 / kQkChunks; ++k, ++itq) {
           const int s = itq % kQkStages;
           if (!mbar_wait(smem_u32(&qk_full[s]), (itq / kQkStages) & 1, abort_p, 3, itq)) {
             ok = false;
             break;
           }
           tc_fence_after();
-          const uint32_t st = sQk + s * kChunk;
+          const uint32_t st = sQk + s * kQkStageBytes;
+          for (int cc = 0; cc < kQkChunks; ++cc) {
+            const int c = kQkChunks * k + cc;  // 64-column chunk of the 576
 #pragma unroll
-          for (int kk = 0; kk < 4; ++kk) {
-            const uint64_t ad = sw128_desc(sQ + c * kChunk + kk * 32, 16, 1024);
-            const uint64_t bd = sw128_desc(st + kk * 32, 16, 1024);
-            mma_bf16_ss<2>(sd, ad, bd, idesc_qk, (c | kk) ? 1u : 0u);
+            for (int kk = 0; kk < 4; ++kk) {
+              const uint64_t ad = sw128_desc(sQ + c * kChunk + kk * 32, 16, 1024);
+              const uint64_t bd = sw128_desc(st + cc * kChunk + kk * 32, 16, 1024);
+              mma_bf16_ss<2>(sd, ad, bd, idesc_qk, (c | kk) ? 1u : 0u);
+            }
           }
           mma_commit_2_mc(smem_u32(&qk_empty[s]), 3);
         }
@@ -509,18 +517,27 @@ inline mla_status launch_decode_tc_impl(
     const int32_t* seq_lens, int B, int S_q, int H, float scale, int G, const int32_t* start,
     float* ws_lse, float* ws_o, cudaStream_t st) {
   using namespace dtc;
-  CUtensorMap tQ, tKV;
+  CUtensorMap tQ, tQK, tPV;
   {
     const uint64_t dims[2] = {(uint64_t)kD, (uint64_t)B * S_q * H};
     const uint64_t strides[1] = {(uint64_t)kD * 2};
     const uint32_t box[2] = {64, 64};
     if (!make_tmap(&tQ, qbuf, 2, dims, strides, box)) return MLA_ERR_CUDA;
   }
+  // The pool [n_pages][64 slots][576] seen as 64-column chunks: element
+  // (col, slot, chunk, page) at page*73728 + slot*1152 + chunk*128 + col*2 bytes.
   {
-    const uint64_t dims[3] = {(uint64_t)kD, (uint64_t)kPage, (uint64_t)n_pages};
-    const uint64_t strides[2] = {(uint64_t)kD * 2, (uint64_t)kD * 2 * kPage};
-    const uint32_t box[3] = {64, 64, 1};
-    if (!make_tmap(&tKV, pool, 3, dims, strides, box)) return MLA_ERR_CUDA;
+    const uint64_t dims[4] = {64, (uint64_t)kPage, 9, (uint64_t)n_pages};
+    const uint64_t strides[3] = {(uint64_t)kD * 2, 128, (uint64_t)kD * 2 * kPage};
+    const uint32_t box[4] = {64, 64, (uint32_t)kQkChunks, 1};
+    if (!make_tmap(&tQK, pool, 4, dims, strides, box)) return MLA_ERR_CUDA;
+  }
+  // Latent chunks grouped as (chunk-in-group 0..3, group n 0..1): chunk 4n + i.
+  {
+    const uint64_t dims[5] = {64, (uint64_t)kPage, 4, 2, (uint64_t)n_pages};
+    const uint64_t strides[4] = {(uint64_t)kD * 2, 128, 512, (uint64_t)kD * 2 * kPage};
+    const uint32_t box[5] = {64, 64, 2, 2, 1};
+    if (!make_tmap(&tPV, pool, 5, dims, strides, box)) return MLA_ERR_CUDA;
   }
   DecodeTcParams p;
   p.page_table = page_table;
@@ -539,7 +556,7 @@ inline mla_status launch_decode_tc_impl(
   if (cudaFuncSetAttribute(decode_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            (int)kSmemBytes) != cudaSuccess)
     return MLA_ERR_CUDA;
-  decode_tc_kernel<<<2 * G, kThreads, kSmemBytes, st>>>(tQ, tKV, p);
+  decode_tc_kernel<<<2 * G, kThreads, kSmemBytes, st>>>(tQ, tQK, tPV, p);
   return cudaGetLastError() == cudaSuccess ? MLA_OK : MLA_ERR_CUDA;
 }
 
