@@ -77,6 +77,7 @@ constexpr float kRescaleLog2 = 8.0f;
 }  // namespace dtc
 
 struct DecodeTcParams {
+  const uint8_t* pool;    // [n_pages][64][576] bf16
   const int32_t* page_table;
   const int32_t* seq_lens;
   const int32_t* start;   // [V + 1] block prefix sums from plan_kernel
@@ -157,7 +158,7 @@ __device__ __forceinline__ void page_of(const DecodeTcParams& P, int b, int L, i
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(dtc::kThreads, 1)
     decode_tc_kernel(const __grid_constant__ CUtensorMap tmQ,
                      const __grid_constant__ CUtensorMap tmQK,
-                     const __grid_constant__ CUtensorMap tmPV, const DecodeTcParams P) {
+                     const DecodeTcParams P) {
   using namespace dtc;
   extern __shared__ uint8_t smem_raw[];
   __shared__ __align__(8) uint64_t qk_full[kQkStages], qk_empty[kQkStages];
@@ -185,7 +186,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(dtc::kThreads, 1)
       mbar_init(smem_u32(&qk_empty[s]), 1);  // MMA commit (multicast)
     }
     for (int s = 0; s < kPvStages; ++s) {
-      mbar_init(smem_u32(&pv_full[s]), 1);
+      // 32 cp.async lanes of one loader warp (+ the peer's relay on the leader)
+      mbar_init(smem_u32(&pv_full[s]), rank == 0 ? 33u : 32u);
       mbar_init(smem_u32(&pv_empty[s]), 1);
     }
     mbar_init(smem_u32(&q_full), 1);
@@ -198,7 +200,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(dtc::kThreads, 1)
     fence_mbar_init();
     tma_prefetch_desc(&tmQ);
     tma_prefetch_desc(&tmQK);
-    tma_prefetch_desc(&tmPV);
   }
   if (warp == 1) {
     tmem_alloc<2>(smem_u32(&tmem_base_sh), kTmemCols);
@@ -260,9 +261,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(dtc::kThreads, 1)
       while (globaltimer() - t0 < 50000ull) {
       }
     }
-  } else if (warp == 2 && lane == 0) {
-    // =================  PV producer: this CTA's latent half of both pages  =====
-    const uint32_t lead_full0 = mapa_shared(smem_u32(&pv_full[0]), 0);
+  } else if (warp == 2 || warp == 3) {
+    // ======  PV loader warps (cp.async): this CTA's latent half of page p  ======
+    // Warp 2 fills the stages of page 0, warp 3 those of page 1.  The copies
+    // go through the load/store path rather than the bulk-copy engine, which
+    // is busy with the QK boxes.  Each stage lands as [n][chunk][slot][64
+    // columns] for latent chunks 4n + 2r + {0, 1}; rows past the sequence
+    // are written as zeros.
+    const int mine = warp - 2;
     uint32_t it = 0;
     PieceIter pi;
     pi.init(P.start, V, lo, hi);
@@ -273,24 +279,54 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(dtc::kThreads, 1)
       const int L = P.seq_lens[b];
       for (int x = x0; x < x1 && ok; ++x)
         for (int p = 0; p < 2; ++p, ++it) {
+          if (p != mine) continue;
+          // same row placement as the QK boxes: shared-memory row i holds
+          // slot i + slot0 (slot0 <= 0; a partial page sits at the bottom),
+          // and slot0 == kPage marks a page past the context (all zeros)
           int page, slot0;
           page_of(P, b, L, x, p, page, slot0);
           const int s = it % kPvStages;
-          if (!mbar_wait(smem_u32(&pv_empty[s]), ((it / kPvStages) & 1) ^ 1, abort_p, 11, it)) {
+          const bool got = mbar_wait(smem_u32(&pv_empty[s]), ((it / kPvStages) & 1) ^ 1,
+                                     abort_p, 11, it);
+          if (!__all_sync(0xffffffffu, got)) { ok = false; break; }
+          const uint8_t* src = P.pool + (size_t)page * (kPage * kD * 2);
+          const uint32_t dst = sPv + s * kPvStageBytes;
+#pragma unroll 8
+          for (int i = 0; i < 64; ++i) {
+            // one 512-byte row per warp step: 4 chunks x 8 units of 16 B
+            const int row = i, q4 = lane >> 3, u = lane & 7;
+            const int chunk = 4 * (q4 >> 1) + 2 * (int)rank + (q4 & 1);
+            const int srow = row + slot0;
+            const uint32_t d = dst + q4 * kChunk + row * 128 + ((u ^ (row & 7)) << 4);
+            if (slot0 < kPage && srow >= 0)
+              cp_async16(d, src + srow * (kD * 2) + chunk * 128 + u * 16);
+            else
+              st_shared_zero16(d);
+          }
+          if (slot0 != 0) fence_proxy_async_smem();
+          cp_async_arrive_noinc(smem_u32(&pv_full[s]));
+        }
+    }
+    asm volatile("cp.async.wait_all;" ::: "memory");
+  } else if (warp == 1 && lane == 0 && rank == 1) {
+    // ======  peer relay: forward landed PV stages to the leader's barriers  ======
+    const uint32_t lead0 = mapa_shared(smem_u32(&pv_full[0]), 0);
+    PieceIter pi;
+    pi.init(P.start, V, lo, hi);
+    int v, x0, x1;
+    uint32_t it = 0;
+    bool ok = true;
+    while (ok && pi.next(v, x0, x1)) {
+      for (int x = x0; x < x1 && ok; ++x)
+        for (int p = 0; p < 2; ++p, ++it) {
+          const int s = it % kPvStages;
+          if (!mbar_wait(smem_u32(&pv_full[s]), (it / kPvStages) & 1, abort_p, 14, it)) {
             ok = false;
             break;
           }
-          const uint32_t fb = lead_full0 + s * 8;
-          if (rank == 0) mbar_expect_tx(smem_u32(&pv_full[s]), 2 * kPvStageBytes);
-          // one box = latent chunks {4n + 2r, 4n + 2r + 1} for n = 0, 1 of page p,
-          // landing as [n][chunk][slot][64 columns]
-          tma_load_5d_pair(sPv + s * kPvStageBytes, &tmPV, 0, slot0, 2 * (int)rank, 0, page, fb);
+          fence_proxy_async_smem();
+          mbar_arrive_cluster(lead0 + s * 8);
         }
-    }
-    if (!ok) {
-      const uint64_t t0 = globaltimer();
-      while (globaltimer() - t0 < 50000ull) {
-      }
     }
   } else if (warp == 1 && lane == 0 && rank == 0) {
     // =================  MMA issuer (leader CTA)  =================
@@ -517,7 +553,7 @@ inline mla_status launch_decode_tc_impl(
     const int32_t* seq_lens, int B, int S_q, int H, float scale, int G, const int32_t* start,
     float* ws_lse, float* ws_o, cudaStream_t st) {
   using namespace dtc;
-  CUtensorMap tQ, tQK, tPV;
+  CUtensorMap tQ, tQK;
   {
     const uint64_t dims[2] = {(uint64_t)kD, (uint64_t)B * S_q * H};
     const uint64_t strides[1] = {(uint64_t)kD * 2};
@@ -532,14 +568,8 @@ inline mla_status launch_decode_tc_impl(
     const uint32_t box[4] = {64, 64, (uint32_t)kQkChunks, 1};
     if (!make_tmap(&tQK, pool, 4, dims, strides, box)) return MLA_ERR_CUDA;
   }
-  // Latent chunks grouped as (chunk-in-group 0..3, group n 0..1): chunk 4n + i.
-  {
-    const uint64_t dims[5] = {64, (uint64_t)kPage, 4, 2, (uint64_t)n_pages};
-    const uint64_t strides[4] = {(uint64_t)kD * 2, 128, 512, (uint64_t)kD * 2 * kPage};
-    const uint32_t box[5] = {64, 64, 2, 2, 1};
-    if (!make_tmap(&tPV, pool, 5, dims, strides, box)) return MLA_ERR_CUDA;
-  }
   DecodeTcParams p;
+  p.pool = static_cast<const uint8_t*>(pool);
   p.page_table = page_table;
   p.seq_lens = seq_lens;
   p.start = start;
@@ -556,7 +586,7 @@ inline mla_status launch_decode_tc_impl(
   if (cudaFuncSetAttribute(decode_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            (int)kSmemBytes) != cudaSuccess)
     return MLA_ERR_CUDA;
-  decode_tc_kernel<<<2 * G, kThreads, kSmemBytes, st>>>(tQ, tQK, tPV, p);
+  decode_tc_kernel<<<2 * G, kThreads, kSmemBytes, st>>>(tQ, tQK, p);
   return cudaGetLastError() == cudaSuccess ? MLA_OK : MLA_ERR_CUDA;
 }
 
