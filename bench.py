@@ -138,6 +138,24 @@ def _traffic_for(kernel_src_paths):
     return rec.get("dram_bytes_per_call")
 
 
+def max_over_ranks(vals, device=None):
+    """Element-wise maximum of `vals` over all ranks of the default process
+    group (the values themselves when there is no group or one rank)."""
+    import torch
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return [float(v) for v in vals]
+    t = torch.tensor([float(v) for v in vals], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return t.tolist()
+
+
+def whole_job_rate(units_per_rank, world, ms):
+    """Units per second of the whole job: every rank's units over the
+    slowest rank's time (ms)."""
+    return units_per_rank * world / (ms * 1e-3)
+
+
 # ---------------------------------------------------------------------------
 # CPU oracle arm
 # ---------------------------------------------------------------------------
@@ -215,8 +233,11 @@ def run_gpu(args, w):
     dev = torch.device("cuda", local)
     if world > 1:
         import datetime
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=600),
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
                                 device_id=dev)
+    # weak scaling: this rank's own sequences of a world * B batch
+    workload_name = w.name
+    w = wl.shard(w, rank, world)
     if rank == 0:
         _build.build()
     if world > 1:
@@ -317,10 +338,7 @@ def run_gpu(args, w):
     t_step = sum(step_ms) / len(step_ms)
     t_dec = sum(dec_ms) / len(dec_ms)
     t_e2e = sum(e2e_ms) / len(e2e_ms)
-    if world > 1:
-        tt = torch.tensor([t_step, t_dec, t_e2e], device=dev)
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        t_step, t_dec, t_e2e = tt.tolist()
+    t_step, t_dec, t_e2e = max_over_ranks([t_step, t_dec, t_e2e], dev)
 
     hbm_peak, tf_peak, peak_kind = _peaks()
     alg_bytes, flops, cache_bytes = _workload_bytes(w)
@@ -328,10 +346,9 @@ def run_gpu(args, w):
     roof_t = max(alg_bytes / (hbm_peak * 1e9), flops / (tf_peak * 1e12))
     csrc = os.path.join(ROOT, "mla_latent_kv_35_b200", "csrc")
     traffic = _traffic_for([os.path.join(csrc, "decode_tc.cuh")])
-    tokens = w.T * world
     line = {
         "metric": "MLA decode tokens/s (one attention layer, whole step A0-A6)",
-        "value": tokens / (t_step * 1e-3),
+        "value": whole_job_rate(w.T, world, t_step),
         "unit": "tokens/s",
         "n_gpus": world,
         "steps": args.steps,
@@ -342,13 +359,16 @@ def run_gpu(args, w):
         "vs_baseline": None,
         "dtype": "bf16" if w.dtype == "bf16" else "f32",
         "data": "synthetic",
-        "config": {"workload": w.name, "batch_per_gpu": w.B, "heads": w.H,
+        "config": {"workload": workload_name, "batch_per_gpu": w.B,
+                   "global_batch": w.B * world,
+                   "heads": w.H,
                    "context": w.ctx[0] if len(set(w.ctx)) == 1 else "ragged",
                    "S_q": w.S_q, "latent": w.d_latent, "rope": w.d_rope,
                    "page": w.page_size, "d_model": w.d_model,
                    "l2": "inputs larger than L2 (cache %.2f GB), no flush" % (cache_bytes / 1e9),
-                   "parallelism": f"replicas x{world}" if world > 1 else "single GPU"},
-        "decode": {"ms": t_dec, "tokens_per_s": tokens / (t_dec * 1e-3),
+                   "parallelism": (f"dp{world}: independent sequence shards, no collective"
+                                   if world > 1 else "single GPU")},
+        "decode": {"ms": t_dec, "tokens_per_s": whole_job_rate(w.T, world, t_dec),
                    "cache_gb_per_s": cache_bytes / (t_dec * 1e-3) / 1e9,
                    "tflops": flops / (t_dec * 1e-3) / 1e12,
                    "roofline_ms": roof_t * 1e3, "frac_of_roofline": roof_t / (t_dec * 1e-3)},
@@ -356,7 +376,8 @@ def run_gpu(args, w):
                      "achieved": achieved, "peak": hbm_peak, "unit": "GB/s",
                      "frac": achieved / hbm_peak, "peak_source": peak_kind,
                      "alg_bytes_per_launch": alg_bytes, "traffic": traffic},
-        "e2e": {"value": tokens / (t_e2e * 1e-3), "unit": "tokens/s", "ms_per_step": t_e2e,
+        "e2e": {"value": whole_job_rate(w.T, world, t_e2e), "unit": "tokens/s",
+                "ms_per_step": t_e2e,
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
         "gpu_launches": launches,
         "clocks": clocks,

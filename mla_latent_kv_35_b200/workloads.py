@@ -56,6 +56,8 @@ class Workload:
     rope_base: float = 10000.0
     page_size: int = PAGE_SIZE
     peaky: bool = False
+    seq_offset: int = 0          # global index of this batch's sequence 0
+    global_B: int = 0            # sequences in the whole (sharded) batch; 0 = B
     extra: dict = field(default_factory=dict, compare=False)
 
     @property
@@ -105,7 +107,7 @@ def workload(name: str, **over) -> Workload:
     elif name == "ragged":
         lens = _ragged_lengths(64, 7)
         w = Workload("ragged", B=64, S_q=1, ctx=tuple(L + 1 for L in lens),
-                     permute_pages=True, **big)
+                     permute_pages=True, extra={"len_seed": 7}, **big)
     elif name in ("long1", "long4"):
         B = 1 if name == "long1" else 4
         w = Workload(name, B=B, S_q=2, ctx=(131072,) * B,
@@ -116,6 +118,27 @@ def workload(name: str, **over) -> Workload:
 
 
 WORKLOADS = ("tiny", "dsv2", "batch128", "ragged", "long1", "long4")
+
+
+def shard(w: Workload, rank: int, world: int) -> Workload:
+    """Rank `rank`'s share of a batch of world * w.B sequences (weak scaling).
+
+    The whole batch is the named workload grown to world * B sequences; rank r
+    takes global sequences [r * B, r * B + B).  Each sequence's cache and
+    hidden state come from streams keyed by its global index, so a shard's
+    sequences are the same numbers wherever they run, rank 0's shard is the
+    unsharded workload, and the ranks' sequences differ.  Weights are shared.
+    """
+    if world <= 1:
+        return w
+    if not 0 <= rank < world:
+        raise ValueError(f"rank {rank} outside world {world}")
+    ctx = w.ctx
+    if "len_seed" in w.extra:
+        lens = _ragged_lengths(world * w.B, w.extra["len_seed"])
+        ctx = tuple(L + w.S_q for L in lens[rank * w.B:(rank + 1) * w.B])
+    return replace(w, ctx=ctx, seq_offset=rank * w.B, global_B=world * w.B,
+                   name=f"{w.name}[rank {rank} of {world}]")
 
 
 # ---------------------------------------------------------------------------
@@ -176,7 +199,8 @@ def draw_weights(w: Workload) -> dict:
 
 def draw_h_new(w: Workload) -> np.ndarray:
     """Hidden states of the new tokens, [B, S_q, d_model] ~ N(0, 1)."""
-    h = _normal(w, _S_H, (w.B, w.S_q, w.d_model))
+    gB = w.global_B or w.B
+    h = _normal(w, _S_H, (gB, w.S_q, w.d_model))[w.seq_offset:w.seq_offset + w.B]
     if w.peaky:
         h *= np.float32(4.0)
     return _quant(w, h)
@@ -184,17 +208,18 @@ def draw_h_new(w: Workload) -> np.ndarray:
 
 def draw_h_ctx(w: Workload, b: int) -> np.ndarray:
     """Hidden states of sequence b's prior tokens (tiny workload only)."""
-    return _quant(w, _normal(w, _S_HCTX, (w.prior[b], w.d_model), idx=b))
+    return _quant(w, _normal(w, _S_HCTX, (w.prior[b], w.d_model), idx=w.seq_offset + b))
 
 
 def draw_prior(w: Workload, b: int):
     """Sequence b's prior cache drawn directly: (latents [Lp, d_c],
     pre-RoPE keys [Lp, d_r]), both ~ N(0, 1), rounded for bf16."""
     Lp = w.prior[b]
-    c = _normal(w, _S_LAT, (Lp, w.d_latent), idx=b)
-    kr = _normal(w, _S_KR, (Lp, w.d_rope), idx=b)
+    g = w.seq_offset + b
+    c = _normal(w, _S_LAT, (Lp, w.d_latent), idx=g)
+    kr = _normal(w, _S_KR, (Lp, w.d_rope), idx=g)
     if w.peaky and Lp > 0:
-        t = int(_rng(w, _S_PEAK, b).integers(0, Lp))
+        t = int(_rng(w, _S_PEAK, g).integers(0, Lp))
         c[t] *= np.float32(6.0)
     return _quant(w, c), _quant(w, kr)
 
@@ -224,7 +249,7 @@ def page_layout(w: Workload):
     n = w.pages_per_seq
     total = int(sum(n))
     if w.permute_pages:
-        perm = _rng(w, _S_PERM).permutation(total).astype(np.int32)
+        perm = _rng(w, _S_PERM, w.seq_offset).permutation(total).astype(np.int32)
     else:
         perm = np.arange(total, dtype=np.int32)
     table = np.full((w.B, max(n)), -1, dtype=np.int32)
