@@ -265,12 +265,8 @@ def run_gpu(args, w):
     pos = torch.from_numpy(pos_np).to(dev)
     stream = torch.cuda.current_stream(dev)
 
-    def step(ev=None):
-        if ev is not None:
-            ev[0].record(stream)
+    def eager_step():
         layer.step(h, bi, pos, w.B, w.S_q)
-        if ev is not None:
-            ev[1].record(stream)
 
     # the decode call alone, with events on the launching stream
     bf = layer.buffers(w.B, w.S_q)
@@ -281,11 +277,20 @@ def run_gpu(args, w):
                      bf["lse"])
 
     for _ in range(args.warmup):
-        step()
+        eager_step()
     torch.cuda.synchronize(dev)
     st = B.mla_get_device_status()
     if st != 0:
         raise RuntimeError(f"device status after warm-up: {B.mla_status_string(st)}")
+    # the timed step is a CUDA graph of the whole step (captured once, replayed)
+    graph, gbuf, kernels_per_step = layer.capture(h, bi, pos, w.B, w.S_q)
+
+    def step():
+        graph.replay()
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize(dev)
 
     def timed(fn, K):
         evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
@@ -308,7 +313,9 @@ def run_gpu(args, w):
         return ms, wall, launches
 
     with ClockSampler(local) as clk:
-        step_ms, wall, launches = timed(step, args.steps)
+        step_ms, wall, _ = timed(step, args.steps)
+        launches = kernels_per_step * args.steps
+        eager_ms, _, eager_launches = timed(eager_step, max(3, args.steps // 4))
         dec_ms, _, dec_launches = timed(decode_only, max(args.steps, 5))
     clocks = clk.summary()
     st = B.mla_get_device_status()
@@ -325,8 +332,8 @@ def run_gpu(args, w):
         h.copy_(h_host, non_blocking=True)
         bi.copy_(bi_host, non_blocking=True)
         pos.copy_(pos_host, non_blocking=True)
-        b = layer.step(h, bi, pos, w.B, w.S_q)
-        out_host.copy_(b["out"], non_blocking=True)
+        graph.replay()
+        out_host.copy_(gbuf["out"], non_blocking=True)
 
     for _ in range(2):
         e2e_step()
@@ -338,7 +345,8 @@ def run_gpu(args, w):
     t_step = sum(step_ms) / len(step_ms)
     t_dec = sum(dec_ms) / len(dec_ms)
     t_e2e = sum(e2e_ms) / len(e2e_ms)
-    t_step, t_dec, t_e2e = max_over_ranks([t_step, t_dec, t_e2e], dev)
+    t_eager = sum(eager_ms) / len(eager_ms)
+    t_step, t_dec, t_e2e, t_eager = max_over_ranks([t_step, t_dec, t_e2e, t_eager], dev)
 
     hbm_peak, tf_peak, peak_kind = _peaks()
     alg_bytes, flops, cache_bytes = _workload_bytes(w)
@@ -380,6 +388,9 @@ def run_gpu(args, w):
                 "ms_per_step": t_e2e,
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
         "gpu_launches": launches,
+        "step": {"cuda_graph": True, "kernels_per_step": kernels_per_step,
+                 "eager_ms_per_step": t_eager,
+                 "eager_launches_per_step": eager_launches / max(1, len(eager_ms))},
         "clocks": clocks,
         "wall_s_timed": wall,
     }
@@ -389,6 +400,7 @@ def run_gpu(args, w):
                                 "sample": sample}
     if rank == 0:
         print(json.dumps(line), flush=True)
+    del graph
     if world > 1:
         dist.barrier()
         dist.destroy_process_group()

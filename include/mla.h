@@ -124,6 +124,30 @@ mla_status mla_cache_append(const mla_dims* dims, const void* c, int cs_tok,
                             const int32_t* page_table, int max_pages,
                             void* pool, int n_pages, int T, void* stream);
 
+/* A1 + A2 + A3 in one call: everything between the projection and the
+ * decode ([DF-1]; the pages describe the steps, not this grouping).
+ * y: device [T][y_stride_tok] rows as mla_project writes them for
+ * W_A0 = [W_Q; W_DKV; W_KR]:
+ *   y[t] = [q_1 .. q_H | c (d_latent) | k_rope_pre (d_rope)],
+ *   q_i = [q_nope (d_nope) ; q_rope (d_rope)],  y_stride_tok >= H*(d_nope+d_rope)
+ *   + d_latent + d_rope.
+ * Effects, each exactly as the separate call would make them:
+ *   qbuf[t][i][0 : d_latent]   = W_UK,i^T q_nope        (mla_absorb_q)
+ *   qbuf[t][i][d_latent : ]    = RoPE(q_rope, pos[t])    (mla_rope)
+ *   y's k_rope_pre of token t  = RoPE(k_rope_pre, pos[t]), in place (mla_rope)
+ *   the cache slot of (batch_idx[t], pos[t]) = [c ; roped k_rope]
+ *                                                          (mla_cache_append)
+ * For bf16 this is one kernel launch: the absorb GEMM's CTAs plus extra CTAs
+ * for the RoPE and append work, which the GEMM does not touch.  For fp32 it
+ * runs the four calls in turn.  w_uk, qbuf, batch_idx, pos, page_table, pool
+ * as in those calls; the same host checks and the same MLA_ERR_BOUNDS
+ * reporting apply.  bf16 needs y_stride_tok % 8 == 0. */
+mla_status mla_pre_attention(const mla_dims* dims, void* y, int y_stride_tok,
+                             const void* w_uk, void* qbuf,
+                             const int32_t* batch_idx, const int32_t* pos,
+                             const int32_t* page_table, int max_pages,
+                             void* pool, int n_pages, int T, void* stream);
+
 /* Workspace bytes mla_decode needs for B sequences of S_q query tokens and
  * num_workers split workers (0 = the default mla_decode would pick). */
 size_t mla_decode_workspace_size(const mla_dims* dims, int B, int S_q,

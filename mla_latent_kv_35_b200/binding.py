@@ -26,7 +26,7 @@ EXPORTS = ("mla_project", "mla_absorb_q", "mla_rope", "mla_cache_append",
            "mla_decode_workspace_size", "mla_decode", "mla_out_proj_scratch_size",
            "mla_out_proj", "mla_get_device_status", "mla_status_string",
            "mla_launch_count", "mla_selftest_wait_timeout", "mla_get_wait_diag",
-           "mla_decode_noalloc")
+           "mla_decode_noalloc", "mla_pre_attention")
 
 
 class MLAError(RuntimeError):
@@ -93,6 +93,8 @@ _SIGS = {
     "mla_get_wait_diag": ([ctypes.POINTER(ctypes.c_uint32)], _I),
     "mla_decode_noalloc": ([ctypes.POINTER(Dims), _P, _P, _I, _P, _I, _P, _I, _I, _I, _P, _P,
                             _P], _I),
+    "mla_pre_attention": ([ctypes.POINTER(Dims), _P, _I, _P, _P, _P, _P, _P, _I, _P, _I, _I,
+                           _P], _I),
 }
 
 
@@ -160,6 +162,14 @@ def mla_cache_append(dims: MLADims, c, cs_tok, kr, ks_tok, batch_idx, pos, page_
     _check("mla_cache_append", lib().mla_cache_append(
         ctypes.byref(dims.c()), _ptr(c), cs_tok, _ptr(kr), ks_tok, _ptr(batch_idx), _ptr(pos),
         _ptr(page_table), max_pages, _ptr(pool), n_pages, T, _stream()))
+
+
+def mla_pre_attention(dims: MLADims, y, y_stride_tok, w_uk, qbuf, batch_idx, pos, page_table,
+                      max_pages, pool, n_pages, T):
+    _dev(y, w_uk, qbuf, batch_idx, pos, page_table, pool)
+    _check("mla_pre_attention", lib().mla_pre_attention(
+        ctypes.byref(dims.c()), _ptr(y), y_stride_tok, _ptr(w_uk), _ptr(qbuf), _ptr(batch_idx),
+        _ptr(pos), _ptr(page_table), max_pages, _ptr(pool), n_pages, T, _stream()))
 
 
 def mla_decode_workspace_size(dims: MLADims, B: int, S_q: int, num_workers: int = 0) -> int:

@@ -3,6 +3,7 @@
 // Host-side validation, TMA descriptor encoding, split planning and kernel
 // launches.  All device work is in the kernels included below; nothing here
 // computes on the host.
+#include <algorithm>
 #include <atomic>
 #include <cmath>
 #include <cstdio>
@@ -132,7 +133,8 @@ TcGemmPlan plan_tc_gemm(int M, int N, int K, int batch, bool allow_split) {
 // out element (b, n, m) at ob*b + on*n + om*m.
 mla_status launch_tc_gemm(const void* A, bool a_mn, long long as_b, const void* X, long long xs_n,
                           long long xs_b, int M, int N, int K, int batch, void* out, long long ob,
-                          long long on, long long om, int out_kind, cudaStream_t st) {
+                          long long on, long long om, int out_kind, cudaStream_t st,
+                          const PreAttnAux* aux = nullptr) {
   if (M <= 0 || N <= 0 || batch <= 0) return MLA_OK;
   if (!aligned16(A) || !aligned16(X) || (K % 8) != 0 || (xs_n % 8) != 0 || (xs_b % 8) != 0 ||
       (as_b % 8) != 0)
@@ -168,7 +170,16 @@ mla_status launch_tc_gemm(const void* A, bool a_mn, long long as_b, const void* 
   g.k_chunks_per_split = p.k_chunks_per_split;
   g.stages = p.stages;
   g.out = out; g.ob = ob; g.on = on; g.om = om;
-  dim3 grid((M + kGemmBM - 1) / kGemmBM, p.n_tiles * p.splits, batch);
+  g.batch = batch;
+  g.aux = PreAttnAux{};
+  int aux_z = 0;
+  if (aux != nullptr && aux->n_items > 0) {
+    // enough extra z-slices for about 8 work items per thread
+    g.aux = *aux;
+    const long long per_slice = (long long)((M + kGemmBM - 1) / kGemmBM) * p.n_tiles * p.splits * 128;
+    aux_z = (int)std::min<long long>(4096, (aux->n_items + 8 * per_slice - 1) / (8 * per_slice));
+  }
+  dim3 grid((M + kGemmBM - 1) / kGemmBM, p.n_tiles * p.splits, batch + aux_z);
 #define MLA_GEMM_LAUNCH(AMN, OUT)                                                              \
   do {                                                                                         \
     auto kfn = gemm_tc_kernel<AMN, OUT>;                                                       \
@@ -346,6 +357,53 @@ mla_status mla_cache_append(const mla_dims* dims, const void* c, int cs_tok, con
         batch_idx, pos, page_table, max_pages, static_cast<uint16_t*>(pool), n_pages,
         dims->page_size, dims->d_latent, dims->d_rope);
   return check_launch();
+}
+
+mla_status mla_pre_attention(const mla_dims* dims, void* y, int y_stride_tok, const void* w_uk,
+                             void* qbuf, const int32_t* batch_idx, const int32_t* pos,
+                             const int32_t* page_table, int max_pages, void* pool, int n_pages,
+                             int T, void* stream) {
+  if (!dims_ok(dims) || T < 0 || max_pages < 1 || n_pages < 1) return MLA_ERR_INVALID_ARG;
+  if (T == 0) return MLA_OK;
+  if (!y || !w_uk || !qbuf || !batch_idx || !pos || !page_table || !pool)
+    return MLA_ERR_INVALID_ARG;
+  const int H = dims->n_heads, dn = dims->d_nope, dc = dims->d_latent, dr = dims->d_rope;
+  const int dqk = dn + dr;
+  const long long off_c = (long long)H * dqk;
+  if ((long long)y_stride_tok < off_c + dc + dr) return MLA_ERR_INVALID_ARG;
+  const int D = dc + dr;
+  if (dims->dtype == MLA_F32) {
+    // the same four steps as separate launches
+    char* yb = static_cast<char*>(y);
+    const int es = 4;
+    MLA_TRY(mla_rope(dims, yb + (long long)dn * es, y_stride_tok, dqk, H,
+                     static_cast<char*>(qbuf) + (long long)dc * es, H * D, D, pos, T, stream));
+    void* kr = yb + (off_c + dc) * es;
+    MLA_TRY(mla_rope(dims, kr, y_stride_tok, 0, 1, kr, y_stride_tok, 0, pos, T, stream));
+    MLA_TRY(mla_cache_append(dims, yb + off_c * es, y_stride_tok, kr, y_stride_tok, batch_idx,
+                             pos, page_table, max_pages, pool, n_pages, T, stream));
+    return mla_absorb_q(dims, y, y_stride_tok, w_uk, qbuf, T, stream);
+  }
+  if ((y_stride_tok % 2) != 0 || (dc % 2) != 0 || (dr % 2) != 0 || (off_c % 2) != 0)
+    return MLA_ERR_UNSUPPORTED;
+  if ((dn % 16) != 0 || (dc % 128) != 0 || (y_stride_tok % 8) != 0 || (dqk % 8) != 0)
+    return MLA_ERR_UNSUPPORTED;
+  PreAttnAux aux{};
+  aux.y = static_cast<__nv_bfloat16*>(y);
+  aux.ys_tok = y_stride_tok;
+  aux.H = H; aux.d_nope = dn; aux.d_latent = dc; aux.d_rope = dr;
+  aux.off_c = off_c;
+  aux.qbuf = static_cast<__nv_bfloat16*>(qbuf);
+  aux.batch_idx = batch_idx; aux.pos = pos; aux.page_table = page_table;
+  aux.max_pages = max_pages;
+  aux.pool = static_cast<uint16_t*>(pool);
+  aux.n_pages = n_pages; aux.page_size = dims->page_size;
+  aux.base = (double)dims->rope_base;
+  aux.n_q = (long long)T * H * (dr / 2);
+  aux.n_items = aux.n_q + (long long)T * (D / 2);
+  // A1 on the GEMM CTAs, A2 and A3 on extra CTAs of the same launch
+  return launch_tc_gemm(w_uk, true, (long long)dn * dc, y, y_stride_tok, dqk, dc, T, dn, H, qbuf,
+                        D, (long long)H * D, 1, kOutBf16, as_stream(stream), &aux);
 }
 
 size_t mla_decode_workspace_size(const mla_dims* dims, int B, int S_q, int num_workers) {

@@ -18,6 +18,7 @@
 #pragma once
 
 #include "common.cuh"
+#include "pre_attn.cuh"
 
 namespace mla {
 
@@ -31,6 +32,8 @@ struct GemmTcArgs {
   int stages;
   void* out;
   long long ob, on, om;  // output strides in elements
+  int batch;             // GEMM batch entries (grid.z slices [0, batch))
+  PreAttnAux aux;        // grid.z slices past `batch` run this (n_items > 0)
 };
 
 constexpr int kGemmBM = 128;
@@ -46,6 +49,17 @@ __global__ void __launch_bounds__(128, 1) gemm_tc_kernel(const __grid_constant__
   __shared__ __align__(8) uint64_t acc_bar;
   __shared__ uint32_t tmem_base_sh;
   __shared__ int abort_flag;
+
+  if ((int)blockIdx.z >= g.batch) {
+    // extra CTAs of a fused pre-attention launch: RoPE and cache append,
+    // independent of the GEMM CTAs (no barrier, no TMEM)
+    const long long per_slice = (long long)gridDim.x * gridDim.y * blockDim.x;
+    const long long cta =
+        ((long long)(blockIdx.z - g.batch) * gridDim.y + blockIdx.y) * gridDim.x + blockIdx.x;
+    pre_attention_aux(g.aux, cta * blockDim.x + threadIdx.x,
+                      per_slice * (long long)(gridDim.z - g.batch));
+    return;
+  }
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int m0 = blockIdx.x * kGemmBM;

@@ -4,6 +4,7 @@
 #pragma once
 
 #include "common.cuh"
+#include "pre_attn.cuh"
 
 namespace mla {
 
@@ -88,19 +89,7 @@ __global__ void rope_kernel(const T* x, long long xs_tok, long long xs_head, int
   const int k = (int)(idx % half);
   const int h = (int)((idx / half) % nh);
   const int t = (int)(idx / ((long long)half * nh));
-  const double theta = pow(base, -2.0 * (double)k / (double)d_rope);
-  const double ang = (double)pos[t] * theta;
-  // reduce to [-pi, pi] in fp64 before taking sine and cosine
-  const double two_pi = 6.283185307179586476925286766559;
-  const double red = ang - two_pi * rint(ang / two_pi);
-  double sn, cs;
-  sincos(red, &sn, &cs);
-  const float c = (float)cs, s = (float)sn;
-  const T* px = x + t * xs_tok + h * xs_head + 2 * k;
-  T* py = y + t * ys_tok + h * ys_head + 2 * k;
-  const float x0 = to_f32(px[0]), x1 = to_f32(px[1]);
-  py[0] = from_f32<T>(x0 * c - x1 * s);
-  py[1] = from_f32<T>(x0 * s + x1 * c);
+  rope_pair(x + t * xs_tok + h * xs_head, y + t * ys_tok + h * ys_head, k, pos[t], d_rope, base);
 }
 
 // ---------------------------------------------------------------------------
@@ -113,20 +102,10 @@ __global__ void append_kernel(const E* c, long long cs_tok, const E* kr, long lo
                               const int32_t* page_table, int max_pages, E* pool, int n_pages,
                               int page_size, int d_c, int d_r) {
   const int t = blockIdx.x;
-  const int b = batch_idx[t];
-  const int p = pos[t];
-  const int lp = p / page_size;
-  if (p < 0 || b < 0 || lp >= max_pages) {
-    if (threadIdx.x == 0) raise_flag(kFlagBounds);
-    return;
-  }
-  const int page = page_table[(long long)b * max_pages + lp];
-  if (page < 0 || page >= n_pages) {
-    if (threadIdx.x == 0) raise_flag(kFlagBounds);
-    return;
-  }
   const int D = d_c + d_r;
-  E* row = pool + ((long long)page * page_size + (p % page_size)) * D;
+  E* row = append_row(batch_idx, pos, t, page_table, max_pages, pool, n_pages, page_size, D,
+                      threadIdx.x == 0);
+  if (row == nullptr) return;
   for (int e = threadIdx.x; e < D; e += blockDim.x)
     row[e] = e < d_c ? c[t * cs_tok + e] : kr[t * ks_tok + (e - d_c)];
 }

@@ -102,9 +102,13 @@ class MLADecodeLayer:
     # ------------------------------------------------------------------
     # the hot path
     # ------------------------------------------------------------------
-    def step(self, h, batch_idx, pos, B: int, S_q: int, num_workers: int = 0):
+    def step(self, h, batch_idx, pos, B: int, S_q: int, num_workers: int = 0,
+             fused: bool = True):
         """h [T, d_model] device (dims dtype), batch_idx/pos int32 [T] device,
-        T = B*S_q tokens b-major.  Returns the dict of step buffers."""
+        T = B*S_q tokens b-major.  Returns the dict of step buffers.
+
+        fused: A1-A3 through mla_pre_attention (one launch for bf16) instead
+        of the four separate calls; both write the same bits."""
         d = self.dims
         H, dn, dc, dr = d.n_heads, d.d_nope, d.d_latent, d.d_rope
         T = B * S_q
@@ -112,19 +116,44 @@ class MLADecodeLayer:
         y, qbuf = bf["y"], bf["qbuf"]
         Y, D, dqk = self.Y, self.D, self.dqk
         _b.mla_project(d, h, self.W_A0, y, T, d.d_model, Y)                        # A0
-        off_c = H * dqk
-        _b.mla_rope(d, y[:, dn:], Y, dqk, H, qbuf[:, :, dc:], H * D, D, pos, T)   # A2 q
-        kr = y[:, off_c + dc:]
-        _b.mla_rope(d, kr, Y, 0, 1, kr, Y, 0, pos, T)                              # A2 k
-        _b.mla_cache_append(d, y[:, off_c:], Y, kr, Y, batch_idx, pos,             # A3
-                            self.page_table, self.max_pages, self.pool, self.n_pages, T)
-        _b.mla_absorb_q(d, y, Y, self.W_UK, qbuf, T)                                # A1
+        if fused:
+            _b.mla_pre_attention(d, y, Y, self.W_UK, qbuf, batch_idx, pos,          # A1-A3
+                                 self.page_table, self.max_pages, self.pool, self.n_pages, T)
+        else:
+            off_c = H * dqk
+            _b.mla_rope(d, y[:, dn:], Y, dqk, H, qbuf[:, :, dc:], H * D, D, pos, T)  # A2 q
+            kr = y[:, off_c + dc:]
+            _b.mla_rope(d, kr, Y, 0, 1, kr, Y, 0, pos, T)                             # A2 k
+            _b.mla_cache_append(d, y[:, off_c:], Y, kr, Y, batch_idx, pos,            # A3
+                                self.page_table, self.max_pages, self.pool, self.n_pages, T)
+            _b.mla_absorb_q(d, y, Y, self.W_UK, qbuf, T)                               # A1
         _b.mla_decode(d, qbuf, self.pool, self.n_pages, self.page_table,            # A4+A5
                       self.max_pages, self.seq_lens, B, S_q, num_workers, bf["ws"],
                       bf["o_lat"], bf["lse"])
         _b.mla_out_proj(d, bf["o_lat"], self.W_UV, self.W_O, bf["scratch"],         # A6
                         bf["out"], T)
         return bf
+
+    def capture(self, h, batch_idx, pos, B: int, S_q: int, num_workers: int = 0,
+                fused: bool = True):
+        """Capture one step on these input buffers into a CUDA graph.
+
+        Returns (graph, buffers, kernels): graph.replay() reruns the whole
+        step (projection through output projection) on whatever h,
+        batch_idx and pos hold at that time, writing the same buffers;
+        kernels is the number of kernel launches the graph contains.  The
+        step's buffers are allocated before capture, so the graph holds no
+        memory of its own.
+        """
+        bf = self.buffers(B, S_q, num_workers)
+        torch.cuda.synchronize(self.device)
+        graph = torch.cuda.CUDAGraph()
+        l0 = _b.mla_launch_count()
+        with torch.cuda.graph(graph):
+            self.step(h, batch_idx, pos, B, S_q, num_workers, fused)
+        kernels = _b.mla_launch_count() - l0
+        return graph, bf, kernels
+
 
 
 def build_pool_host(w, page_table, n_pages, prior_bits, canary=0xFFFF):

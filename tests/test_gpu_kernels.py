@@ -318,3 +318,35 @@ def test_decode_rejects_short_context():
     assert torch.isinf(lse[0]).all() and (o_lat[0] == 0).all()
     ref = _decode_ref(d, c, 1)
     check(to_np(o_lat)[1], ref["o_lat"], "bf16", "valid sequence still correct")
+
+
+@gpu
+@pytest.mark.parametrize("dtype,H,S_q", [("bf16", 128, 1), ("bf16", 128, 2), ("f32", 8, 1)])
+def test_decode_reports_page_outside_pool(dtype, H, S_q):
+    """A page id past the pool is reported as MLA_ERR_BOUNDS and never read;
+    the other sequences of the batch are unaffected."""
+    dc, dr = (64, 16) if dtype == "f32" else (512, 64)
+    lens = [300, 200, 90]
+    d, c = _decode_case(dtype, H, lens, S_q, seed=11, dc=dc, dr=dr)
+    c["table"][0, 2] = c["n_pages"] + 7
+    o_lat, lse = _run_decode_status(d, c, S_q, expect=5)
+    assert status() == 0                         # cleared by the first read
+    for b in (1, 2):
+        ref = _decode_ref(d, c, b)
+        check(o_lat[b], ref["o_lat"], dtype, f"o_lat b={b}")
+        check(lse[b], ref["lse"], dtype, f"lse b={b}")
+    assert np.isfinite(o_lat[0]).all()
+
+
+def _run_decode_status(d, c, S_q, expect):
+    Bn = len(c["lens"])
+    H, dc = d.n_heads, d.d_latent
+    ws = torch.empty((B.mla_decode_workspace_size(d, Bn, S_q, 0),), dtype=torch.uint8,
+                     device=DEV)
+    o_lat = torch.full((Bn, S_q, H, dc), float("nan"), device=DEV)
+    lse = torch.full((Bn, S_q, H), float("nan"), device=DEV)
+    B.mla_decode(d, to_dev(c["qb"], d.dtype), c["pool_d"], c["n_pages"],
+                 torch.from_numpy(c["table"]).to(DEV), c["maxp"],
+                 torch.from_numpy(c["lens"]).to(DEV), Bn, S_q, 0, ws, o_lat, lse)
+    assert status() == expect
+    return to_np(o_lat), to_np(lse)
