@@ -293,29 +293,31 @@ def run_gpu(args, w):
     torch.cuda.synchronize(dev)
 
     def timed(fn, K):
-        evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-               for _ in range(K)]
+        """K back-to-back calls between one pair of CUDA events on the
+        launching stream (barrier + synchronize on both sides); returns the
+        mean ms per call, the wall time and this process's kernel launches."""
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         if world > 1:
             dist.barrier()
         torch.cuda.synchronize(dev)
         l0 = B.mla_launch_count()
         t0 = time.perf_counter()
-        for e in evs:
-            e[0].record(stream)
+        e0.record(stream)
+        for _ in range(K):
             fn()
-            e[1].record(stream)
+        e1.record(stream)
         torch.cuda.synchronize(dev)
         wall = time.perf_counter() - t0
         launches = B.mla_launch_count() - l0
         if world > 1:
             dist.barrier()
-        ms = [a.elapsed_time(b) for a, b in evs]
-        return ms, wall, launches
+        return e0.elapsed_time(e1) / K, wall, launches
 
     with ClockSampler(local) as clk:
         step_ms, wall, _ = timed(step, args.steps)
         launches = kernels_per_step * args.steps
-        eager_ms, _, eager_launches = timed(eager_step, max(3, args.steps // 4))
+        n_eager = max(3, args.steps // 4)
+        eager_ms, _, eager_launches = timed(eager_step, n_eager)
         dec_ms, _, dec_launches = timed(decode_only, max(args.steps, 5))
     clocks = clk.summary()
     st = B.mla_get_device_status()
@@ -342,10 +344,7 @@ def run_gpu(args, w):
     d2h = out_host.numel() * 4
 
     # max over ranks
-    t_step = sum(step_ms) / len(step_ms)
-    t_dec = sum(dec_ms) / len(dec_ms)
-    t_e2e = sum(e2e_ms) / len(e2e_ms)
-    t_eager = sum(eager_ms) / len(eager_ms)
+    t_step, t_dec, t_e2e, t_eager = step_ms, dec_ms, e2e_ms, eager_ms
     t_step, t_dec, t_e2e, t_eager = max_over_ranks([t_step, t_dec, t_e2e, t_eager], dev)
 
     hbm_peak, tf_peak, peak_kind = _peaks()
@@ -390,7 +389,7 @@ def run_gpu(args, w):
         "gpu_launches": launches,
         "step": {"cuda_graph": True, "kernels_per_step": kernels_per_step,
                  "eager_ms_per_step": t_eager,
-                 "eager_launches_per_step": eager_launches / max(1, len(eager_ms))},
+                 "eager_launches_per_step": eager_launches / n_eager},
         "clocks": clocks,
         "wall_s_timed": wall,
     }
