@@ -174,11 +174,12 @@ mla_status launch_tc_gemm(const void* A, bool a_mn, long long as_b, const void* 
   g.aux = PreAttnAux{};
   int aux_z = 0;
   if (aux != nullptr && aux->n_items > 0) {
-    // enough extra z-slices for about 8 work items per thread
+    // enough extra z-slices for about 2 work items per thread
     g.aux = *aux;
     const long long per_slice = (long long)((M + kGemmBM - 1) / kGemmBM) * p.n_tiles * p.splits * 128;
-    aux_z = (int)std::min<long long>(4096, (aux->n_items + 8 * per_slice - 1) / (8 * per_slice));
+    aux_z = (int)std::min<long long>(4096, (aux->n_items + 2 * per_slice - 1) / (2 * per_slice));
   }
+  g.aux_z = aux_z;
   dim3 grid((M + kGemmBM - 1) / kGemmBM, p.n_tiles * p.splits, batch + aux_z);
 #define MLA_GEMM_LAUNCH(AMN, OUT)                                                              \
   do {                                                                                         \
@@ -384,7 +385,10 @@ mla_status mla_pre_attention(const mla_dims* dims, void* y, int y_stride_tok, co
                              pos, page_table, max_pages, pool, n_pages, T, stream));
     return mla_absorb_q(dims, y, y_stride_tok, w_uk, qbuf, T, stream);
   }
-  if ((y_stride_tok % 2) != 0 || (dc % 2) != 0 || (dr % 2) != 0 || (off_c % 2) != 0)
+  // 16-byte pieces of the latent and 4-byte RoPE pairs in y, qbuf and the pool
+  if ((y_stride_tok % 8) != 0 || (dc % 8) != 0 || (dr % 8) != 0 || (off_c % 8) != 0 ||
+      (reinterpret_cast<uintptr_t>(y) & 15u) != 0 || (reinterpret_cast<uintptr_t>(pool) & 15u) != 0 ||
+      (reinterpret_cast<uintptr_t>(qbuf) & 3u) != 0)
     return MLA_ERR_UNSUPPORTED;
   if ((dn % 16) != 0 || (dc % 128) != 0 || (y_stride_tok % 8) != 0 || (dqk % 8) != 0)
     return MLA_ERR_UNSUPPORTED;
@@ -399,8 +403,8 @@ mla_status mla_pre_attention(const mla_dims* dims, void* y, int y_stride_tok, co
   aux.pool = static_cast<uint16_t*>(pool);
   aux.n_pages = n_pages; aux.page_size = dims->page_size;
   aux.base = (double)dims->rope_base;
-  aux.n_q = (long long)T * H * (dr / 2);
-  aux.n_items = aux.n_q + (long long)T * (D / 2);
+  aux.n_rope = (long long)T * (dr / 2);
+  aux.n_items = aux.n_rope + (long long)T * (dc / 8);
   // A1 on the GEMM CTAs, A2 and A3 on extra CTAs of the same launch
   return launch_tc_gemm(w_uk, true, (long long)dn * dc, y, y_stride_tok, dqk, dc, T, dn, H, qbuf,
                         D, (long long)H * D, 1, kOutBf16, as_stream(stream), &aux);

@@ -32,8 +32,9 @@ struct GemmTcArgs {
   int stages;
   void* out;
   long long ob, on, om;  // output strides in elements
-  int batch;             // GEMM batch entries (grid.z slices [0, batch))
-  PreAttnAux aux;        // grid.z slices past `batch` run this (n_items > 0)
+  int batch;             // GEMM batch entries
+  int aux_z;             // grid.z slices [0, aux_z) run `aux`; GEMM entry b is slice aux_z + b
+  PreAttnAux aux;
 };
 
 constexpr int kGemmBM = 128;
@@ -50,14 +51,12 @@ __global__ void __launch_bounds__(128, 1) gemm_tc_kernel(const __grid_constant__
   __shared__ uint32_t tmem_base_sh;
   __shared__ int abort_flag;
 
-  if ((int)blockIdx.z >= g.batch) {
-    // extra CTAs of a fused pre-attention launch: RoPE and cache append,
-    // independent of the GEMM CTAs (no barrier, no TMEM)
+  if ((int)blockIdx.z < g.aux_z) {
+    // extra CTAs of a fused pre-attention launch (scheduled first): RoPE and
+    // cache append, independent of the GEMM CTAs (no barrier, no TMEM)
     const long long per_slice = (long long)gridDim.x * gridDim.y * blockDim.x;
-    const long long cta =
-        ((long long)(blockIdx.z - g.batch) * gridDim.y + blockIdx.y) * gridDim.x + blockIdx.x;
-    pre_attention_aux(g.aux, cta * blockDim.x + threadIdx.x,
-                      per_slice * (long long)(gridDim.z - g.batch));
+    const long long cta = ((long long)blockIdx.z * gridDim.y + blockIdx.y) * gridDim.x + blockIdx.x;
+    pre_attention_aux(g.aux, cta * blockDim.x + threadIdx.x, per_slice * (long long)g.aux_z);
     return;
   }
 
@@ -66,7 +65,7 @@ __global__ void __launch_bounds__(128, 1) gemm_tc_kernel(const __grid_constant__
   const int n_tile_idx = blockIdx.y % g.n_tiles;
   const int split = blockIdx.y / g.n_tiles;
   const int n0 = n_tile_idx * g.n_tile;
-  const int b = blockIdx.z;
+  const int b = blockIdx.z - g.aux_z;
   const int BN = g.n_tile;
   const int S = g.stages;
   const int k_chunks_total = (g.K + kGemmBK - 1) / kGemmBK;

@@ -73,11 +73,14 @@ __device__ __forceinline__ E* append_row(const int32_t* batch_idx, const int32_t
 // mla_project writes them for W_A0 = [W_Q; W_DKV; W_KR]:
 //   y[t] = [q_1 .. q_H | c | k_rope_pre],  q_i = [q_nope (d_n) ; q_rope (d_r)].
 // Work items, grid-strided:
-//   [0, n_q)          RoPE pair (t, head, k) of q_rope -> qbuf[t][head][d_c + 2k ..]
-//   [n_q, n_items)    pair e of token t's cache row: e < d_c/2 copies two latent
-//                     numbers, otherwise RoPE pair e - d_c/2 of k_rope, written to
-//                     the pool row and back into y (as the standalone in-place
-//                     RoPE of k does).
+//   [0, n_rope)        (token t, pair k): one angle, applied to pair k of every
+//                      head's q_rope (-> qbuf[t][head][d_c + 2k ..]) and of
+//                      k_rope (-> the pool row and back into y, as the
+//                      standalone in-place RoPE of k does)
+//   [n_rope, n_items)  (token t, 16-byte piece u) of the latent: copied to the
+//                      pool row
+// Consecutive items of a warp take consecutive k (or u), so every access of
+// the warp is one contiguous run.
 struct PreAttnAux {
   __nv_bfloat16* y;
   long long ys_tok;       // elements per token row of y
@@ -91,7 +94,7 @@ struct PreAttnAux {
   uint16_t* pool;
   int n_pages, page_size;
   double base;
-  long long n_q, n_items;
+  long long n_rope, n_items;
 };
 
 __device__ __forceinline__ void pre_attention_aux(const PreAttnAux& a, long long i0,
@@ -99,38 +102,47 @@ __device__ __forceinline__ void pre_attention_aux(const PreAttnAux& a, long long
   const int half = a.d_rope / 2;
   const int dqk = a.d_nope + a.d_rope;
   const int D = a.d_latent + a.d_rope;
-  const int row_pairs = D / 2;
+  const int pieces = a.d_latent / 8;
   for (long long i = i0; i < a.n_items; i += stride) {
-    if (i < a.n_q) {
+    if (i < a.n_rope) {
+      const int t = (int)(i / half);
       const int k = (int)(i % half);
-      const int h = (int)((i / half) % a.H);
-      const int t = (int)(i / ((long long)half * a.H));
-      const __nv_bfloat16* x = a.y + t * a.ys_tok + (long long)h * dqk + a.d_nope;
-      __nv_bfloat16* q = a.qbuf + ((long long)t * a.H + h) * D + a.d_latent;
-      rope_pair(x, q, k, a.pos[t], a.d_rope, a.base);
-    } else {
-      const long long j = i - a.n_q;
-      const int t = (int)(j / row_pairs);
-      const int e = (int)(j % row_pairs);
+      const int p = a.pos[t];
+      float c, sn;
+      rope_cos_sin(k, p, a.d_rope, a.base, c, sn);
+      const __nv_bfloat16* xq = a.y + t * a.ys_tok + a.d_nope + 2 * k;
+      __nv_bfloat16* yq = a.qbuf + (long long)t * a.H * D + a.d_latent + 2 * k;
+#pragma unroll 8
+      for (int h = 0; h < a.H; ++h) {
+        const __nv_bfloat162 v = *reinterpret_cast<const __nv_bfloat162*>(xq + (long long)h * dqk);
+        float y0, y1;
+        rope_rotate(to_f32(v.x), to_f32(v.y), c, sn, y0, y1);
+        __nv_bfloat162 o;
+        o.x = from_f32<__nv_bfloat16>(y0);
+        o.y = from_f32<__nv_bfloat16>(y1);
+        *reinterpret_cast<__nv_bfloat162*>(yq + (long long)h * D) = o;
+      }
+      __nv_bfloat16* kr = a.y + t * a.ys_tok + a.off_c + a.d_latent + 2 * k;
+      float y0, y1;
+      rope_rotate(to_f32(kr[0]), to_f32(kr[1]), c, sn, y0, y1);
+      const __nv_bfloat16 r0 = from_f32<__nv_bfloat16>(y0), r1 = from_f32<__nv_bfloat16>(y1);
+      kr[0] = r0;
+      kr[1] = r1;
       uint16_t* row = append_row(a.batch_idx, a.pos, t, a.page_table, a.max_pages, a.pool,
-                                 a.n_pages, a.page_size, D, e == 0);
-      if (row == nullptr) continue;
-      __nv_bfloat16* yt = a.y + t * a.ys_tok + a.off_c;
-      if (2 * e < a.d_latent) {
-        const uint32_t v = *reinterpret_cast<const uint32_t*>(yt + 2 * e);
-        *reinterpret_cast<uint32_t*>(row + 2 * e) = v;
-      } else {
-        const int k = e - a.d_latent / 2;
-        __nv_bfloat16* kr = yt + a.d_latent;
-        float c, sn, y0, y1;
-        rope_cos_sin(k, a.pos[t], a.d_rope, a.base, c, sn);
-        rope_rotate(to_f32(kr[2 * k]), to_f32(kr[2 * k + 1]), c, sn, y0, y1);
-        const __nv_bfloat16 r0 = from_f32<__nv_bfloat16>(y0), r1 = from_f32<__nv_bfloat16>(y1);
-        kr[2 * k] = r0;
-        kr[2 * k + 1] = r1;
+                                 a.n_pages, a.page_size, D, false);
+      if (row != nullptr) {
         row[a.d_latent + 2 * k] = __bfloat16_as_ushort(r0);
         row[a.d_latent + 2 * k + 1] = __bfloat16_as_ushort(r1);
       }
+    } else {
+      const long long j = i - a.n_rope;
+      const int t = (int)(j / pieces);
+      const int u = (int)(j % pieces);
+      uint16_t* row = append_row(a.batch_idx, a.pos, t, a.page_table, a.max_pages, a.pool,
+                                 a.n_pages, a.page_size, D, u == 0);
+      if (row == nullptr) continue;
+      const uint4 v = *reinterpret_cast<const uint4*>(a.y + t * a.ys_tok + a.off_c + 8 * u);
+      *reinterpret_cast<uint4*>(row + 8 * u) = v;
     }
   }
 }
