@@ -120,40 +120,35 @@ class ClockSampler:
                 "samples": len(sm)}
 
 
+def code_digest(paths):
+    """sha256 of the sources with comments and blank lines removed, so an
+    edit to comments alone does not count as a kernel change."""
+    import re
+    h = hashlib.sha256()
+    for p in paths:
+        with open(p) as f:
+            src = f.read()
+        src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+        src = re.sub(r"//[^\n]*", "", src)
+        for line in src.split("\n"):
+            line = line.strip()
+            if line:
+                h.update(line.encode() + b"\n")
+    return h.hexdigest()
+
+
 def _traffic_for(kernel_src_paths):
     """ncu DRAM bytes per decode call recorded in profiles/, if the kernel
-    source is unchanged since the capture (else None)."""
+    code is unchanged since the capture (else None)."""
     path = os.path.join(ROOT, "profiles", "decode_tc_traffic.json")
     try:
         with open(path) as f:
             rec = json.load(f)
     except Exception:
         return None
-    h = hashlib.sha256()
-    for p in kernel_src_paths:
-        with open(p, "rb") as f:
-            h.update(f.read())
-    if rec.get("source_sha256") != h.hexdigest():
+    if rec.get("code_sha256") != code_digest(kernel_src_paths):
         return None
     return rec.get("dram_bytes_per_call")
-
-
-def max_over_ranks(vals, device=None):
-    """Element-wise maximum of `vals` over all ranks of the default process
-    group (the values themselves when there is no group or one rank)."""
-    import torch
-    import torch.distributed as dist
-    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
-        return [float(v) for v in vals]
-    t = torch.tensor([float(v) for v in vals], dtype=torch.float64, device=device)
-    dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    return t.tolist()
-
-
-def whole_job_rate(units_per_rank, world, ms):
-    """Units per second of the whole job: every rank's units over the
-    slowest rank's time (ms)."""
-    return units_per_rank * world / (ms * 1e-3)
 
 
 # ---------------------------------------------------------------------------

@@ -11,8 +11,8 @@
 // Work decomposition
 //   * A cluster of two CTAs (one per SM of a TPC) owns 128 query rows
 //     (S_q*H rows of one sequence, 128 at a time) and a contiguous run of
-//     128-token blocks.  CTA r holds rows [64r, 64r+64): its Q slice (72 KB)
-//     stays in shared memory for the whole piece.
+//     128-token blocks.  CTA r holds rows [64r, 64r+64): its Q slice (72 KB,
+//     one TMA load per piece) stays in shared memory for the whole piece.
 //   * QK: pair MMAs (cta_group::2, M = 128 rows, N = 128 tokens, K = 576).
 //     CTA r supplies the B half of page r of the block.  Each SM gets its 64
 //     rows x 128 tokens in TMEM folded onto 128 lanes x 64 columns: lane l<64
@@ -22,21 +22,36 @@
 //     [256n + 128r, +128) of all 128 tokens (MN-major B read straight from
 //     the cache tile) and its own 64 rows of P (bf16, K-major).  O therefore
 //     takes 256 TMEM columns per SM; S is double buffered in 2 x 64 more.
-//   * QK tiles and PV tiles travel through two separate TMA rings with their
-//     own producer warps, so PV tiles waiting for P never hold back the QK
-//     loads of later blocks.
-//   * Each 128-thread softmax warpgroup reads its SM's S, exchanges row
-//     maxima between the two lanes that share a row, keeps a lazily rescaled
-//     running max (O is only rescaled in TMEM when the max grows by more than
-//     2^8), writes P to shared memory and signals the MMA warp of the leader.
+//   * Loads.  Warp 0 lane 0 of each CTA streams its own page of the block
+//     for QK through a 3-stage ring.  Each stage is one 24 KB TMA box (64
+//     columns x 64 slots x 3 chunks) of a 4-D view of the pool: (64 columns,
+//     64 slots, 9 chunks, pages), strides (1152 B, 128 B, 73728 B).  Only the
+//     leader arms the stage barrier, for the bytes of both CTAs; the peer's
+//     box completes on the leader's barrier.
+//   * PV tiles come through a second ring of two 32 KB stages, one page's
+//     latent half each.  Warps 2 and 3 fill them with 16-byte cp.async into
+//     the 128-byte-swizzled layout, so this traffic bypasses the bulk-copy
+//     engine the QK boxes keep busy.  In the peer CTA, warp 1 lane 0 relays
+//     each landed stage to the leader's barrier.
+//   * Each 128-thread softmax warpgroup reads its SM's S and exchanges row
+//     maxima between the two lanes that share a row.  It keeps a lazily
+//     rescaled running max: O is rescaled in TMEM only when the max grows by
+//     more than 2^8, and warp-uniformly, since tcgen05.ld/st are collective.
+//     It then writes P to shared memory and signals the leader's MMA warp.
 //   * Pieces (sequence, block range) of a worker write normalised partial
 //     outputs and natural-log LSE into slot worker + v of the workspace; the
 //     combine kernel merges them.
 //
-// Partial pages: a page with `valid` < 64 tokens is loaded through a 3-D
-// tensor map [pages][64 slots][576] starting at slot valid-64, so the rows
-// before the page are out of bounds and arrive as zeros; pages past the end
-// are loaded entirely out of bounds.  Unused cache slots are never read.
+// Shared memory: Q 72 KB + P 16 KB + QK ring 72 KB + PV ring 64 KB.  Each
+// ring holds one block.  The QK MMA shape the pair split gives, 64 x 128 x 16
+// per SM, costs about as much per instruction as a full-size one.  So the
+// MMA sequence and the one block of ring depth bound this kernel, not HBM.
+//
+// Partial pages: a page with `valid` < 64 tokens starts its boxes at slot
+// valid - 64.  The rows before the page are out of bounds and arrive as
+// zeros, and the cp.async loader shifts its rows the same way.  Pages past
+// the end load entirely out of bounds (slot 64).  Unused cache slots are
+// never read.
 //
 // Every mbarrier wait is bounded (MLA_WAIT_NS); on expiry the kernel raises
 // MLA_ERR_TIMEOUT in the device status, every role leaves its loop, the pair
@@ -57,7 +72,7 @@ constexpr int kPage = 64;          // tokens per page
 constexpr int kBlk = 128;          // tokens per block (two pages)
 constexpr int kChunk = 8192;       // 64 tokens x 64 columns bf16, one swizzled operand tile
 constexpr int kQkChunks = 3;       // chunks per QK stage (one TMA box)
-constexpr int kQkStages = 3;       // QK ring: 3 stages x 3 chunks = one page per block
+constexpr int kQkStages = 3;       // QK ring: 3 stages x 3 chunks = this CTA's page of one block
 constexpr int kQkStageBytes = kQkChunks * kChunk;
 constexpr int kPvStages = 2;       // PV ring: one page's latent half (4 chunks) per stage
 constexpr int kPvStageBytes = 4 * kChunk;
