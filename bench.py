@@ -151,6 +151,24 @@ def _traffic_for(kernel_src_paths):
     return rec.get("dram_bytes_per_call")
 
 
+def max_over_ranks(vals, device=None):
+    """Element-wise maximum of `vals` over all ranks of the default process
+    group (the values themselves when there is no group or one rank)."""
+    import torch
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return [float(v) for v in vals]
+    t = torch.tensor([float(v) for v in vals], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return t.tolist()
+
+
+def whole_job_rate(units_per_rank, world, ms):
+    """Units per second of the whole job: every rank's units over the
+    slowest rank's time (ms)."""
+    return units_per_rank * world / (ms * 1e-3)
+
+
 # ---------------------------------------------------------------------------
 # CPU oracle arm
 # ---------------------------------------------------------------------------
