@@ -64,7 +64,9 @@ def _workload_bytes(w):
 
 
 class ClockSampler:
-    """nvidia-smi samples of SM clock and throttle reasons while running."""
+    """nvidia-smi samples of SM clock and throttle reasons while running.
+    Entering waits for nvidia-smi's first sample; summary() keeps only the
+    samples taken after mark(), i.e. during the timed region."""
 
     Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
          "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
@@ -74,22 +76,29 @@ class ClockSampler:
         self.idx = gpu_index
         self.proc = None
         self.lines = []
+        self.t_mark = 0.0
 
     def __enter__(self):
         try:
             self.proc = subprocess.Popen(
                 ["nvidia-smi", "-i", str(self.idx), f"--query-gpu={self.Q}",
-                 "--format=csv,noheader,nounits", "-lms", "100"],
+                 "--format=csv,noheader,nounits", "-lms", "25"],
                 stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
             self.t = threading.Thread(target=self._read, daemon=True)
             self.t.start()
+            t0 = time.perf_counter()
+            while not self.lines and time.perf_counter() - t0 < 3.0:
+                time.sleep(0.01)
         except Exception:
             self.proc = None
         return self
 
+    def mark(self):
+        self.t_mark = time.perf_counter()
+
     def _read(self):
         for line in self.proc.stdout:
-            self.lines.append(line.strip())
+            self.lines.append((time.perf_counter(), line.strip()))
 
     def __exit__(self, *a):
         if self.proc is not None:
@@ -102,7 +111,9 @@ class ClockSampler:
     def summary(self):
         sm, mx, reasons = [], None, set()
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        for ln in self.lines:
+        for t, ln in self.lines:
+            if t < self.t_mark:
+                continue
             f = [x.strip() for x in ln.split(",")]
             if len(f) < 9:
                 continue
@@ -326,17 +337,6 @@ def run_gpu(args, w):
             dist.barrier()
         return e0.elapsed_time(e1) / K, wall, launches
 
-    with ClockSampler(local) as clk:
-        step_ms, wall, _ = timed(step, args.steps)
-        launches = kernels_per_step * args.steps
-        n_eager = max(3, args.steps // 4)
-        eager_ms, _, eager_launches = timed(eager_step, n_eager)
-        dec_ms, _, dec_launches = timed(decode_only, max(args.steps, 5))
-    clocks = clk.summary()
-    st = B.mla_get_device_status()
-    if st != 0:
-        raise RuntimeError(f"device status after timing: {B.mla_status_string(st)}")
-
     # end to end through the public API with host buffers
     h_host = torch.from_numpy(h_np).to(d.torch_dtype).pin_memory()
     bi_host = torch.from_numpy(bi_np).pin_memory()
@@ -352,7 +352,20 @@ def run_gpu(args, w):
 
     for _ in range(2):
         e2e_step()
-    e2e_ms, _, _ = timed(e2e_step, args.steps)
+    torch.cuda.synchronize(dev)
+
+    with ClockSampler(local) as clk:
+        clk.mark()
+        step_ms, wall, _ = timed(step, args.steps)
+        launches = kernels_per_step * args.steps
+        n_eager = max(3, args.steps // 4)
+        eager_ms, _, eager_launches = timed(eager_step, n_eager)
+        dec_ms, _, dec_launches = timed(decode_only, max(args.steps, 5))
+        e2e_ms, _, _ = timed(e2e_step, args.steps)
+    clocks = clk.summary()
+    st = B.mla_get_device_status()
+    if st != 0:
+        raise RuntimeError(f"device status after timing: {B.mla_status_string(st)}")
     h2d = h_host.numel() * h_host.element_size() + bi_host.numel() * 4 + pos_host.numel() * 4
     d2h = out_host.numel() * 4
 

@@ -1,0 +1,48 @@
+"""Host-side pieces of bench.py that need no GPU: the kernel-code digest that
+decides whether the recorded ncu traffic still applies, the clock-sample
+summary, and the whole-job rate."""
+
+import os
+import sys
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+sys.path.insert(0, ROOT)
+
+import bench  # noqa: E402
+
+
+def test_code_digest_ignores_comments_only(tmp_path):
+    a = tmp_path / "a.cuh"
+    b = tmp_path / "b.cuh"
+    c = tmp_path / "c.cuh"
+    a.write_text("// header\nint f(int x) {  // inline\n  return x + 1;\n}\n")
+    b.write_text("/* another\n   header */\n\nint f(int x) {\n  return x + 1;  // changed note\n}\n")
+    c.write_text("int f(int x) {\n  return x + 2;\n}\n")
+    assert bench.code_digest([str(a)]) == bench.code_digest([str(b)])
+    assert bench.code_digest([str(a)]) != bench.code_digest([str(c)])
+
+
+def test_recorded_traffic_matches_current_decode_source():
+    src = os.path.join(ROOT, "mla_latent_kv_35_b200", "csrc", "decode_tc.cuh")
+    assert bench._traffic_for([src]) is not None
+
+
+def test_clock_summary_uses_samples_after_mark():
+    s = bench.ClockSampler(0)
+    s.lines = [(0.5, "0, 1000, 1965, 100.0, 0x0, Not Active, Not Active, Not Active, Not Active"),
+               (2.0, "0, 1900, 1965, 900.0, 0x4, Not Active, Not Active, Not Active, Active"),
+               (2.1, "0, 1700, 1965, 990.0, 0x4, Not Active, Not Active, Not Active, Active"),
+               (2.2, "0, 1800, 1965, 950.0, 0x0, Not Active, Not Active, Not Active, Not Active")]
+    s.t_mark = 1.0
+    out = s.summary()
+    assert out == {"sm_mhz": 1800.0, "sm_max_mhz": 1965.0, "reasons": ["sw_power_cap"],
+                   "samples": 3}
+    s.t_mark = 5.0
+    assert s.summary()["samples"] == 0
+
+
+def test_whole_job_rate():
+    assert bench.whole_job_rate(128, 1, 1.6) == pytest.approx(80000.0)
+    assert bench.whole_job_rate(128, 8, 1.6) == pytest.approx(640000.0)
