@@ -177,6 +177,43 @@ mla_status mla_decode(const mla_dims* dims, const void* qbuf, const void* pool,
                       void* workspace, size_t ws_bytes, float* o_lat,
                       float* lse, void* stream);
 
+/* A4 + A5 on one contiguous token range of each sequence, for context
+ * parallelism: the token range of a long sequence is split over several
+ * caches (one per GPU), each returns the attention over its range, and
+ * mla_combine_parts merges them.  The pages give the decode ([DF-0], [DF-1]);
+ * the split and merge are an addition of this library.
+ * Cache b here holds seq_lens[b] >= 0 tokens: global tokens
+ * [G_b - seq_tail[b] - seq_lens[b], G_b - seq_tail[b]) of a sequence with G_b
+ * tokens in all, at local positions 0.. in pool/page_table as for mla_decode.
+ * The S_q query tokens are the last S_q of the whole sequence, so query j
+ * sees local token t iff t < seq_lens[b] + seq_tail[b] - S_q + j + 1.
+ * Outputs are those of mla_decode over the visible local tokens; a row that
+ * sees none gets o_lat = 0 and lse = -inf.  seq_tail: device int32 [B],
+ * >= 0; seq_lens[b] may be 0 (this cache holds none of sequence b).  A
+ * negative length or tail, or a length past max_pages*page_size, raises
+ * MLA_ERR_BOUNDS in the device status.  With seq_tail all zero and
+ * seq_lens[b] >= S_q this is mla_decode.  Workspace as for mla_decode. */
+mla_status mla_decode_partial(const mla_dims* dims, const void* qbuf,
+                              const void* pool, int n_pages,
+                              const int32_t* page_table, int max_pages,
+                              const int32_t* seq_lens, const int32_t* seq_tail,
+                              int B, int S_q, int num_workers, void* workspace,
+                              size_t ws_bytes, float* o_lat, float* lse,
+                              void* stream);
+
+/* Merge attention results over disjoint token sets (the log-sum-exp merge of
+ * mla_decode's own split-KV combine, here across callers' parts):
+ *   m = max_p lse_p,  z = sum_p exp(lse_p - m),
+ *   o_lat = sum_p exp(lse_p - m) * o_p / z,  lse = m + ln z,
+ * with parts of lse = -inf contributing nothing and a row with no visible
+ * token in any part giving o_lat = 0, lse = -inf.
+ * o_parts: device fp32 [n_parts][rows][d_latent]; lse_parts: device fp32
+ * [n_parts][rows]; o_lat: device fp32 [rows][d_latent]; lse: device fp32
+ * [rows].  rows = B * S_q * H for mla_decode_partial outputs. */
+mla_status mla_combine_parts(const mla_dims* dims, const float* o_parts,
+                             const float* lse_parts, int n_parts, int rows,
+                             float* o_lat, float* lse, void* stream);
+
 /* A4 + A5 without caller-provided scratch.  The pages have no counterpart
  * for this call; it exists for callers that cannot allocate device memory:
  * code running under a host framework that owns every byte of device memory

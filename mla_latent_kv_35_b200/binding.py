@@ -26,7 +26,8 @@ EXPORTS = ("mla_project", "mla_absorb_q", "mla_rope", "mla_cache_append",
            "mla_decode_workspace_size", "mla_decode", "mla_out_proj_scratch_size",
            "mla_out_proj", "mla_get_device_status", "mla_status_string",
            "mla_launch_count", "mla_selftest_wait_timeout", "mla_get_wait_diag",
-           "mla_decode_noalloc", "mla_pre_attention")
+           "mla_decode_noalloc", "mla_pre_attention", "mla_decode_partial",
+           "mla_combine_parts")
 
 
 class MLAError(RuntimeError):
@@ -95,6 +96,9 @@ _SIGS = {
                             _P], _I),
     "mla_pre_attention": ([ctypes.POINTER(Dims), _P, _I, _P, _P, _P, _P, _P, _I, _P, _I, _I,
                            _P], _I),
+    "mla_decode_partial": ([ctypes.POINTER(Dims), _P, _P, _I, _P, _I, _P, _P, _I, _I, _I, _P,
+                            _Z, _P, _P, _P], _I),
+    "mla_combine_parts": ([ctypes.POINTER(Dims), _P, _P, _I, _I, _P, _P, _P], _I),
 }
 
 
@@ -170,6 +174,23 @@ def mla_pre_attention(dims: MLADims, y, y_stride_tok, w_uk, qbuf, batch_idx, pos
     _check("mla_pre_attention", lib().mla_pre_attention(
         ctypes.byref(dims.c()), _ptr(y), y_stride_tok, _ptr(w_uk), _ptr(qbuf), _ptr(batch_idx),
         _ptr(pos), _ptr(page_table), max_pages, _ptr(pool), n_pages, T, _stream()))
+
+
+def mla_decode_partial(dims: MLADims, qbuf, pool, n_pages, page_table, max_pages, seq_lens,
+                       seq_tail, B, S_q, num_workers, workspace, o_lat, lse):
+    _dev(qbuf, pool, page_table, seq_lens, seq_tail, workspace, o_lat, lse)
+    ws_bytes = workspace.numel() * workspace.element_size()
+    _check("mla_decode_partial", lib().mla_decode_partial(
+        ctypes.byref(dims.c()), _ptr(qbuf), _ptr(pool), n_pages, _ptr(page_table), max_pages,
+        _ptr(seq_lens), _ptr(seq_tail), B, S_q, num_workers, _ptr(workspace), ws_bytes,
+        _ptr(o_lat), _ptr(lse), _stream()))
+
+
+def mla_combine_parts(dims: MLADims, o_parts, lse_parts, n_parts, rows, o_lat, lse):
+    _dev(o_parts, lse_parts, o_lat, lse)
+    _check("mla_combine_parts", lib().mla_combine_parts(
+        ctypes.byref(dims.c()), _ptr(o_parts), _ptr(lse_parts), n_parts, rows, _ptr(o_lat),
+        _ptr(lse), _stream()))
 
 
 def mla_decode_workspace_size(dims: MLADims, B: int, S_q: int, num_workers: int = 0) -> int:

@@ -415,10 +415,11 @@ size_t mla_decode_workspace_size(const mla_dims* dims, int B, int S_q, int num_w
   return decode_layout(dims, B, S_q, num_workers).total;
 }
 
-mla_status mla_decode(const mla_dims* dims, const void* qbuf, const void* pool, int n_pages,
-                      const int32_t* page_table, int max_pages, const int32_t* seq_lens, int B,
-                      int S_q, int num_workers, void* workspace, size_t ws_bytes, float* o_lat,
-                      float* lse, void* stream) {
+static mla_status decode_impl(const mla_dims* dims, const void* qbuf, const void* pool, int n_pages,
+                              const int32_t* page_table, int max_pages, const int32_t* seq_lens,
+                              const int32_t* tail, int B, int S_q, int num_workers,
+                              void* workspace, size_t ws_bytes, float* o_lat, float* lse,
+                              void* stream) {
   if (!dims_ok(dims) || B < 0 || S_q < 1 || S_q > 2 || num_workers < 0 || n_pages < 1 ||
       max_pages < 1)
     return MLA_ERR_INVALID_ARG;
@@ -435,14 +436,14 @@ mla_status mla_decode(const mla_dims* dims, const void* qbuf, const void* pool, 
   float* ws_lse = reinterpret_cast<float*>(ws + L.off_lse);
   float* ws_o = reinterpret_cast<float*>(ws + L.off_o);
   const int max_tokens = max_pages * dims->page_size;
-  plan_kernel<<<1, 1024, 0, st>>>(seq_lens, B, L.R, S_q, max_tokens, kBlockTokens, start);
+  plan_kernel<<<1, 1024, 0, st>>>(seq_lens, tail, B, L.R, S_q, max_tokens, kBlockTokens, start);
   MLA_TRY(check_launch());
   const int H = dims->n_heads, dc = dims->d_latent, dr = dims->d_rope;
   if (use_tc_decode(dims, S_q)) {
     if (!aligned16(qbuf) || !aligned16(pool)) return MLA_ERR_INVALID_ARG;
     MLA_TRY(launch_decode_tc_impl(make_tmap_bf16, qbuf, pool, n_pages, page_table, max_pages,
-                                  seq_lens, B, S_q, H, dims->scale, L.G, start, ws_lse, ws_o,
-                                  st));
+                                  seq_lens, tail, B, S_q, H, dims->scale, L.G, start, ws_lse,
+                                  ws_o, st));
     g_launches.fetch_add(1, std::memory_order_relaxed);
   } else {
     dim3 grid(L.G, (L.rows_per_v + 7) / 8);
@@ -450,8 +451,8 @@ mla_status mla_decode(const mla_dims* dims, const void* qbuf, const void* pool, 
 #define MLA_SIMT_DECODE(T, KC)                                                                 \
   decode_simt_kernel<T, KC><<<grid, 256, 0, st>>>(                                             \
       static_cast<const T*>(qbuf), static_cast<const T*>(pool), n_pages, page_table, max_pages, \
-      seq_lens, B, S_q, H, dc, dr, dims->page_size, dims->scale, L.G, kBlockTokens, start,      \
-      ws_lse, ws_o)
+      seq_lens, tail, B, S_q, H, dc, dr, dims->page_size, dims->scale, L.G, kBlockTokens,       \
+      start, ws_lse, ws_o)
     if (dims->dtype == MLA_F32) {
       if (kc <= 2) MLA_SIMT_DECODE(float, 2);
       else if (kc <= 4) MLA_SIMT_DECODE(float, 4);
@@ -469,6 +470,35 @@ mla_status mla_decode(const mla_dims* dims, const void* qbuf, const void* pool, 
   dim3 cgrid(L.V, (L.rows_per_v + 7) / 8);
   combine_kernel<<<cgrid, 256, 0, st>>>(ws_lse, ws_o, start, L.V, L.R, L.G, L.rows_per_v, dc,
                                         o_lat, lse);
+  return check_launch();
+}
+
+mla_status mla_decode(const mla_dims* dims, const void* qbuf, const void* pool, int n_pages,
+                      const int32_t* page_table, int max_pages, const int32_t* seq_lens, int B,
+                      int S_q, int num_workers, void* workspace, size_t ws_bytes, float* o_lat,
+                      float* lse, void* stream) {
+  return decode_impl(dims, qbuf, pool, n_pages, page_table, max_pages, seq_lens, nullptr, B, S_q,
+                     num_workers, workspace, ws_bytes, o_lat, lse, stream);
+}
+
+mla_status mla_decode_partial(const mla_dims* dims, const void* qbuf, const void* pool,
+                              int n_pages, const int32_t* page_table, int max_pages,
+                              const int32_t* seq_lens, const int32_t* seq_tail, int B, int S_q,
+                              int num_workers, void* workspace, size_t ws_bytes, float* o_lat,
+                              float* lse, void* stream) {
+  if (!seq_tail && B > 0) return MLA_ERR_INVALID_ARG;
+  return decode_impl(dims, qbuf, pool, n_pages, page_table, max_pages, seq_lens, seq_tail, B, S_q,
+                     num_workers, workspace, ws_bytes, o_lat, lse, stream);
+}
+
+mla_status mla_combine_parts(const mla_dims* dims, const float* o_parts, const float* lse_parts,
+                             int n_parts, int rows, float* o_lat, float* lse, void* stream) {
+  if (!dims_ok(dims) || n_parts < 1 || rows < 0) return MLA_ERR_INVALID_ARG;
+  if (rows == 0) return MLA_OK;
+  if (!o_parts || !lse_parts || !o_lat || !lse) return MLA_ERR_INVALID_ARG;
+  cudaStream_t st = as_stream(stream);
+  combine_parts_kernel<<<(unsigned)((rows + 7) / 8), 256, 0, st>>>(
+      o_parts, lse_parts, n_parts, rows, dims->d_latent, o_lat, lse);
   return check_launch();
 }
 

@@ -95,6 +95,7 @@ struct DecodeTcParams {
   const uint8_t* pool;    // [n_pages][64][576] bf16
   const int32_t* page_table;
   const int32_t* seq_lens;
+  const int32_t* tail;    // [B] tokens past this cache's range, or nullptr
   const int32_t* start;   // [V + 1] block prefix sums from plan_kernel
   float* ws_lse;          // [slots][128]
   float* ws_o;            // [slots][128][512]
@@ -432,7 +433,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(dtc::kThreads, 1)
       const int b = v / P.R, rb = v % P.R;
       const int L = P.seq_lens[b];
       const int grow = rb * 128 + 64 * (int)rank + h;      // row within the sequence
-      const int limit = L - P.S_q + grow / P.H + 1;         // visible tokens t < limit
+      const int tl = P.tail != nullptr ? P.tail[b] : 0;
+      const int limit = L + tl - P.S_q + grow / P.H + 1;    // visible tokens t < limit
       float m = -INFINITY, l = 0.f;
       bool o_started = false;
       for (int x = x0; x < x1; ++x, ++j) {
@@ -565,8 +567,8 @@ inline mla_status launch_decode_tc_impl(
     bool (*make_tmap)(CUtensorMap*, const void*, int, const uint64_t*, const uint64_t*,
                       const uint32_t*),
     const void* qbuf, const void* pool, int n_pages, const int32_t* page_table, int max_pages,
-    const int32_t* seq_lens, int B, int S_q, int H, float scale, int G, const int32_t* start,
-    float* ws_lse, float* ws_o, cudaStream_t st) {
+    const int32_t* seq_lens, const int32_t* tail, int B, int S_q, int H, float scale, int G,
+    const int32_t* start, float* ws_lse, float* ws_o, cudaStream_t st) {
   using namespace dtc;
   CUtensorMap tQ, tQK;
   {
@@ -587,6 +589,7 @@ inline mla_status launch_decode_tc_impl(
   p.pool = static_cast<const uint8_t*>(pool);
   p.page_table = page_table;
   p.seq_lens = seq_lens;
+  p.tail = tail;
   p.start = start;
   p.ws_lse = ws_lse;
   p.ws_o = ws_o;

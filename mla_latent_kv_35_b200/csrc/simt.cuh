@@ -130,8 +130,13 @@ __global__ void cast_f32_bf16_kernel(const float* x, __nv_bfloat16* y, long long
 // concatenation, lo_k = floor(k * total / G).  The piece of worker k in v
 // writes partial slot k + v (unique: pieces form a monotone staircase).
 // ---------------------------------------------------------------------------
-__global__ void plan_kernel(const int32_t* seq_lens, int B, int R, int S_q, int max_tokens,
-                            int BLK, int32_t* start) {
+// Block counts per virtual sequence and their exclusive prefix sums.  With
+// `tail` (tokens of the sequence held elsewhere, after this cache's range) a
+// sequence may hold any number of tokens here, none included, since its
+// queries may sit in another cache; without it, it must hold the S_q query
+// tokens.
+__global__ void plan_kernel(const int32_t* seq_lens, const int32_t* tail, int B, int R, int S_q,
+                            int max_tokens, int BLK, int32_t* start) {
   __shared__ int32_t warp_sums[32];
   __shared__ int32_t carry;
   if (threadIdx.x == 0) carry = 0;
@@ -142,7 +147,8 @@ __global__ void plan_kernel(const int32_t* seq_lens, int B, int R, int S_q, int 
     int nb = 0;
     if (v < V) {
       const int L = seq_lens[v / R];
-      if (L < S_q || L > max_tokens) {
+      const int tl = tail != nullptr ? tail[v / R] : 0;
+      if (L < 0 || tl < 0 || L > max_tokens || (tail == nullptr && L < S_q)) {
         if (v % R == 0) raise_flag(kFlagBounds);
       } else {
         nb = (L + BLK - 1) / BLK;
@@ -202,8 +208,9 @@ __device__ __forceinline__ int seq_of_block(const int32_t* start, int V, int x) 
 template <typename T, int kMaxC>
 __global__ void __launch_bounds__(256) decode_simt_kernel(
     const T* qbuf, const T* pool, int n_pages, const int32_t* page_table, int max_pages,
-    const int32_t* seq_lens, int B, int S_q, int H, int d_c, int d_r, int page_size, float scale,
-    int G, int BLK, const int32_t* start, float* ws_lse, float* ws_o) {
+    const int32_t* seq_lens, const int32_t* tail, int B, int S_q, int H, int d_c, int d_r,
+    int page_size, float scale, int G, int BLK, const int32_t* start, float* ws_lse,
+    float* ws_o) {
   const int k = blockIdx.x;
   const int lane = threadIdx.x & 31;
   const int rows = S_q * H;
@@ -221,7 +228,9 @@ __global__ void __launch_bounds__(256) decode_simt_kernel(
     const int x1 = min(hi, start[v + 1]) - start[v];
     if (x1 <= x0) continue;
     const int L = seq_lens[v];
-    const int limit = L - S_q + j + 1;  // visible tokens t < limit
+    // visible tokens t < limit; the query tokens are the last S_q of the
+    // sequence, `tail` of which lie past this cache's range
+    const int limit = L + (tail != nullptr ? tail[v] : 0) - S_q + j + 1;
     const int t0 = x0 * BLK, t1 = min(min(x1 * BLK, L), limit);
     const T* q = qbuf + ((long long)v * rows + r) * D;
     float m = -INFINITY, l = 0.f;
@@ -318,6 +327,40 @@ __global__ void __launch_bounds__(256) combine_kernel(const float* ws_lse, const
 }
 
 // A bounded wait that nothing completes: exercises the timeout path.
+// Merge of partial attention results over disjoint token sets (the parts):
+// one warp per row, parts with lse = -inf (nothing visible) contribute
+// nothing, a row with no visible token anywhere gets o = 0, lse = -inf.
+//   m = max_p lse_p,  z = sum_p e^(lse_p - m),
+//   o = sum_p e^(lse_p - m) o_p / z,  lse = m + ln z.
+__global__ void __launch_bounds__(256) combine_parts_kernel(const float* o_parts,
+                                                            const float* lse_parts, int n_parts,
+                                                            long long rows, int d_c, float* o,
+                                                            float* lse) {
+  const long long r = (long long)blockIdx.x * 8 + (threadIdx.x >> 5);
+  const int lane = threadIdx.x & 31;
+  if (r >= rows) return;
+  float mx = -INFINITY;
+  for (int p = 0; p < n_parts; ++p) mx = fmaxf(mx, lse_parts[p * rows + r]);
+  float* dst = o + r * d_c;
+  if (mx == -INFINITY) {
+    for (int c = lane; c < d_c; c += 32) dst[c] = 0.f;
+    if (lane == 0) lse[r] = -INFINITY;
+    return;
+  }
+  float z = 0.f;
+  for (int p = 0; p < n_parts; ++p) z += __expf(lse_parts[p * rows + r] - mx);
+  const float inv_z = 1.f / z;
+  for (int c = lane; c < d_c; c += 32) {
+    float acc = 0.f;
+    for (int p = 0; p < n_parts; ++p) {
+      const float w = __expf(lse_parts[p * rows + r] - mx) * inv_z;
+      acc = fmaf(w, o_parts[((long long)p * rows + r) * d_c + c], acc);
+    }
+    dst[c] = acc;
+  }
+  if (lane == 0) lse[r] = mx + logf(z);
+}
+
 __global__ void wait_selftest_kernel(unsigned long long wait_ns) {
   __shared__ __align__(8) uint64_t bar;
   if (threadIdx.x == 0) {

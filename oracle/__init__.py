@@ -13,6 +13,7 @@ from .mla_oracle import (  # noqa: F401
     attention_absorbed,
     absorb_query,
     latent_attention,
+    latent_attention_range,
     out_proj,
     decode_step,
     cache_append,

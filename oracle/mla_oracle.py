@@ -212,6 +212,36 @@ def latent_attention(q_abs, C, KR, scale):
     return {"o_lat": o_lat, "lse": lse}
 
 
+def latent_attention_range(q_abs, C_rng, KR_rng, scale, first, total):
+    """latent_attention restricted to one contiguous range of the cache.
+
+    The sequence has ``total`` tokens (its last S_q are the queries, causal as
+    in latent_attention); C_rng [n, d_c] and KR_rng [n, d_r] are its tokens
+    first .. first + n - 1.  Query j sees token t when t <= total - S_q + j.
+    Returns o_lat and lse over the visible tokens of the range; a row that
+    sees none of them gets o_lat = 0 and lse = -inf.  Merging the ranges of a
+    partition of the sequence with combine_splits gives latent_attention of
+    the whole sequence (the softmax normalisation splits over disjoint token
+    sets, the same identity the split-KV merge rests on).
+    """
+    q_abs = np.asarray(q_abs, dtype=F64)
+    C_rng = np.asarray(C_rng, dtype=F64)
+    KR_rng = np.asarray(KR_rng, dtype=F64)
+    S_q, H, _ = q_abs.shape
+    n, d_c = C_rng.shape
+    o_lat = np.zeros((S_q, H, d_c))
+    lse = np.full((S_q, H), -np.inf)
+    for j in range(S_q):
+        last_visible = total - S_q + j          # global index
+        vis = min(n, max(0, last_visible - first + 1))
+        if vis == 0:
+            continue
+        for i in range(H):
+            s = scale * (C_rng[:vis] @ q_abs[j, i, :d_c] + KR_rng[:vis] @ q_abs[j, i, d_c:])
+            _, o_lat[j, i], lse[j, i] = _softmax_attend(s, C_rng[:vis])
+    return {"o_lat": o_lat, "lse": lse}
+
+
 def out_proj(o_lat, W_UV, W_O):
     """Output side with W_UV folded in: o_i = W_UV[i] o_lat_i, then
     out = W_O [o_1; ...; o_H].  o_lat [T, H, d_c] -> (o [T, H, d_v], out [T, d_model])."""

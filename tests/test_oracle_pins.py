@@ -283,6 +283,31 @@ def test_combine_splits_equals_full():
     np.testing.assert_allclose(o2, full["o_lat"], atol=1e-15)
 
 
+def test_range_partition_merges_to_full():
+    """Range attention of a partition of the sequence, merged, is the whole
+    sequence's attention; the causal cut falls inside the last ranges."""
+    rng = np.random.default_rng(17)
+    S_q, H, L, d_c, d_r = 2, 3, 40, 6, 4
+    q = rng.standard_normal((S_q, H, d_c + d_r))
+    C = rng.standard_normal((L, d_c))
+    KR = rng.standard_normal((L, d_r))
+    full = oracle.latent_attention(q, C, KR, 0.4)
+    for cuts in ([0, 7, 8, 39, 40], [0, 20, 38, 40], [0, 40], [0, 1, 2, 39, 40]):
+        parts = [oracle.latent_attention_range(q, C[a:b], KR[a:b], 0.4, a, L)
+                 for a, b in zip(cuts[:-1], cuts[1:])]
+        o, lse = oracle.combine_splits([r["o_lat"] for r in parts], [r["lse"] for r in parts])
+        np.testing.assert_allclose(o, full["o_lat"], atol=1e-12)
+        np.testing.assert_allclose(lse, full["lse"], atol=1e-12)
+    # the last token is the second query: query 0 sees nothing in [39, 40)
+    last = oracle.latent_attention_range(q, C[39:], KR[39:], 0.4, 39, L)
+    assert np.all(last["lse"][0] == -np.inf) and np.all(last["o_lat"][0] == 0)
+    assert np.all(np.isfinite(last["lse"][1]))
+    # a single visible token: its own latent, lse = its score
+    np.testing.assert_allclose(last["o_lat"][1], np.broadcast_to(C[39], (H, d_c)), atol=1e-15)
+    s = 0.4 * (q[1, :, :d_c] @ C[39] + q[1, :, d_c:] @ KR[39])
+    np.testing.assert_allclose(last["lse"][1], s, atol=1e-12)
+
+
 def test_cache_append_scatter():
     rng = np.random.default_rng(10)
     pool = np.full((6, 4, 5), 0xFFFF, dtype=np.uint16)
