@@ -3,7 +3,8 @@
 Decode sequences are independent, so N GPUs run N shards of one batch with no
 data-path collective (weak scaling).  What needs checking without GPUs:
 each rank draws its own global sequences, the shards tile the whole batch,
-and the timing reduction takes the slowest rank.
+the timing reduction takes the slowest rank, and a rank that leaves makes the
+others' next collective end with an error instead of waiting for good.
 """
 
 import os
@@ -127,3 +128,47 @@ def test_two_rank_gloo_reduction_and_sharding():
         # 4 tokens per rank, 2 ranks, slowest rank 2 ms
         assert rate == pytest.approx(4 * 2 / 2e-3)
     assert res[0][1] == res[1][1]
+
+
+def _failing_rank_main(rank, world, port, out):
+    import datetime
+    import time
+    import torch.distributed as dist
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=world,
+                            timeout=datetime.timedelta(seconds=5))
+    import bench
+    if rank == 1:
+        # this rank fails between steps and never reaches the collective
+        out[rank] = "left"
+        time.sleep(8)
+        os._exit(3)
+    t0 = time.time()
+    try:
+        bench.max_over_ranks([1.0])
+        out[rank] = "returned"
+    except Exception as e:  # the collective must end with an error, not hang
+        out[rank] = ("error", type(e).__name__, time.time() - t0)
+    os._exit(0)
+
+
+def test_rank_that_leaves_ends_the_others_collective_with_an_error():
+    world = 2
+    port = _free_port()
+    ctx = mp.get_context("spawn")
+    with ctx.Manager() as m:
+        out = m.dict()
+        procs = [ctx.Process(target=_failing_rank_main, args=(r, world, port, out))
+                 for r in range(world)]
+        for p in procs:
+            p.start()
+        for p in procs:
+            p.join(60)
+        alive = [p.is_alive() for p in procs]
+        for p in procs:
+            if p.is_alive():
+                p.kill()
+        res = dict(out)
+    assert alive == [False, False]
+    assert res[1] == "left"
+    assert res[0][0] == "error" and res[0][2] < 30, res[0]
