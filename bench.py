@@ -161,6 +161,18 @@ def _traffic_for(kernel_src_paths):
     return rec.get("dram_bytes_per_call")
 
 
+def run_config(w, workload_name, world):
+    """The JSON line's `config`, shared by both arms."""
+    _, _, cache_bytes = _workload_bytes(w)
+    return {"workload": workload_name, "batch_per_gpu": w.B, "global_batch": w.B * world,
+            "heads": w.H, "context": w.ctx[0] if len(set(w.ctx)) == 1 else "ragged",
+            "S_q": w.S_q, "latent": w.d_latent, "rope": w.d_rope, "page": w.page_size,
+            "d_model": w.d_model,
+            "l2": "inputs larger than L2 (cache %.2f GB), no flush" % (cache_bytes / 1e9),
+            "parallelism": (f"dp{world}: independent sequence shards, no collective"
+                            if world > 1 else "single GPU")}
+
+
 def max_over_ranks(vals, device=None):
     """Element-wise maximum of `vals` over all ranks of the default process
     group (the values themselves when there is no group or one rank)."""
@@ -227,8 +239,7 @@ def run_reference(args, w):
         "warmup": args.warmup, "ms_per_step": 1000.0 * w.T / value,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
         "data": "synthetic",
-        "config": {"workload": w.name, "batch": w.B, "heads": w.H, "context": w.ctx[0],
-                   "S_q": w.S_q, "latent": w.d_latent, "rope": w.d_rope},
+        "config": run_config(w, w.name, args.gpus),
         "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": cores, "kind": "oracle",
                          "sample": sample},
         "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0,
@@ -391,15 +402,7 @@ def run_gpu(args, w):
         "vs_baseline": None,
         "dtype": "bf16" if w.dtype == "bf16" else "f32",
         "data": "synthetic",
-        "config": {"workload": workload_name, "batch_per_gpu": w.B,
-                   "global_batch": w.B * world,
-                   "heads": w.H,
-                   "context": w.ctx[0] if len(set(w.ctx)) == 1 else "ragged",
-                   "S_q": w.S_q, "latent": w.d_latent, "rope": w.d_rope,
-                   "page": w.page_size, "d_model": w.d_model,
-                   "l2": "inputs larger than L2 (cache %.2f GB), no flush" % (cache_bytes / 1e9),
-                   "parallelism": (f"dp{world}: independent sequence shards, no collective"
-                                   if world > 1 else "single GPU")},
+        "config": run_config(w, workload_name, world),
         "decode": {"ms": t_dec, "tokens_per_s": whole_job_rate(w.T, world, t_dec),
                    "cache_gb_per_s": cache_bytes / (t_dec * 1e-3) / 1e9,
                    "tflops": flops / (t_dec * 1e-3) / 1e12,
