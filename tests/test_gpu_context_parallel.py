@@ -141,3 +141,37 @@ def test_decode_context_parallel_through_nccl_one_rank():
         ref = _decode_ref(d, c, b)
         check(to_np(o)[b], ref["o_lat"], "bf16", f"o_lat b={b}")
         check(to_np(lse)[b], ref["lse"], "bf16", f"lse b={b}")
+
+
+@gpu
+def test_full_size_context_over_eight_ranks():
+    """Two 131072-token sequences (two speculative query tokens) split over 8
+    emulated ranks, merged, against mla_decode on the whole cache."""
+    rng = torch.Generator(device="cpu").manual_seed(31)
+    d = B.MLADims(128, 128, 512, 64, 128, 5120, 64, 192 ** -0.5, 10000.0, "bf16")
+    lens, S_q, world, Bn = [131072, 131071], 2, 8, 2
+    maxp = 131072 // 64
+    n_pages = Bn * maxp + 1
+    perm = torch.randperm(Bn * maxp, generator=rng).to(torch.int32).reshape(Bn, maxp)
+    pool = torch.randn((n_pages, 64, 576), generator=rng).to(DEV, torch.bfloat16)
+    qb = torch.randn((Bn, S_q, 128, 576), generator=rng).to(DEV, torch.bfloat16)
+    table = perm.numpy()
+    c = {"table": table, "qb": None, "pool_d": pool, "n_pages": n_pages, "maxp": maxp}
+    ws = torch.empty((B.mla_decode_workspace_size(d, Bn, S_q, 0),), dtype=torch.uint8, device=DEV)
+    o_parts = torch.empty((world, Bn, S_q, 128, 512), device=DEV)
+    l_parts = torch.empty((world, Bn, S_q, 128), device=DEV)
+    for r, (tab, n_loc, tail) in enumerate(_rank_tables(c, lens, world)):
+        B.mla_decode_partial(d, qb, pool, n_pages, torch.from_numpy(tab).to(DEV), maxp,
+                             torch.from_numpy(n_loc).to(DEV), torch.from_numpy(tail).to(DEV),
+                             Bn, S_q, 0, ws, o_parts[r], l_parts[r])
+    o = torch.empty((Bn, S_q, 128, 512), device=DEV)
+    lse = torch.empty((Bn, S_q, 128), device=DEV)
+    B.mla_combine_parts(d, o_parts, l_parts, world, Bn * S_q * 128, o, lse)
+    o_full = torch.empty_like(o)
+    l_full = torch.empty_like(lse)
+    B.mla_decode(d, qb, pool, n_pages, torch.from_numpy(table).to(DEV), maxp,
+                 torch.tensor(lens, dtype=torch.int32, device=DEV), Bn, S_q, 0, ws, o_full, l_full)
+    assert status() == 0
+    # both are bf16-P decodes of the same data with different splits
+    check(to_np(o), to_np(o_full).astype(np.float64), "bf16", "o_lat vs whole-cache decode")
+    check(to_np(lse), to_np(l_full).astype(np.float64), "bf16", "lse vs whole-cache decode")
