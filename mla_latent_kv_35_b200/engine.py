@@ -80,8 +80,10 @@ class MLADecodeLayer:
     # ------------------------------------------------------------------
     # step buffers
     # ------------------------------------------------------------------
-    def buffers(self, B: int, S_q: int, num_workers: int = 0):
-        key = (B, S_q, num_workers)
+    def buffers(self, B: int, S_q: int, num_workers: int = 0, slot: int = 0):
+        """Device buffers of one step (slot: an independent second set, for
+        steps that overlap in DecodePipeline)."""
+        key = (B, S_q, num_workers, slot)
         if key not in self._bufs:
             d = self.dims
             T = B * S_q
@@ -103,7 +105,7 @@ class MLADecodeLayer:
     # the hot path
     # ------------------------------------------------------------------
     def step(self, h, batch_idx, pos, B: int, S_q: int, num_workers: int = 0,
-             fused: bool = True):
+             fused: bool = True, slot: int = 0):
         """h [T, d_model] device (dims dtype), batch_idx/pos int32 [T] device,
         T = B*S_q tokens b-major.  Returns the dict of step buffers.
 
@@ -112,7 +114,7 @@ class MLADecodeLayer:
         d = self.dims
         H, dn, dc, dr = d.n_heads, d.d_nope, d.d_latent, d.d_rope
         T = B * S_q
-        bf = self.buffers(B, S_q, num_workers)
+        bf = self.buffers(B, S_q, num_workers, slot)
         y, qbuf = bf["y"], bf["qbuf"]
         Y, D, dqk = self.Y, self.D, self.dqk
         _b.mla_project(d, h, self.W_A0, y, T, d.d_model, Y)                        # A0
@@ -135,7 +137,7 @@ class MLADecodeLayer:
         return bf
 
     def capture(self, h, batch_idx, pos, B: int, S_q: int, num_workers: int = 0,
-                fused: bool = True):
+                fused: bool = True, slot: int = 0):
         """Capture one step on these input buffers into a CUDA graph.
 
         Returns (graph, buffers, kernels): graph.replay() reruns the whole
@@ -145,15 +147,85 @@ class MLADecodeLayer:
         step's buffers are allocated before capture, so the graph holds no
         memory of its own.
         """
-        bf = self.buffers(B, S_q, num_workers)
+        bf = self.buffers(B, S_q, num_workers, slot)
         torch.cuda.synchronize(self.device)
         graph = torch.cuda.CUDAGraph()
         l0 = _b.mla_launch_count()
         with torch.cuda.graph(graph):
-            self.step(h, batch_idx, pos, B, S_q, num_workers, fused)
+            self.step(h, batch_idx, pos, B, S_q, num_workers, fused, slot)
         kernels = _b.mla_launch_count() - l0
         return graph, bf, kernels
 
+
+
+class DecodePipeline:
+    """A decode loop that overlaps each step's host transfers with compute.
+
+    Two slots, each with its own input buffers, step buffers and CUDA graph
+    of the whole step.  submit() enqueues step i in slot i % 2: the inputs
+    are copied from pinned host memory on an upload stream while the
+    previous step computes, the graph replays on the current stream once its
+    inputs are in (and the slot's previous output has left), and the output
+    is copied back on a download stream while the next step computes.  Every
+    step still moves its own inputs in and its own output out.
+    """
+
+    def __init__(self, layer: MLADecodeLayer, B: int, S_q: int, num_workers: int = 0,
+                 fused: bool = True):
+        d = layer.dims
+        dev = layer.device
+        T = B * S_q
+        self.layer = layer
+        self.up = torch.cuda.Stream(dev)
+        self.down = torch.cuda.Stream(dev)
+        self.slots = []
+        for s in range(2):
+            h = torch.zeros((T, d.d_model), dtype=d.torch_dtype, device=dev)
+            bi = torch.zeros((T,), dtype=torch.int32, device=dev)
+            pos = torch.zeros((T,), dtype=torch.int32, device=dev)
+            graph, bf, kernels = layer.capture(h, bi, pos, B, S_q, num_workers, fused, slot=s)
+            self.slots.append(dict(h=h, bi=bi, pos=pos, graph=graph, out=bf["out"],
+                                   inputs_in=torch.cuda.Event(), done=torch.cuda.Event(),
+                                   out_read=torch.cuda.Event()))
+        self.kernels_per_step = kernels
+        self.i = 0
+
+    def submit(self, h_host, bi_host, pos_host, out_host):
+        """Enqueue one step: h_host [T, d_model], bi_host/pos_host int32 [T]
+        and out_host fp32 [T, d_model] are pinned host tensors; out_host
+        holds the step's output once the step's `out_read` event has
+        completed (after wait(), at the latest)."""
+        sl = self.slots[self.i % 2]
+        self.i += 1
+        compute = torch.cuda.current_stream(self.layer.device)
+        # the slot's inputs are free once its previous step has run
+        self.up.wait_event(sl["done"])
+        with torch.cuda.stream(self.up):
+            sl["h"].copy_(h_host, non_blocking=True)
+            sl["bi"].copy_(bi_host, non_blocking=True)
+            sl["pos"].copy_(pos_host, non_blocking=True)
+            sl["inputs_in"].record(self.up)
+        compute.wait_event(sl["inputs_in"])
+        compute.wait_event(sl["out_read"])
+        sl["graph"].replay()
+        sl["done"].record(compute)
+        self.down.wait_event(sl["done"])
+        with torch.cuda.stream(self.down):
+            out_host.copy_(sl["out"], non_blocking=True)
+            sl["out_read"].record(self.down)
+        return sl["out_read"]
+
+    def drain(self, stream=None):
+        """Make `stream` (default: the current one) wait for every submitted
+        step's output transfer."""
+        stream = stream or torch.cuda.current_stream(self.layer.device)
+        for sl in self.slots:
+            stream.wait_event(sl["out_read"])
+
+    def wait(self):
+        """Block the host until every submitted step's output is on the host."""
+        for sl in self.slots:
+            sl["out_read"].synchronize()
 
 
 def build_pool_host(w, page_table, n_pages, prior_bits, canary=0xFFFF):

@@ -160,3 +160,33 @@ def test_graph_replay_matches_eager_step():
     same(bf, eager2)
     assert not torch.equal(eager2["o_lat"], eager["o_lat"])
     del graph
+
+
+@gpu
+def test_pipeline_matches_eager_steps():
+    """DecodePipeline (two slots, uploads and downloads on side streams)
+    gives every step the output the eager step gives for the same inputs."""
+    from mla_latent_kv_35_b200.engine import DecodePipeline
+    w = wl.workload("dsv2", B=6, ctx=(900, 64, 65, 3000, 129, 7))
+    d = B.MLADims.of(w)
+    layer = MLADecodeLayer(d, wl.draw_weights(w), DEV)
+    table, n_pages = wl.page_layout(w)
+    layer.set_cache(pool_to_device(build_pool_host_drawn(w, table, n_pages), w.dtype, DEV),
+                    torch.from_numpy(table).to(DEV),
+                    torch.tensor(w.ctx, dtype=torch.int32, device=DEV))
+    bi_np, pos_np = wl.positions(w)
+    h0 = torch.from_numpy(wl.draw_h_new(w).reshape(w.T, w.d_model)).to(d.torch_dtype)
+    inputs = [(h0 * (1.0 + 0.25 * k)).to(d.torch_dtype).pin_memory() for k in range(5)]
+    bi_h = torch.from_numpy(bi_np).pin_memory()
+    pos_h = torch.from_numpy(pos_np).pin_memory()
+    pipe = DecodePipeline(layer, w.B, w.S_q)
+    outs = [torch.full((w.T, w.d_model), float("nan")).pin_memory() for _ in inputs]
+    for x, o in zip(inputs, outs):
+        pipe.submit(x, bi_h, pos_h, o)
+    pipe.wait()
+    assert status() == 0
+    for k, x in enumerate(inputs):
+        ref = layer.step(x.to(DEV), bi_h.to(DEV), pos_h.to(DEV), w.B, w.S_q)["out"].cpu()
+        err = float((outs[k] - ref).abs().max())
+        assert err <= 1e-5 * max(1.0, float(ref.abs().max())), (k, err)
+    assert not torch.equal(outs[0], outs[1])
