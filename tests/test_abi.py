@@ -78,3 +78,32 @@ def test_workspace_sizes_grow_with_work(lib):
     f32 = _dims(dtype="f32", n_heads=8, d_nope=32, d_latent=64, d_rope=16, d_v=32,
                 d_model=256)
     assert B.mla_out_proj_scratch_size(f32, 2) >= 2 * 8 * 32 * 4
+
+
+def test_header_is_plain_c_and_a_c_program_links(tmp_path, lib):
+    """include/mla.h compiles as pedantic C99 and a C program links against
+    libmla_b200.so and calls it (host-only calls: no GPU needed)."""
+    import shutil
+    import subprocess
+    cc = shutil.which("gcc") or shutil.which("cc")
+    if cc is None:
+        pytest.skip("no C compiler")
+    src = tmp_path / "probe.c"
+    src.write_text(
+        "#include <stdio.h>\n#include \"mla.h\"\n"
+        "int main(void) {\n"
+        "  mla_dims d = {128, 128, 512, 64, 128, 5120, 64, 0.0721687836f, 10000.0f, MLA_BF16};\n"
+        "  printf(\"%s|%zu\\n\", mla_status_string(MLA_ERR_BOUNDS),\n"
+        "         mla_decode_workspace_size(&d, 128, 1, 74));\n"
+        "  return 0;\n}\n")
+    libdir = os.path.dirname(B.LIB_PATH)
+    exe = tmp_path / "probe"
+    r = subprocess.run([cc, "-std=c99", "-Wall", "-Wextra", "-pedantic", "-Werror",
+                        "-I", os.path.join(ROOT, "include"), str(src), "-L", libdir,
+                        "-lmla_b200", f"-Wl,-rpath,{libdir}", "-o", str(exe)],
+                       capture_output=True, text=True)
+    assert r.returncode == 0, r.stderr
+    out = subprocess.run([str(exe)], capture_output=True, text=True,
+                         check=True).stdout.strip().split("|")
+    assert out[0] == B.mla_status_string(5)
+    assert int(out[1]) == B.mla_decode_workspace_size(_dims(), 128, 1, 74)
