@@ -178,7 +178,7 @@ def max_over_ranks(vals, device=None):
     group (the values themselves when there is no group or one rank)."""
     import torch
     import torch.distributed as dist
-    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+    if not (dist.is_available() and dist.is_initialized()):
         return [float(v) for v in vals]
     t = torch.tensor([float(v) for v in vals], dtype=torch.float64, device=device)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
@@ -263,9 +263,11 @@ def run_gpu(args, w):
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
+    # launched by torchrun (any world size): one NCCL process group
+    distributed = "WORLD_SIZE" in os.environ
     torch.cuda.set_device(local)
     dev = torch.device("cuda", local)
-    if world > 1:
+    if distributed:
         import datetime
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
                                 device_id=dev)
@@ -274,7 +276,7 @@ def run_gpu(args, w):
     w = wl.shard(w, rank, world)
     if rank == 0:
         _build.build()
-    if world > 1:
+    if distributed:
         dist.barrier()
     B.lib()
 
@@ -333,7 +335,7 @@ def run_gpu(args, w):
         the mean ms per call, the wall time and this process's kernel
         launches."""
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        if world > 1:
+        if distributed:
             dist.barrier()
         torch.cuda.synchronize(dev)
         l0 = B.mla_launch_count()
@@ -347,7 +349,7 @@ def run_gpu(args, w):
         torch.cuda.synchronize(dev)
         wall = time.perf_counter() - t0
         launches = B.mla_launch_count() - l0
-        if world > 1:
+        if distributed:
             dist.barrier()
         return e0.elapsed_time(e1) / K, wall, launches
 
@@ -439,7 +441,7 @@ def run_gpu(args, w):
     if rank == 0:
         print(json.dumps(line), flush=True)
     del graph, pipe
-    if world > 1:
+    if distributed:
         dist.barrier()
         dist.destroy_process_group()
 
