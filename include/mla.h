@@ -34,10 +34,14 @@
  *     the pool, a bounded wait that ran out) set a per-device status word
  *     that mla_get_device_status reads and clears; the offending access is
  *     skipped, never performed.
- *   - The library allocates no device memory except the 4-byte status word
- *     per device; scratch space is passed in by the caller.
- *   - Calls are stateless apart from a host-side cache of TMA descriptors;
- *     calls on different streams may run concurrently.
+ *   - The library allocates no device memory at run time.  Its only device
+ *     state is a few static words per device (status, wait diagnostics) and
+ *     the fixed scratch array of mla_decode_noalloc.  Callers pass in every
+ *     other buffer.
+ *   - Calls keep no host state beyond a launch counter: TMA descriptors are
+ *     encoded for each call and passed by value to the kernels.  Calls on
+ *     different streams and host threads may run concurrently, except
+ *     mla_decode_noalloc, whose calls share one scratch array.
  */
 #ifndef MLA_B200_H
 #define MLA_B200_H
