@@ -152,6 +152,24 @@ mla_status mla_pre_attention(const mla_dims* dims, void* y, int y_stride_tok,
                              const int32_t* page_table, int max_pages,
                              void* pool, int n_pages, int T, void* stream);
 
+/* Which split kernel mla_decode runs for these dims (a plain query of the
+ * dispatch, for tests and benchmarks; nothing is launched). */
+typedef enum {
+  MLA_DECODE_KERNEL_SIMT = 0,  /* CUDA-core kernel (fp32, and bf16 shapes the
+                                  tensor-core kernel does not cover) */
+  MLA_DECODE_KERNEL_TC = 1     /* tcgen05 tensor-core kernel */
+} mla_decode_kernel;
+
+/* For query blocks of S_q tokens and num_workers split workers (0 = the
+ * default): *kernel receives an mla_decode_kernel value, *block_tokens the
+ * number of cache tokens per work block, *workers the number of split
+ * workers the planner uses (worker k takes blocks [k*total/workers,
+ * (k+1)*total/workers) of all sequences' blocks in order).  Any output
+ * pointer may be NULL.  Returns MLA_ERR_INVALID_ARG for bad dims or S_q
+ * outside [1, 2]. */
+mla_status mla_decode_config(const mla_dims* dims, int S_q, int num_workers,
+                             int* kernel, int* block_tokens, int* workers);
+
 /* Workspace bytes mla_decode needs for B sequences of S_q query tokens and
  * num_workers split workers (0 = the default mla_decode would pick). */
 size_t mla_decode_workspace_size(const mla_dims* dims, int B, int S_q,
@@ -239,6 +257,9 @@ mla_status mla_combine_parts(const mla_dims* dims, const float* o_parts,
  * one array, so calls whose kernels overlap on the GPU (different streams
  * without ordering) race on it.  The call itself allocates nothing. */
 #define MLA_NOALLOC_SCRATCH_BYTES (64u << 20)
+/* The size of that array in bytes, as the library was built
+ * (MLA_NOALLOC_SCRATCH_BYTES of its own copy of this header). */
+size_t mla_decode_noalloc_scratch_bytes(void);
 mla_status mla_decode_noalloc(const mla_dims* dims, const void* qbuf,
                               const void* pool, int n_pages,
                               const int32_t* page_table, int max_pages,

@@ -27,7 +27,7 @@ EXPORTS = ("mla_project", "mla_absorb_q", "mla_rope", "mla_cache_append",
            "mla_out_proj", "mla_get_device_status", "mla_status_string",
            "mla_launch_count", "mla_selftest_wait_timeout", "mla_get_wait_diag",
            "mla_decode_noalloc", "mla_pre_attention", "mla_decode_partial",
-           "mla_combine_parts")
+           "mla_combine_parts", "mla_decode_config", "mla_decode_noalloc_scratch_bytes")
 
 
 class MLAError(RuntimeError):
@@ -99,7 +99,12 @@ _SIGS = {
     "mla_decode_partial": ([ctypes.POINTER(Dims), _P, _P, _I, _P, _I, _P, _P, _I, _I, _I, _P,
                             _Z, _P, _P, _P], _I),
     "mla_combine_parts": ([ctypes.POINTER(Dims), _P, _P, _I, _I, _P, _P, _P], _I),
+    "mla_decode_config": ([ctypes.POINTER(Dims), _I, _I, ctypes.POINTER(_I),
+                           ctypes.POINTER(_I), ctypes.POINTER(_I)], _I),
+    "mla_decode_noalloc_scratch_bytes": ([], _Z),
 }
+
+DECODE_KERNEL_SIMT, DECODE_KERNEL_TC = 0, 1
 
 
 def lib():
@@ -207,7 +212,18 @@ def mla_decode(dims: MLADims, qbuf, pool, n_pages, page_table, max_pages, seq_le
         _stream()))
 
 
-NOALLOC_SCRATCH_BYTES = 64 << 20
+def mla_decode_config(dims: MLADims, S_q: int, num_workers: int = 0):
+    """(kernel, block_tokens, workers) mla_decode uses for these dims."""
+    k, bt, g = _I(), _I(), _I()
+    _check("mla_decode_config", lib().mla_decode_config(
+        ctypes.byref(dims.c()), S_q, num_workers, ctypes.byref(k), ctypes.byref(bt),
+        ctypes.byref(g)))
+    return k.value, bt.value, g.value
+
+
+def mla_decode_noalloc_scratch_bytes() -> int:
+    """Size of the library's built-in decode scratch array."""
+    return int(lib().mla_decode_noalloc_scratch_bytes())
 
 
 def mla_decode_noalloc(dims: MLADims, qbuf, pool, n_pages, page_table, max_pages, seq_lens,

@@ -410,6 +410,16 @@ mla_status mla_pre_attention(const mla_dims* dims, void* y, int y_stride_tok, co
                         D, (long long)H * D, 1, kOutBf16, as_stream(stream), &aux);
 }
 
+mla_status mla_decode_config(const mla_dims* dims, int S_q, int num_workers, int* kernel,
+                             int* block_tokens, int* workers) {
+  if (!dims_ok(dims) || S_q < 1 || S_q > 2 || num_workers < 0) return MLA_ERR_INVALID_ARG;
+  const DecodeLayout L = decode_layout(dims, 1, S_q, num_workers);
+  if (kernel) *kernel = use_tc_decode(dims, S_q) ? MLA_DECODE_KERNEL_TC : MLA_DECODE_KERNEL_SIMT;
+  if (block_tokens) *block_tokens = kBlockTokens;
+  if (workers) *workers = L.G;
+  return MLA_OK;
+}
+
 size_t mla_decode_workspace_size(const mla_dims* dims, int B, int S_q, int num_workers) {
   if (!dims_ok(dims) || B < 0 || S_q < 1 || num_workers < 0) return 0;
   return decode_layout(dims, B, S_q, num_workers).total;
@@ -582,6 +592,10 @@ mla_status noalloc_scratch_address(void** out) {
 }
 
 }  // namespace
+
+extern "C" size_t mla_decode_noalloc_scratch_bytes(void) {
+  return (size_t)MLA_NOALLOC_SCRATCH_BYTES;
+}
 
 extern "C" mla_status mla_decode_noalloc(const mla_dims* dims, const void* qbuf,
                                          const void* pool, int n_pages,

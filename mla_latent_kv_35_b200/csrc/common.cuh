@@ -112,6 +112,21 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatil
   }
 }
 
+// Wait for phase `parity` for at most `ns` nanoseconds, ignoring the abort
+// flag and raising nothing: the drain a role runs after giving up, so that
+// copies or MMAs it already issued finish before the CTA exits.
+__device__ __forceinline__ bool mbar_wait_bounded(uint32_t bar, uint32_t parity, uint64_t ns) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const uint64_t t0 = globaltimer();
+  while (!mbar_try_wait(bar, parity))
+    if (globaltimer() - t0 > ns) return false;
+  return true;
+}
+
+// Bound of each drain wait on the way out after a timeout (2 ms: far above
+// the latency of any copy or MMA still in flight).
+constexpr uint64_t kDrainNs = 2000000ull;
+
 // ---------------------------------------------------------------------------
 // Cluster helpers
 // ---------------------------------------------------------------------------

@@ -54,8 +54,11 @@
 // never read.
 //
 // Every mbarrier wait is bounded (MLA_WAIT_NS); on expiry the kernel raises
-// MLA_ERR_TIMEOUT in the device status, every role leaves its loop, the pair
-// meets at a final cluster barrier and frees its TMEM.
+// MLA_ERR_TIMEOUT in the device status and every role leaves its loop.  On
+// the way out the leader's producer waits (bounded) for the boxes it armed
+// and its MMA thread for a last commit, the loader warps for their own
+// cp.async; then the pair meets at a final cluster barrier and frees its
+// TMEM.
 #pragma once
 
 #include "common.cuh"
@@ -179,7 +182,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(dtc::kThreads, 1)
   extern __shared__ uint8_t smem_raw[];
   __shared__ __align__(8) uint64_t qk_full[kQkStages], qk_empty[kQkStages];
   __shared__ __align__(8) uint64_t pv_full[kPvStages], pv_empty[kPvStages];
-  __shared__ __align__(8) uint64_t q_full, q_empty, o_empty, p_full, pv_done;
+  __shared__ __align__(8) uint64_t q_full, q_empty, o_empty, p_full, pv_done, mma_drain;
   __shared__ __align__(8) uint64_t s_full[2];
   __shared__ float red_max[2][2][64];
   __shared__ float red_sum[2][64];
@@ -211,6 +214,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(dtc::kThreads, 1)
     mbar_init(smem_u32(&o_empty), 8);        // 4 softmax warps x 2 CTAs
     mbar_init(smem_u32(&p_full), 8);
     mbar_init(smem_u32(&pv_done), 1);
+    mbar_init(smem_u32(&mma_drain), 1);
     mbar_init(smem_u32(&s_full[0]), 1);
     mbar_init(smem_u32(&s_full[1]), 1);
     fence_mbar_init();
@@ -241,6 +245,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(dtc::kThreads, 1)
     PieceIter pi;
     pi.init(P.start, V, lo, hi);
     int v, x0, x1, piece = 0;
+    uint32_t q_issued = 0;
     bool ok = true;
     while (ok && pi.next(v, x0, x1)) {
       const int b = v / P.R, rb = v % P.R;
@@ -254,6 +259,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(dtc::kThreads, 1)
       const int row0 = b * rows_seq + rb * 128 + 64 * (int)rank;
       for (int c = 0; c < 9; ++c)
         tma_load_2d_pair(sQ + c * kChunk, &tmQ, c * 64, row0, lead_qfull);
+      ++q_issued;
       for (int x = x0; x < x1 && ok; ++x) {
         int page, slot0;
         page_of(P, b, L, x, (int)rank, page, slot0);
@@ -271,11 +277,16 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(dtc::kThreads, 1)
       }
       ++piece;
     }
-    if (!ok) {
-      // give copies already issued time to land before the CTA can exit
-      const uint64_t t0 = globaltimer();
-      while (globaltimer() - t0 < 50000ull) {
-      }
+    if (!ok && rank == 0) {
+      // Leaving early: wait (bounded) until the boxes already issued have
+      // landed, so that no copy writes into this pair's shared memory after
+      // it exits.  Only the leader's barriers count bytes; they count both
+      // CTAs' boxes of a stage, and the peer waits for the leader at the
+      // final cluster barrier.  A stage the peer never issued cannot
+      // complete, so each wait is bounded on its own.
+      for (uint32_t i = it > (uint32_t)kQkStages ? it - kQkStages : 0u; i < it; ++i)
+        mbar_wait_bounded(smem_u32(&qk_full[i % kQkStages]), (i / kQkStages) & 1, kDrainNs);
+      if (q_issued > 0) mbar_wait_bounded(smem_u32(&q_full), (q_issued - 1) & 1, kDrainNs);
     }
   } else if (warp == 2 || warp == 3) {
     // ======  PV loader warps (cp.async): this CTA's latent half of page p  ======
@@ -366,6 +377,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(dtc::kThreads, 1)
         const int s = itv % kPvStages;
         if (!mbar_wait(smem_u32(&pv_full[s]), (itv / kPvStages) & 1, abort_p, 12, itv))
           return false;
+        // The stage was written by cp.async and st.shared (generic proxy);
+        // the MMA reads it through the async proxy.  The writes are ordered
+        // before this thread by the barrier; the proxy fence makes them
+        // visible to the MMAs this thread issues next.  (The peer's half
+        // is fenced the same way by its relay lane.)
+        fence_proxy_async_smem();
         tc_fence_after();
         const uint32_t st = sPv + s * kPvStageBytes;
         for (int n = 0; n < 2; ++n) {
@@ -415,7 +432,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(dtc::kThreads, 1)
       }
       ++piece;
     }
-    if (ok && pend >= 0) issue_pv(pend, pend_first, pend_piece);
+    if (ok && pend >= 0) ok = issue_pv(pend, pend_first, pend_piece);
+    if (!ok) {
+      // Leaving early: one more commit tracks every MMA issued so far; wait
+      // (bounded) for it, so that no MMA still reads shared memory or writes
+      // TMEM when the pair frees them.
+      mma_commit_2_mc(smem_u32(&mma_drain), 1);
+      mbar_wait_bounded(smem_u32(&mma_drain), 0, kDrainNs);
+    }
   } else if (warp >= kSoftmaxWarp0) {
     // =================  softmax + epilogue (both CTAs)  =================
     const int tid = threadIdx.x - kSoftmaxWarp0 * 32;  // = TMEM lane

@@ -24,9 +24,22 @@ def test_code_digest_ignores_comments_only(tmp_path):
     assert bench.code_digest([str(a)]) != bench.code_digest([str(c)])
 
 
-def test_recorded_traffic_matches_current_decode_source():
-    src = os.path.join(ROOT, "mla_latent_kv_35_b200", "csrc", "decode_tc.cuh")
-    assert bench._traffic_for([src]) is not None
+def test_recorded_traffic_applies_only_to_the_captured_source(tmp_path, monkeypatch):
+    """The ncu DRAM bytes recorded under profiles/ are reported only while the
+    kernel source (comments aside) is the one the capture ran."""
+    import json
+    src = tmp_path / "k.cuh"
+    src.write_text("int f() { return 1; }  // kernel\n")
+    prof = tmp_path / "profiles"
+    prof.mkdir()
+    rec = {"dram_bytes_per_call": 123.0, "code_sha256": bench.code_digest([str(src)])}
+    (prof / "decode_tc_traffic.json").write_text(json.dumps(rec))
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    assert bench._traffic_for([str(src)]) == 123.0
+    src.write_text("int f() { return 1; }  // comment edited\n")
+    assert bench._traffic_for([str(src)]) == 123.0
+    src.write_text("int f() { return 2; }\n")
+    assert bench._traffic_for([str(src)]) is None
 
 
 def test_clock_summary_uses_samples_after_mark():

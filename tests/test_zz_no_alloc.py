@@ -76,7 +76,7 @@ def test_noalloc_refuses_oversized_problem():
     ensure_lib()
     d = dims("bf16")
     n = 2048                                    # workspace far above the 64 MiB scratch
-    assert B.mla_decode_workspace_size(d, n, 1, 0) > B.NOALLOC_SCRATCH_BYTES
+    assert B.mla_decode_workspace_size(d, n, 1, 0) > B.mla_decode_noalloc_scratch_bytes()
     dummy = torch.zeros(16, device=DEV)
     with pytest.raises(B.MLAError) as e:
         B.mla_decode_noalloc(d, dummy, dummy, 1, dummy, 1, dummy, n, 1, 0, dummy, dummy)
