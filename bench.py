@@ -161,14 +161,30 @@ def _traffic_for(kernel_src_paths):
     return rec.get("dram_bytes_per_call")
 
 
-def run_config(w, workload_name, world):
+L2_BYTES = 126 * 1024 * 1024
+L2_FLUSH_BYTES = 2 * L2_BYTES
+
+
+def flush_needed(w):
+    """The decode call reads only the cache (plus small q and outputs): when
+    the cache is under twice the L2 size, repeated calls would be served
+    partly from L2, so the bench flushes L2 between timed calls."""
+    _, _, cache_bytes = _workload_bytes(w)
+    return cache_bytes < 2 * L2_BYTES
+
+
+def run_config(w, workload_name, world, flush=None):
     """The JSON line's `config`, shared by both arms."""
     _, _, cache_bytes = _workload_bytes(w)
+    flush = flush_needed(w) if flush is None else flush
+    l2 = ("L2 flushed (%d MB write) before every timed call; cache %.3f GB"
+          % (L2_FLUSH_BYTES >> 20, cache_bytes / 1e9) if flush else
+          "inputs larger than L2 (cache %.2f GB), no flush" % (cache_bytes / 1e9))
     return {"workload": workload_name, "batch_per_gpu": w.B, "global_batch": w.B * world,
             "heads": w.H, "context": w.ctx[0] if len(set(w.ctx)) == 1 else "ragged",
             "S_q": w.S_q, "latent": w.d_latent, "rope": w.d_rope, "page": w.page_size,
             "d_model": w.d_model,
-            "l2": "inputs larger than L2 (cache %.2f GB), no flush" % (cache_bytes / 1e9),
+            "l2": l2,
             "parallelism": (f"dp{world}: independent sequence shards, no collective"
                             if world > 1 else "single GPU")}
 
@@ -328,30 +344,52 @@ def run_gpu(args, w):
         step()
     torch.cuda.synchronize(dev)
 
+    # L2 flush between timed calls when the decode's inputs fit in L2: a
+    # write of twice the L2 size, outside every timed region
+    flush = args.flush_l2 == "on" or (args.flush_l2 == "auto" and flush_needed(w))
+    flush_buf = torch.empty((L2_FLUSH_BYTES // 4,), dtype=torch.int32, device=dev) \
+        if flush else None
+
     def timed(fn, K, end=None):
-        """K back-to-back calls between one pair of CUDA events on the
-        launching stream (barrier + synchronize on both sides); `end` makes
-        that stream wait for work the calls left on other streams.  Returns
-        the mean ms per call, the wall time and this process's kernel
-        launches."""
-        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        """K calls timed with CUDA events on the launching stream (barrier +
+        synchronize on both sides); `end` makes that stream wait for work the
+        calls left on other streams.  Without a flush the K calls run back to
+        back between one pair of events; with it, each call has its own pair
+        and an L2 flush runs before it, outside the pair.  Returns the mean ms
+        per call, the wall time and this process's kernel launches."""
         if distributed:
             dist.barrier()
         torch.cuda.synchronize(dev)
         l0 = B.mla_launch_count()
         t0 = time.perf_counter()
-        e0.record(stream)
-        for _ in range(K):
-            fn()
-        if end is not None:
-            end()
-        e1.record(stream)
-        torch.cuda.synchronize(dev)
+        if flush_buf is None:
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            for _ in range(K):
+                fn()
+            if end is not None:
+                end()
+            e1.record(stream)
+            torch.cuda.synchronize(dev)
+            ms = e0.elapsed_time(e1)
+        else:
+            pairs = []
+            for _ in range(K):
+                flush_buf.add_(1)
+                e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                e0.record(stream)
+                fn()
+                if end is not None:
+                    end()
+                e1.record(stream)
+                pairs.append((e0, e1))
+            torch.cuda.synchronize(dev)
+            ms = sum(a.elapsed_time(b) for a, b in pairs)
         wall = time.perf_counter() - t0
         launches = B.mla_launch_count() - l0
         if distributed:
             dist.barrier()
-        return e0.elapsed_time(e1) / K, wall, launches
+        return ms / K, wall, launches
 
     # end to end through the public API with host buffers
     h_host = torch.from_numpy(h_np).to(d.torch_dtype).pin_memory()
@@ -415,7 +453,7 @@ def run_gpu(args, w):
         "vs_baseline": None,
         "dtype": "bf16" if w.dtype == "bf16" else "f32",
         "data": "synthetic",
-        "config": run_config(w, workload_name, world),
+        "config": run_config(w, workload_name, world, flush),
         "decode": {"ms": t_dec, "tokens_per_s": whole_job_rate(w.T, world, t_dec),
                    "cache_gb_per_s": cache_bytes / (t_dec * 1e-3) / 1e9,
                    "tflops": flops / (t_dec * 1e-3) / 1e12,
@@ -454,6 +492,9 @@ def main():
     ap.add_argument("--workload", default="batch128")
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--flush-l2", default="auto", choices=["auto", "on", "off"],
+                    help="flush L2 before every timed call (auto: when the cache is "
+                         "under twice the L2 size)")
     ap.add_argument("--batch", type=int, default=0,
                     help="use only the first N sequences of the workload")
     args = ap.parse_args()

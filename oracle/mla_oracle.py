@@ -25,7 +25,8 @@ rebuilds per-head keys ``k_{i,t} = [W_UK,i c_t ; RoPE(k_rope_t)]`` and values
 :func:`attention_absorbed` is the independent absorbed formulation used only
 to pin the absorption identity.
 
-Readings of points the pages leave open (each is listed in the design doc):
+Readings of points the pages leave open (the readings R1-R8 of this
+library, stated here in full):
 
 * R1  the 64-dim RoPE key is one vector per token, shared by all heads
       (576 = 512 + 64 numbers per token only adds up that way).

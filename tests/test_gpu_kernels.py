@@ -244,6 +244,14 @@ def _run_decode(d, c, S_q, workers=0):
     return to_np(o_lat), to_np(lse)
 
 
+def _expected_kernel(dtype, H, S_q):
+    """The split kernel mla_decode should pick: tensor cores for bf16 query
+    blocks of a multiple of 128 rows, CUDA cores otherwise."""
+    if dtype == "bf16" and (S_q * H) % 128 == 0:
+        return B.DECODE_KERNEL_TC
+    return B.DECODE_KERNEL_SIMT
+
+
 def _decode_ref(d, c, b):
     dc = d.d_latent
     r = c["rows"][b].astype(np.float64)
@@ -258,10 +266,14 @@ def _decode_ref(d, c, b):
     ("bf16", 128, 2, [2, 63, 64, 65, 128, 129, 700]),
     ("bf16", 64, 2, [5, 130, 257]),
     ("bf16", 16, 1, [40, 300]),
+    ("bf16", 32, 1, [33, 200, 129]),
+    ("bf16", 64, 1, [1, 190, 64]),
 ])
 def test_decode_matches_oracle(dtype, H, S_q, lens):
     dc, dr = (64, 16) if dtype == "f32" else (512, 64)
     d, c = _decode_case(dtype, H, lens, S_q, dc=dc, dr=dr)
+    kind, _, _ = B.mla_decode_config(d, S_q, 0)
+    assert kind == _expected_kernel(dtype, H, S_q)
     o_lat, lse = _run_decode(d, c, S_q)
     for b in range(len(lens)):
         ref = _decode_ref(d, c, b)

@@ -2,10 +2,12 @@
 
 tiny: every sequence, non-absorbed oracle, fp32 tolerance.
 bf16 workloads at full size, in the launch configuration the benchmark
-times: sampled sequences.  For each sampled sequence a few heads go through
-the non-absorbed oracle (explicit per-head keys and values) and all heads
-through the oracle's absorbed formulation (pinned equal to it to 1e-10),
-which also gives the reference for the output projection.
+times: every sequence of dsv2, ragged, long1 and long4, and for batch128
+every sequence whose token range a split-worker boundary cuts (plus both
+ends), all heads, against the oracle's absorbed formulation (pinned equal to
+the non-absorbed one to 1e-10), which also gives the reference for the
+output projection; a few heads of a few sequences also go through the
+non-absorbed oracle (explicit per-head keys and values).
 """
 
 import numpy as np
@@ -16,6 +18,8 @@ import oracle
 from mla_latent_kv_35_b200 import workloads as wl
 from mla_latent_kv_35_b200.binding import MLADims
 from mla_latent_kv_35_b200.engine import MLADecodeLayer, build_pool_host, pool_to_device
+import oracle_pool
+from mla_latent_kv_35_b200 import binding as B
 from gpu_util import DEV, check, ensure_lib, status, to_np
 
 gpu = pytest.mark.gpu
@@ -80,55 +84,88 @@ def test_tiny_full_path_fp32():
         check(out[b], res["out"][b][0], "f32", "A6 out")
 
 
-def _check_bf16_workload(name, sample, nonabs_heads=(0, 77, 127)):
+def _check_bf16_workload(name, sample, nonabs_sample, nonabs_heads=(0, 77, 127)):
+    """Every sequence in `sample`: all heads against the oracle's absorbed
+    formulation (run in a pool of host processes); sequences in
+    `nonabs_sample`: a few heads against the non-absorbed oracle too."""
     w = wl.workload(name)
     W, layer, bf, h, _, table = _setup(w)
     o_lat = to_np(bf["o_lat"]).reshape(w.B, w.S_q, w.H, w.d_latent)
     lse = to_np(bf["lse"]).reshape(w.B, w.S_q, w.H)
     out = to_np(bf["out"]).reshape(w.B, w.S_q, w.d_model)
-    pool = layer.pool.view(torch.int16)
+    pool_bits = layer.pool.view(torch.int16)
+    new_rows = {}
     for b in sample:
+        L = w.ctx[b]
+        new_rows[b] = [pool_bits[int(table[b, p // 64]), p % 64].cpu().numpy().view(np.uint16)
+                       for p in range(L - w.S_q, L)]
+    del layer, bf
+    torch.cuda.empty_cache()
+    ref = oracle_pool.workload_reference(w, W, h, sample)
+    for b in sample:
+        r = ref[b]
+        check(o_lat[b], r["o_lat"], "bf16", f"{name} b={b} o_lat (all heads)")
+        check(lse[b], r["lse"], "bf16", f"{name} b={b} lse")
+        check(out[b], r["out"], "bf16", f"{name} b={b} out")
+        # the appended rows hold the new tokens' latent and rotated RoPE key
+        for j, row in enumerate(new_rows[b]):
+            rowf = wl.bf16_to_f32(row).astype(np.float64)
+            check(rowf[:w.d_latent], r["c_new"][j], "bf16", "A3 c_new")
+            check(rowf[w.d_latent:], r["kr_new"][j], "bf16", "A3 kr_new")
+    for b in nonabs_sample:
         c, kr = wl.draw_prior(w, b)
-        args = (h[b:b + 1], [c], [kr], W["W_Q"], W["W_DKV"], W["W_KR"], W["W_UK"], W["W_UV"],
-                W["W_O"], w.scale, w.rope_base, w.H)
-        ab = oracle.decode_step(*args, prior_kr_rotated=True, formulation="absorbed")
-        na = oracle.decode_step(*args, prior_kr_rotated=True, heads=list(nonabs_heads))
-        check(o_lat[b], ab["o_lat"][0], "bf16", f"{name} b={b} o_lat (all heads)")
-        check(lse[b], ab["lse"][0], "bf16", f"{name} b={b} lse")
-        check(out[b], ab["out"][0], "bf16", f"{name} b={b} out")
+        na = oracle.decode_step(h[b:b + 1], [c], [kr], W["W_Q"], W["W_DKV"], W["W_KR"],
+                                W["W_UK"], W["W_UV"], W["W_O"], w.scale, w.rope_base, w.H,
+                                prior_kr_rotated=True, heads=list(nonabs_heads))
         check(o_lat[b][:, list(nonabs_heads)], na["o_lat"][0], "bf16",
               f"{name} b={b} o_lat vs non-absorbed")
         check(lse[b][:, list(nonabs_heads)], na["lse"][0], "bf16",
               f"{name} b={b} lse vs non-absorbed")
-        # the appended rows hold the new tokens' latent and rotated RoPE key
-        L = w.ctx[b]
-        for j in range(w.S_q):
-            p = L - w.S_q + j
-            row = pool[int(table[b, p // 64]), p % 64].cpu().numpy().view(np.uint16)
-            rowf = wl.bf16_to_f32(row).astype(np.float64)
-            check(rowf[:w.d_latent], ab["c_new"][0][j], "bf16", "A3 c_new")
-            check(rowf[w.d_latent:], ab["kr_new"][0][j], "bf16", "A3 kr_new")
+
+
+def boundary_sequences(w, S_q=1):
+    """Sequences whose block range is cut by a split-worker boundary, from
+    the planner's own rule (worker k starts at block floor(k*total/G))."""
+    d = MLADims.of(w)
+    _, bt, G = B.mla_decode_config(d, S_q, 0)
+    R = max(1, S_q * w.H // 128)
+    nb = [-(-L // bt) for L in w.ctx for _ in range(R)]
+    starts = np.concatenate([[0], np.cumsum(nb)])
+    total = int(starts[-1])
+    out = set()
+    for k in range(1, G):
+        x = k * total // G
+        v = int(np.searchsorted(starts, x, side="right") - 1)
+        if x != starts[v]:
+            out.add(v // R)
+    return sorted(out)
 
 
 @gpu
 def test_dsv2_full_path():
-    _check_bf16_workload("dsv2", sample=[0, 9, 15])
+    _check_bf16_workload("dsv2", sample=range(16), nonabs_sample=[0, 9, 15])
 
 
 @gpu
 def test_ragged_full_path():
     w = wl.workload("ragged")
     lens = np.array(w.ctx)
-    sample = [int(np.argmin(lens)), int(np.argmax(lens)), 5]
-    _check_bf16_workload("ragged", sample=sample)
+    _check_bf16_workload("ragged", sample=range(64),
+                         nonabs_sample=[int(np.argmin(lens)), int(np.argmax(lens)), 5])
 
 
 @gpu
 def test_batch128_full_path():
-    _check_bf16_workload("batch128", sample=[0, 127], nonabs_heads=(3, 100))
+    w = wl.workload("batch128")
+    ensure_lib()
+    seqs = sorted(set(boundary_sequences(w)) | {0, 1, 63, 64, 126, 127})
+    assert len(seqs) >= 16
+    _check_bf16_workload("batch128", sample=seqs, nonabs_sample=[0, seqs[len(seqs) // 2]],
+                         nonabs_heads=(3, 100))
 
 
 @gpu
 @pytest.mark.parametrize("name", ["long1", "long4"])
 def test_long_context_full_path(name):
-    _check_bf16_workload(name, sample=[0] if name == "long1" else [0, 3], nonabs_heads=(64,))
+    w = wl.workload(name)
+    _check_bf16_workload(name, sample=range(w.B), nonabs_sample=[0], nonabs_heads=(64,))

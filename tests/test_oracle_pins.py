@@ -375,10 +375,8 @@ def test_planted_mistakes_are_caught(monkeypatch):
                         lambda s, v: orig(s * 0.5, v))
     assert disagrees()
     monkeypatch.setattr(om, "_softmax_attend", orig)
-    # wrong RoPE sign is caught by the closed form
-    x = np.array([0.3, -1.2])
-    wrong = oracle.rope(x, -5, 10000.0)
-    assert np.abs(wrong - _rope_complex(x, 5, 10000.0)).max() > 1e-3
+    # RoPE slips are planted inside rope in test_rope_planted_mistakes_are_caught,
+    # the projection's transpose in test_project_transpose_slip_is_caught
 
 
 def test_out_proj_matches_nonabsorbed_output():
@@ -390,3 +388,163 @@ def test_out_proj_matches_nonabsorbed_output():
     o, out = oracle.out_proj(res["o_lat"], P["W_UV"], W_O)
     np.testing.assert_allclose(o, res["o"], atol=1e-12)
     np.testing.assert_allclose(out, res["o"].reshape(1, -1) @ W_O.T, atol=1e-12)
+
+
+# --------------------------------------------------------------------------
+# projection: pure-Python brute force, square and non-square weights
+# --------------------------------------------------------------------------
+
+def _project_brute(x, w):
+    """y[r][o] = sum_i x[r][i] * w[o][i], written out with loops (w is
+    [out, in]: each output feature is one row of w)."""
+    return [[sum(x[r][i] * w[o][i] for i in range(len(x[r]))) for o in range(len(w))]
+            for r in range(len(x))]
+
+
+@pytest.mark.parametrize("rows,in_f,out_f", [(3, 4, 4), (2, 5, 3), (1, 3, 7)])
+def test_project_matches_brute_force(rows, in_f, out_f):
+    rng = np.random.default_rng(rows * 100 + in_f * 10 + out_f)
+    x = rng.standard_normal((rows, in_f))
+    w = rng.standard_normal((out_f, in_f))
+    np.testing.assert_allclose(oracle.project(x, w), _project_brute(x, w), rtol=0, atol=1e-12)
+
+
+def test_project_transpose_slip_is_caught(monkeypatch):
+    """A transposed weight (x @ w instead of x @ w^T) planted in the oracle
+    fails the brute-force pin on a square, non-symmetric weight."""
+    rng = np.random.default_rng(31)
+    x = rng.standard_normal((3, 4))
+    w = rng.standard_normal((4, 4))
+    assert np.abs(w - w.T).max() > 0.1
+    monkeypatch.setattr(om, "project", lambda a, b: np.asarray(a, float) @ np.asarray(b, float))
+    assert np.abs(om.project(x, w) - np.array(_project_brute(x, w))).max() > 1e-3
+
+
+# --------------------------------------------------------------------------
+# decode_step wiring, worked by hand
+# --------------------------------------------------------------------------
+
+def test_decode_step_hand_worked_example():
+    """One sequence with two cached tokens and two new query tokens, two
+    heads, every weight chosen so the step can be followed by hand.
+
+    Sizes: d_model 2, d_nope 1, latent 1, rope 2 (one pair, theta = 1 rad per
+    position whatever the base), d_v 1, scale 1/2.
+    Cached before the step (reading R2): token 0 with c = 3, pre-RoPE key
+    (1, 0); token 1 with c = -1, pre-RoPE key (0, 1).  The new tokens sit at
+    positions 2 and 3 (L - S_q + j), with hidden states (1, 0) and (0, 1).
+      W_DKV = [1 2]  -> c_2 = 1, c_3 = 2
+      W_KR  = I      -> pre-RoPE keys (1, 0) and (0, 1)
+    RoPE by position t rotates the key by t rad:
+      k_0 = (1, 0), k_1 = (-sin 1, cos 1), k_2 = (cos 2, sin 2),
+      k_3 = (-sin 3, cos 3)
+    W_Q gives both heads q_nope = 1 and q_rope = h, so the rotated query
+    parts are (cos 2, sin 2) at position 2 and (-sin 3, cos 3) at position 3.
+    Head 0: W_UK = 2, W_UV = 1, so its key is (2 c_t ; k_t); head 1: W_UK = 0,
+    W_UV = 2.  Dot products of rotated RoPE parts depend on the position
+    difference: (cos 2, sin 2).(-sin 1, cos 1) = sin 1,
+    (-sin 3, cos 3).(1, 0) = -sin 3, (-sin 3, cos 3).(-sin 1, cos 1) = cos 2,
+    (-sin 3, cos 3).(cos 2, sin 2) = -sin 1, and a part with itself gives 1.
+    Query at position 2 sees tokens 0..2; query at position 3 sees 0..3.
+    Raw scores (before the scale 1/2):
+      head 0, pos 2: 6 + cos 2,  -2 + sin 1,  2 + 1
+      head 0, pos 3: 6 - sin 3,  -2 + cos 2,  2 - sin 1,  4 + 1
+      head 1, pos 2: cos 2,  sin 1,  1
+      head 1, pos 3: -sin 3,  cos 2,  -sin 1,  1
+    o_lat = sum p_t c_t over c = (3, -1, 1, 2); o = W_UV o_lat;
+    W_O = [[1, 0], [3, 1]] gives out = (o_0, 3 o_0 + o_1).
+    """
+    sin, cos, exp, log = math.sin, math.cos, math.exp, math.log
+    raw = {(0, 0): [6 + cos(2), -2 + sin(1), 3.0],
+           (0, 1): [6 - sin(3), -2 + cos(2), 2 - sin(1), 5.0],
+           (1, 0): [cos(2), sin(1), 1.0],
+           (1, 1): [-sin(3), cos(2), -sin(1), 1.0]}
+    cvals = [3.0, -1.0, 1.0, 2.0]
+    W_UV = [1.0, 2.0]
+    expect_olat = np.zeros((2, 2, 1))
+    expect_lse = np.zeros((2, 2))
+    for (i, j), s in raw.items():
+        s = [0.5 * v for v in s]
+        z = sum(exp(v) for v in s)
+        expect_olat[j, i, 0] = sum(exp(v) / z * cvals[t] for t, v in enumerate(s))
+        expect_lse[j, i] = log(z)
+    o = expect_olat[:, :, 0] * np.array(W_UV)           # [S_q, H]
+    expect_out = np.stack([o[:, 0], 3 * o[:, 0] + o[:, 1]], axis=1)
+
+    W = dict(W_Q=np.array([[1., 1.], [1., 0.], [0., 1.], [1., 1.], [1., 0.], [0., 1.]]),
+             W_DKV=np.array([[1., 2.]]), W_KR=np.eye(2),
+             W_UK=np.array([[[2.]], [[0.]]]), W_UV=np.array([[[1.]], [[2.]]]),
+             W_O=np.array([[1., 0.], [3., 1.]]))
+    h = np.array([[[1., 0.], [0., 1.]]])
+    c_prior = [np.array([[3.], [-1.]])]
+    kr_prior = [np.array([[1., 0.], [0., 1.]])]
+    for form in ("nonabsorbed", "absorbed"):
+        res = oracle.decode_step(h, c_prior, kr_prior, scale=0.5, rope_base=10000.0,
+                                 n_heads=2, formulation=form, **W)
+        np.testing.assert_allclose(res["o_lat"][0], expect_olat, rtol=0, atol=1e-12)
+        np.testing.assert_allclose(res["lse"][0], expect_lse, rtol=0, atol=1e-12)
+        np.testing.assert_allclose(res["out"][0], expect_out, rtol=0, atol=1e-12)
+        np.testing.assert_allclose(res["c_new"][0], [[1.], [2.]], atol=0)
+        np.testing.assert_allclose(res["kr_new"][0], [[cos(2), sin(2)], [-sin(3), cos(3)]],
+                                   atol=1e-15)
+    # the same cache given as already rotated keys
+    kr_rot = [np.array([[1., 0.], [-sin(1), cos(1)]])]
+    res = oracle.decode_step(h, c_prior, kr_rot, scale=0.5, rope_base=10000.0, n_heads=2,
+                             prior_kr_rotated=True, **W)
+    np.testing.assert_allclose(res["o_lat"][0], expect_olat, rtol=0, atol=1e-12)
+    # a subset of heads: the same numbers for that head, no output projection
+    res = oracle.decode_step(h, c_prior, kr_prior, scale=0.5, rope_base=10000.0, n_heads=2,
+                             heads=[1], **W)
+    np.testing.assert_allclose(res["o_lat"][0][:, 0], expect_olat[:, 1], rtol=0, atol=1e-12)
+    np.testing.assert_allclose(res["lse"][0][:, 0], expect_lse[:, 1], rtol=0, atol=1e-12)
+    assert res["out"][0] is None
+    # planted in the oracle: the new tokens placed at positions 0..S_q-1
+    # instead of L-S_q..L-1 (decode_step builds them with a two-argument
+    # arange; the one-argument calls stay correct)
+    def arange(*a, **k):
+        if len(a) == 2:
+            return np.arange(0, a[1] - a[0], **k)
+        return np.arange(*a, **k)
+    orig_np = om.np
+    try:
+        om.np = _NumpyWith(arange=arange)
+        res = oracle.decode_step(h, c_prior, kr_prior, scale=0.5, rope_base=10000.0,
+                                 n_heads=2, **W)
+    finally:
+        om.np = orig_np
+    assert np.abs(res["o_lat"][0] - expect_olat).max() > 1e-3
+
+
+# --------------------------------------------------------------------------
+# RoPE: mistakes planted inside the oracle's own function are caught
+# --------------------------------------------------------------------------
+
+class _NumpyWith:
+    """numpy with some functions replaced, to plant a slip inside the
+    oracle's rope (which reaches numpy through the module's `np`)."""
+
+    def __init__(self, **over):
+        self.__dict__.update(over)
+
+    def __getattr__(self, name):
+        return getattr(np, name)
+
+
+@pytest.mark.parametrize("slip", ["sin_sign", "theta_exponent", "angle_units"])
+def test_rope_planted_mistakes_are_caught(monkeypatch, slip):
+    """Slips planted inside the oracle's rope (through the numpy it calls)
+    make it disagree with the complex-exponential closed form."""
+    rng = np.random.default_rng(32)
+    x = rng.standard_normal(16)
+    expect = _rope_complex(x, 37, 10000.0)
+    np.testing.assert_allclose(oracle.rope(x, 37, 10000.0), expect, atol=1e-9)
+    if slip == "sin_sign":                  # rotating the wrong way
+        fake = _NumpyWith(sin=lambda a: -np.sin(a))
+    elif slip == "theta_exponent":          # base^(-k/d) instead of base^(-2k/d)
+        fake = _NumpyWith(power=lambda a, b: np.power(a, b / 2.0))
+    else:                                   # angle taken in degrees
+        fake = _NumpyWith(cos=lambda a: np.cos(np.deg2rad(a)),
+                          sin=lambda a: np.sin(np.deg2rad(a)))
+    monkeypatch.setattr(om, "np", fake)
+    got = oracle.rope(x, 37, 10000.0)
+    assert np.abs(got - expect).max() > 1e-3
