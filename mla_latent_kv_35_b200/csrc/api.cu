@@ -72,7 +72,7 @@ EncodeTiledFn encode_fn() {
   return fn;
 }
 
-// bf16 tensor of rank `rank` (<= 3), dims innermost first, byte strides of
+// bf16 tensor of rank `rank` (<= 5), dims innermost first, byte strides of
 // dims 1.., 128-byte swizzle, zero fill out of bounds.
 bool make_tmap_bf16(CUtensorMap* m, const void* ptr, int rank, const uint64_t* dims,
                     const uint64_t* strides_bytes, const uint32_t* box) {
@@ -205,11 +205,18 @@ mla_status launch_tc_gemm(const void* A, bool a_mn, long long as_b, const void* 
 // ---------------------------------------------------------------------------
 // decode planning
 // ---------------------------------------------------------------------------
-constexpr int kBlockTokens = 128;
+// cache tokens per work block: the tensor-core kernel's block (four pages),
+// and the CUDA-core kernel's
+constexpr int kBlockTokensSimt = 128;
 
+// The tensor-core kernel covers every bf16 shape with DeepSeek-V2's cache
+// row (512 + 64) and 64-token pages; query blocks of fewer than 128 rows
+// (S_q * H < 128, or the last block of a sequence) are padded to the MMA's
+// 128 rows, whose extra rows are computed and dropped.
 bool use_tc_decode(const mla_dims* d, int S_q) {
-  return kDecodeTcReady && d->dtype == MLA_BF16 && d->d_latent == 512 && d->d_rope == 64 && d->page_size == 64 &&
-         ((S_q * d->n_heads) % 128) == 0;
+  (void)S_q;
+  return kDecodeTcReady && d->dtype == MLA_BF16 && d->d_latent == 512 && d->d_rope == 64 &&
+         d->page_size == 64;
 }
 
 struct DecodeLayout {
@@ -220,8 +227,10 @@ struct DecodeLayout {
 DecodeLayout decode_layout(const mla_dims* d, int B, int S_q, int num_workers) {
   DecodeLayout L;
   const bool tc = use_tc_decode(d, S_q);
-  L.R = tc ? (S_q * d->n_heads) / 128 : 1;
-  L.rows_per_v = (S_q * d->n_heads) / L.R;
+  // R blocks of rows_per_v workspace rows per sequence (the last block of
+  // the tensor-core path may be partly padding)
+  L.R = tc ? (S_q * d->n_heads + 127) / 128 : 1;
+  L.rows_per_v = tc ? 128 : S_q * d->n_heads;
   L.V = B * L.R;
   const int sms = sm_count();
   L.G = num_workers > 0 ? num_workers : (tc ? sms / 2 : 2 * sms);
@@ -415,7 +424,7 @@ mla_status mla_decode_config(const mla_dims* dims, int S_q, int num_workers, int
   if (!dims_ok(dims) || S_q < 1 || S_q > 2 || num_workers < 0) return MLA_ERR_INVALID_ARG;
   const DecodeLayout L = decode_layout(dims, 1, S_q, num_workers);
   if (kernel) *kernel = use_tc_decode(dims, S_q) ? MLA_DECODE_KERNEL_TC : MLA_DECODE_KERNEL_SIMT;
-  if (block_tokens) *block_tokens = kBlockTokens;
+  if (block_tokens) *block_tokens = use_tc_decode(dims, S_q) ? dtc::kBlk : kBlockTokensSimt;
   if (workers) *workers = L.G;
   return MLA_OK;
 }
@@ -446,10 +455,12 @@ static mla_status decode_impl(const mla_dims* dims, const void* qbuf, const void
   float* ws_lse = reinterpret_cast<float*>(ws + L.off_lse);
   float* ws_o = reinterpret_cast<float*>(ws + L.off_o);
   const int max_tokens = max_pages * dims->page_size;
-  plan_kernel<<<1, 1024, 0, st>>>(seq_lens, tail, B, L.R, S_q, max_tokens, kBlockTokens, start);
+  const bool tc = use_tc_decode(dims, S_q);
+  plan_kernel<<<1, 1024, 0, st>>>(seq_lens, tail, B, L.R, S_q, max_tokens,
+                                  tc ? dtc::kBlk : kBlockTokensSimt, start);
   MLA_TRY(check_launch());
   const int H = dims->n_heads, dc = dims->d_latent, dr = dims->d_rope;
-  if (use_tc_decode(dims, S_q)) {
+  if (tc) {
     if (!aligned16(qbuf) || !aligned16(pool)) return MLA_ERR_INVALID_ARG;
     MLA_TRY(launch_decode_tc_impl(make_tmap_bf16, qbuf, pool, n_pages, page_table, max_pages,
                                   seq_lens, tail, B, S_q, H, dims->scale, L.G, start, ws_lse,
@@ -461,7 +472,7 @@ static mla_status decode_impl(const mla_dims* dims, const void* qbuf, const void
 #define MLA_SIMT_DECODE(T, KC)                                                                 \
   decode_simt_kernel<T, KC><<<grid, 256, 0, st>>>(                                             \
       static_cast<const T*>(qbuf), static_cast<const T*>(pool), n_pages, page_table, max_pages, \
-      seq_lens, tail, B, S_q, H, dc, dr, dims->page_size, dims->scale, L.G, kBlockTokens,       \
+      seq_lens, tail, B, S_q, H, dc, dr, dims->page_size, dims->scale, L.G, kBlockTokensSimt,   \
       start, ws_lse, ws_o)
     if (dims->dtype == MLA_F32) {
       if (kc <= 2) MLA_SIMT_DECODE(float, 2);
@@ -478,7 +489,8 @@ static mla_status decode_impl(const mla_dims* dims, const void* qbuf, const void
     MLA_TRY(check_launch());
   }
   dim3 cgrid(L.V, (L.rows_per_v + 7) / 8);
-  combine_kernel<<<cgrid, 256, 0, st>>>(ws_lse, ws_o, start, L.V, L.R, L.G, L.rows_per_v, dc,
+  combine_kernel<<<cgrid, 256, 0, st>>>(ws_lse, ws_o, start, L.V, L.R, L.G, L.rows_per_v,
+                                        S_q * H, dc,
                                         o_lat, lse);
   return check_launch();
 }

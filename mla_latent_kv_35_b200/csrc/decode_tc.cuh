@@ -11,47 +11,50 @@
 // Work decomposition
 //   * A cluster of two CTAs (one per SM of a TPC) owns 128 query rows
 //     (S_q*H rows of one sequence, 128 at a time) and a contiguous run of
-//     128-token blocks.  CTA r holds rows [64r, 64r+64): its Q slice (72 KB,
-//     one TMA load per piece) stays in shared memory for the whole piece.
-//   * QK: pair MMAs (cta_group::2, M = 128 rows, N = 128 tokens, K = 576).
-//     CTA r supplies the B half of page r of the block.  Each SM gets its 64
-//     rows x 128 tokens in TMEM folded onto 128 lanes x 64 columns: lane l<64
-//     holds row l, tokens 0..63; lane l>=64 holds row l-64, tokens 64..127.
-//   * PV: two pair MMAs per 16-token step (N = 256 latent columns each,
-//     M = 128 rows, K = 128 tokens per block).  CTA r supplies latent columns
-//     [256n + 128r, +128) of all 128 tokens (MN-major B read straight from
-//     the cache tile) and its own 64 rows of P (bf16, K-major).  O therefore
-//     takes 256 TMEM columns per SM; S is double buffered in 2 x 64 more.
-//   * Loads.  Warp 0 lane 0 of each CTA streams its own page of the block
-//     for QK through a 3-stage ring.  Each stage is one 24 KB TMA box (64
-//     columns x 64 slots x 3 chunks) of a 4-D view of the pool: (64 columns,
-//     64 slots, 9 chunks, pages), strides (1152 B, 128 B, 73728 B).  Only the
-//     leader arms the stage barrier, for the bytes of both CTAs; the peer's
-//     box completes on the leader's barrier.
-//   * PV tiles come through a second ring of two 32 KB stages, one page's
-//     latent half each.  Warps 2 and 3 fill them with 16-byte cp.async into
-//     the 128-byte-swizzled layout, so this traffic bypasses the bulk-copy
-//     engine the QK boxes keep busy.  In the peer CTA, warp 1 lane 0 relays
-//     each landed stage to the leader's barrier.
-//   * Each 128-thread softmax warpgroup reads its SM's S and exchanges row
-//     maxima between the two lanes that share a row.  It keeps a lazily
-//     rescaled running max: O is rescaled in TMEM only when the max grows by
-//     more than 2^8, and warp-uniformly, since tcgen05.ld/st are collective.
-//     It then writes P to shared memory and signals the leader's MMA warp.
+//     256-token blocks (four 64-token pages).  CTA r holds rows [64r, 64r+64)
+//     of Q (72 KB, one TMA load per piece), resident for the whole piece.
+//   * QK: pair MMAs (cta_group::2, M = 128 rows, N = 256 tokens, K = 576).
+//     CTA r supplies the B half of pages 2r and 2r+1 of the block.  Each SM
+//     gets its 64 rows x 256 tokens in TMEM folded onto 128 lanes x 128
+//     columns: lane l < 64 holds row l, tokens 0..127; lane l >= 64 holds row
+//     l - 64, tokens 128..255.  Per SM every MMA is 64 x 256 x 16, a shape
+//     the tensor core runs at full rate (64 x 128 x 16 costs about as much
+//     per instruction, so 256-token blocks halve the QK instruction count).
+//   * PV: pair MMAs with N = 256 latent columns (two per 16-token step, one
+//     per latent half n).  CTA r supplies latent columns [256n + 128r, +128)
+//     of all 256 tokens (MN-major B) and its own 64 rows of P (bf16,
+//     K-major).  O takes 256 TMEM columns per SM, S 2 x 128 more: all 512.
+//   * QK loads.  Lane 0 of warp 0 in each CTA streams its two pages through a
+//     ring of two 32 KB stages; a stage holds two 64-column chunks of both
+//     pages, one 16 KB TMA box per page from a 5-D view of the pool:
+//     (64 columns, 8 slots, 9 chunks, 8 slot groups, pages).  The box lands as
+//     [slot group][chunk][8 slots][128 B], so the two pages' slot groups of a
+//     chunk sit at one uniform stride (2 KB) and form the 128-row K-major B
+//     operand.  Only the leader arms each stage barrier, for both CTAs' bytes.
+//     The same lane prefetches the next block's pages into L2 (bulk
+//     prefetch, one request per page), so the boxes are served from L2.
+//   * PV loads.  Warps 2 and 3 fill a ring of three 16 KB stages (one page x
+//     128 latent columns) with 16-byte cp.async into the 128-byte-swizzled
+//     layout; they read the same pages the QK boxes just brought into L2.
+//     In the peer CTA, warp 1 lane 0 relays each landed stage to the
+//     leader's barrier.
+//   * Softmax: eight warps per CTA.  Warps w and w + 4 share TMEM lane
+//     quadrant w and take 64 of its 128 columns each, so every thread holds
+//     the scores of one row on one page.  Row maxima of the four pages meet
+//     in shared memory.  The running max is rescaled lazily: O is rescaled
+//     in TMEM only when a row's max grows by more than 2^8, warp-uniformly.
+//     P goes to shared memory and the leader's MMA warp is signalled.
 //   * Pieces (sequence, block range) of a worker write normalised partial
 //     outputs and natural-log LSE into slot worker + v of the workspace; the
 //     combine kernel merges them.
 //
-// Shared memory: Q 72 KB + P 16 KB + QK ring 72 KB + PV ring 64 KB.  Each
-// ring holds one block.  The QK MMA shape the pair split gives, 64 x 128 x 16
-// per SM, costs about as much per instruction as a full-size one.  So the
-// MMA sequence and the one block of ring depth bound this kernel, not HBM.
+// Shared memory: Q 72 KB + P 32 KB + QK ring 64 KB + PV ring 48 KB.
 //
-// Partial pages: a page with `valid` < 64 tokens starts its boxes at slot
-// valid - 64.  The rows before the page are out of bounds and arrive as
-// zeros, and the cp.async loader shifts its rows the same way.  Pages past
-// the end load entirely out of bounds (slot 64).  Unused cache slots are
-// never read.
+// Partial and missing pages.  QK boxes always load a whole page; slots past
+// the sequence hold whatever the pool holds there and are masked by index in
+// the softmax (P = 0).  The PV loader writes zeros for those rows, so no
+// unused slot ever reaches O.  Pages past the end load entirely out of
+// bounds (zeros) and their page-table entries are never read.
 //
 // Every mbarrier wait is bounded (MLA_WAIT_NS); on expiry the kernel raises
 // MLA_ERR_TIMEOUT in the device status and every role leaves its loop.  On
@@ -69,28 +72,37 @@ namespace mla {
 constexpr bool kDecodeTcReady = true;
 
 namespace dtc {
-constexpr int kDC = 512;           // latent width
-constexpr int kD = 576;            // cached numbers per token
-constexpr int kPage = 64;          // tokens per page
-constexpr int kBlk = 128;          // tokens per block (two pages)
-constexpr int kChunk = 8192;       // 64 tokens x 64 columns bf16, one swizzled operand tile
-constexpr int kQkChunks = 3;       // chunks per QK stage (one TMA box)
-constexpr int kQkStages = 3;       // QK ring: 3 stages x 3 chunks = this CTA's page of one block
-constexpr int kQkStageBytes = kQkChunks * kChunk;
-constexpr int kPvStages = 2;       // PV ring: one page's latent half (4 chunks) per stage
-constexpr int kPvStageBytes = 4 * kChunk;
-constexpr int kQBytes = 9 * kChunk;  // 64 rows x 576 cols bf16
-constexpr int kPBytes = 2 * kChunk;  // 64 rows x 128 tokens bf16
+constexpr int kDC = 512;             // latent width
+constexpr int kD = 576;              // cached numbers per token
+constexpr int kPage = 64;            // tokens per page
+constexpr int kBlk = 256;            // tokens per block (four pages)
+constexpr int kPageBytes = kPage * kD * 2;
+constexpr int kChunk = 8192;         // 64 rows x 64 columns bf16, one swizzled operand tile
+constexpr int kQkBox = 2 * kChunk;   // one page x two chunks (16 KB)
+constexpr int kQkStageBytes = 2 * kQkBox;
+constexpr int kQkStages = 2;
+constexpr int kQkStagesPerBlock = 5; // chunks {0,1} {2,3} {4,5} {6,7} {8}
+constexpr int kPvStageBytes = 2 * kChunk;  // one page x 128 latent columns
+constexpr int kPvStages = 3;
+constexpr int kPvStagesPerBlock = 8;       // 4 pages x 2 latent halves
+constexpr int kQBytes = 9 * kChunk;        // 64 rows x 576 columns
+constexpr int kPBytes = 4 * kChunk;        // 64 rows x 256 tokens
 constexpr uint32_t kOffQ = 0;
 constexpr uint32_t kOffP = kOffQ + kQBytes;
 constexpr uint32_t kOffQk = kOffP + kPBytes;
 constexpr uint32_t kOffPv = kOffQk + kQkStages * kQkStageBytes;
 constexpr uint32_t kSmemBytes = kOffPv + kPvStages * kPvStageBytes + 1024;  // + alignment
-constexpr int kThreads = 256;
+constexpr int kThreads = 384;
 constexpr int kSoftmaxWarp0 = 4;
+constexpr int kSoftmaxThreads = 256;
+// registers per thread: at launch (65536 / 384, rounded down to 8), then
+// after the split of the control warpgroup and the softmax warpgroups
+constexpr int kRegsLaunch = 168;
+constexpr int kRegsControl = 72;
+constexpr int kRegsSoftmax = 216;
 constexpr uint32_t kTmemCols = 512;
-constexpr uint32_t kTmemO = 0;     // O_n at columns [128n, 128n + 128)
-constexpr uint32_t kTmemS = 256;   // S_b at columns [256 + 64b, +64)
+constexpr uint32_t kTmemO = 0;       // O_n at columns [128n, 128n + 128)
+constexpr uint32_t kTmemS = 256;     // S_b at columns [256 + 128b, +128)
 constexpr float kRescaleLog2 = 8.0f;
 }  // namespace dtc
 
@@ -121,14 +133,6 @@ __device__ __forceinline__ void named_bar_sync(int id, int nthreads) {
   asm volatile("barrier.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
 }
 
-__device__ __forceinline__ void mbar_expect_tx_cluster(uint32_t bar_cluster, uint32_t bytes) {
-  asm volatile(
-      "mbarrier.arrive.expect_tx.release.cluster.shared::cluster.b64 _, [%0], %1;" ::"r"(
-          bar_cluster),
-      "r"(bytes)
-      : "memory");
-}
-
 // Piece iteration shared by all roles: worker k's blocks [lo, hi) split by
 // virtual sequence.
 struct PieceIter {
@@ -150,28 +154,18 @@ struct PieceIter {
   }
 };
 
-// Page of token block x, half p (0/1) of sequence b: the pool page and the
-// first slot to load.  A partial page starts at a negative slot (the rows
-// before the page load as zeros); a page past the context, or a page id
-// outside the pool (raising MLA_ERR_BOUNDS), loads entirely out of bounds.
-__device__ __forceinline__ void page_of(const DecodeTcParams& P, int b, int L, int x, int p,
-                                        int& page, int& slot0) {
+// Pool page holding page p (0..3) of token block x of sequence b, or -1 when
+// that page lies past the sequence (its table entry is not read).  A page id
+// outside the pool raises MLA_ERR_BOUNDS and reads as -1 too.
+__device__ __forceinline__ int page_of(const DecodeTcParams& P, int b, int L, int x, int p) {
   const int first = x * dtc::kBlk + p * dtc::kPage;
-  const int valid = min(L - first, dtc::kPage);
-  if (valid <= 0) {
-    page = 0;
-    slot0 = dtc::kPage;
-    return;
-  }
+  if (first >= L) return -1;
   const int pg = P.page_table[(long long)b * P.max_pages + first / dtc::kPage];
   if (pg < 0 || pg >= P.n_pages) {
     raise_flag(kFlagBounds);
-    page = 0;
-    slot0 = dtc::kPage;
-    return;
+    return -1;
   }
-  page = pg;
-  slot0 = valid - dtc::kPage;
+  return pg;
 }
 
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(dtc::kThreads, 1)
@@ -184,8 +178,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(dtc::kThreads, 1)
   __shared__ __align__(8) uint64_t pv_full[kPvStages], pv_empty[kPvStages];
   __shared__ __align__(8) uint64_t q_full, q_empty, o_empty, p_full, pv_done, mma_drain;
   __shared__ __align__(8) uint64_t s_full[2];
-  __shared__ float red_max[2][2][64];
-  __shared__ float red_sum[2][64];
+  __shared__ float red_max[2][4][64];
+  __shared__ float red_sum[4][64];
   __shared__ uint32_t tmem_base_sh;
   __shared__ int abort_flag;
 
@@ -200,7 +194,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(dtc::kThreads, 1)
     abort_flag = 0;
     for (int s = 0; s < kQkStages; ++s) {
       // full barriers: the leader's producer arrives once with the bytes of
-      // both CTAs; the peer's copies only complete transactions on it
+      // both CTAs; the peer's boxes only complete transactions on it
       mbar_init(smem_u32(&qk_full[s]), 1);
       mbar_init(smem_u32(&qk_empty[s]), 1);  // MMA commit (multicast)
     }
@@ -211,8 +205,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(dtc::kThreads, 1)
     }
     mbar_init(smem_u32(&q_full), 1);
     mbar_init(smem_u32(&q_empty), 1);
-    mbar_init(smem_u32(&o_empty), 8);        // 4 softmax warps x 2 CTAs
-    mbar_init(smem_u32(&p_full), 8);
+    mbar_init(smem_u32(&o_empty), 16);       // 8 softmax warps x 2 CTAs
+    mbar_init(smem_u32(&p_full), 16);
     mbar_init(smem_u32(&pv_done), 1);
     mbar_init(smem_u32(&mma_drain), 1);
     mbar_init(smem_u32(&s_full[0]), 1);
@@ -237,217 +231,295 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(dtc::kThreads, 1)
   const int hi = total > 0 ? worker_lo(worker + 1, total, P.G) : 0;
   const int rows_seq = P.S_q * P.H;
 
-  if (warp == 0 && lane == 0) {
-    // =================  QK producer: Q slices and QK chunks  =================
-    const uint32_t lead_full0 = mapa_shared(smem_u32(&qk_full[0]), 0);
-    const uint32_t lead_qfull = mapa_shared(smem_u32(&q_full), 0);
-    uint32_t it = 0;
-    PieceIter pi;
-    pi.init(P.start, V, lo, hi);
-    int v, x0, x1, piece = 0;
-    uint32_t q_issued = 0;
-    bool ok = true;
-    while (ok && pi.next(v, x0, x1)) {
-      const int b = v / P.R, rb = v % P.R;
-      const int L = P.seq_lens[b];
-      // the Q slice is free once the previous piece's QK MMAs completed
-      if (piece > 0 && !mbar_wait(smem_u32(&q_empty), (piece - 1) & 1, abort_p, 2, piece)) {
-        ok = false;
-        break;
+  // Registers: the control warpgroup (producer, MMA, loaders) gives up most
+  // of its share to the two softmax warpgroups.
+  static_assert(128 * kRegsControl + 256 * kRegsSoftmax <= 65536 &&
+                    kRegsLaunch * kThreads <= 65536,
+                "register split exceeds the launch allocation");
+  if (warp < kSoftmaxWarp0) {
+    // (the register budget applies to the code it dominates)
+    setmaxnreg_dec<kRegsControl>();
+    if (warp == 0 && lane == 0) {
+      // ==========  QK producer: Q slices, QK boxes, L2 prefetch  ==========
+      const uint32_t lead_full0 = mapa_shared(smem_u32(&qk_full[0]), 0);
+      const uint32_t lead_qfull = mapa_shared(smem_u32(&q_full), 0);
+      uint32_t it = 0, q_issued = 0;
+      PieceIter pi;
+      pi.init(P.start, V, lo, hi);
+      // cursor of the next block to prefetch into L2 (global block index)
+      int pf_g = lo, pf_v = lo < hi ? seq_of_block(P.start, V, lo) : V;
+      auto prefetch_upto = [&](int g_end) {
+        for (; pf_g < min(g_end, hi); ++pf_g) {
+          while (P.start[pf_v + 1] <= pf_g) ++pf_v;
+          const int b = pf_v / P.R;
+          const int L = P.seq_lens[b];
+          const int x = pf_g - P.start[pf_v];
+          for (int i = 0; i < 2; ++i) {
+            const int pg = page_of(P, b, L, x, 2 * (int)rank + i);
+            if (pg >= 0) prefetch_l2_bulk(P.pool + (size_t)pg * kPageBytes, kPageBytes);
+          }
+        }
+      };
+      int v, x0, x1, piece = 0;
+      bool ok = true;
+      while (ok && pi.next(v, x0, x1)) {
+        const int b = v / P.R, rb = v % P.R;
+        const int L = P.seq_lens[b];
+        // the Q slice is free once the previous piece's QK MMAs completed
+        if (piece > 0 && !mbar_wait(smem_u32(&q_empty), (piece - 1) & 1, abort_p, 2, piece)) {
+          ok = false;
+          break;
+        }
+        if (rank == 0) mbar_expect_tx(smem_u32(&q_full), 2 * kQBytes);
+        const int row0 = b * rows_seq + rb * 128 + 64 * (int)rank;
+        for (int c = 0; c < 9; ++c)
+          tma_load_2d_pair(sQ + c * kChunk, &tmQ, c * 64, row0, lead_qfull);
+        ++q_issued;
+        for (int x = x0; x < x1 && ok; ++x) {
+          // this block and the next one go to L2 ahead of the boxes
+          prefetch_upto(P.start[v] + x + 2);
+          int pg[2];
+          for (int i = 0; i < 2; ++i) {
+            pg[i] = page_of(P, b, L, x, 2 * (int)rank + i);
+            if (pg[i] < 0) pg[i] = P.n_pages;   // out of bounds: the box reads zeros
+          }
+          for (int k = 0; k < kQkStagesPerBlock; ++k, ++it) {
+            const int s = it % kQkStages;
+            if (!mbar_wait(smem_u32(&qk_empty[s]), ((it / kQkStages) & 1) ^ 1, abort_p, 1, it)) {
+              ok = false;
+              break;
+            }
+            const uint32_t fb = lead_full0 + s * 8;
+            if (rank == 0) mbar_expect_tx(smem_u32(&qk_full[s]), 2 * kQkStageBytes);
+            const uint32_t dst = sQk + s * kQkStageBytes;
+            // chunks 2k, 2k+1 of each page (chunk 9 is out of bounds: zeros)
+            tma_load_5d_pair(dst, &tmQK, 0, 0, 2 * k, 0, pg[0], fb);
+            tma_load_5d_pair(dst + kQkBox, &tmQK, 0, 0, 2 * k, 0, pg[1], fb);
+          }
+        }
+        ++piece;
       }
-      if (rank == 0) mbar_expect_tx(smem_u32(&q_full), 2 * kQBytes);
-      const int row0 = b * rows_seq + rb * 128 + 64 * (int)rank;
-      for (int c = 0; c < 9; ++c)
-        tma_load_2d_pair(sQ + c * kChunk, &tmQ, c * 64, row0, lead_qfull);
-      ++q_issued;
-      for (int x = x0; x < x1 && ok; ++x) {
-        int page, slot0;
-        page_of(P, b, L, x, (int)rank, page, slot0);
-        // one box = chunks [3k, 3k+3) of the page (64 slots x 64 columns each)
-        for (int k = 0; k < 9 / kQkChunks; ++k, ++it) {
-          const int s = it % kQkStages;
-          if (!mbar_wait(smem_u32(&qk_empty[s]), ((it / kQkStages) & 1) ^ 1, abort_p, 1, it)) {
-            ok = false;
-            break;
-          }
-          const uint32_t fb = lead_full0 + s * 8;
-          if (rank == 0) mbar_expect_tx(smem_u32(&qk_full[s]), 2 * kQkStageBytes);
-          tma_load_4d_pair(sQk + s * kQkStageBytes, &tmQK, 0, slot0, kQkChunks * k, page, fb);
-        }
+      if (!ok && rank == 0) {
+        // Leaving early: wait (bounded) until the boxes already issued have
+        // landed, so that no copy writes into this pair's shared memory after
+        // it exits.  Only the leader's barriers count bytes; they count both
+        // CTAs' boxes of a stage, and the peer waits for the leader at the
+        // final cluster barrier.  A stage the peer never issued cannot
+        // complete, so each wait is bounded on its own.
+        for (uint32_t i = it > (uint32_t)kQkStages ? it - kQkStages : 0u; i < it; ++i)
+          mbar_wait_bounded(smem_u32(&qk_full[i % kQkStages]), (i / kQkStages) & 1, kDrainNs);
+        if (q_issued > 0) mbar_wait_bounded(smem_u32(&q_full), (q_issued - 1) & 1, kDrainNs);
       }
-      ++piece;
-    }
-    if (!ok && rank == 0) {
-      // Leaving early: wait (bounded) until the boxes already issued have
-      // landed, so that no copy writes into this pair's shared memory after
-      // it exits.  Only the leader's barriers count bytes; they count both
-      // CTAs' boxes of a stage, and the peer waits for the leader at the
-      // final cluster barrier.  A stage the peer never issued cannot
-      // complete, so each wait is bounded on its own.
-      for (uint32_t i = it > (uint32_t)kQkStages ? it - kQkStages : 0u; i < it; ++i)
-        mbar_wait_bounded(smem_u32(&qk_full[i % kQkStages]), (i / kQkStages) & 1, kDrainNs);
-      if (q_issued > 0) mbar_wait_bounded(smem_u32(&q_full), (q_issued - 1) & 1, kDrainNs);
-    }
-  } else if (warp == 2 || warp == 3) {
-    // ======  PV loader warps (cp.async): this CTA's latent half of page p  ======
-    // Warp 2 fills the stages of page 0, warp 3 those of page 1.  The copies
-    // go through the load/store path rather than the bulk-copy engine, which
-    // is busy with the QK boxes.  Each stage lands as [n][chunk][slot][64
-    // columns] for latent chunks 4n + 2r + {0, 1}; rows past the sequence
-    // are written as zeros.
-    const int mine = warp - 2;
-    uint32_t it = 0;
-    PieceIter pi;
-    pi.init(P.start, V, lo, hi);
-    int v, x0, x1;
-    bool ok = true;
-    while (ok && pi.next(v, x0, x1)) {
-      const int b = v / P.R;
-      const int L = P.seq_lens[b];
-      for (int x = x0; x < x1 && ok; ++x)
-        for (int p = 0; p < 2; ++p, ++it) {
-          if (p != mine) continue;
-          // same row placement as the QK boxes: shared-memory row i holds
-          // slot i + slot0 (slot0 <= 0; a partial page sits at the bottom),
-          // and slot0 == kPage marks a page past the context (all zeros)
-          int page, slot0;
-          page_of(P, b, L, x, p, page, slot0);
-          const int s = it % kPvStages;
-          const bool got = mbar_wait(smem_u32(&pv_empty[s]), ((it / kPvStages) & 1) ^ 1,
-                                     abort_p, 11, it);
-          if (!__all_sync(0xffffffffu, got)) { ok = false; break; }
-          const uint8_t* src = P.pool + (size_t)page * (kPage * kD * 2);
-          const uint32_t dst = sPv + s * kPvStageBytes;
-#pragma unroll 8
-          for (int i = 0; i < 64; ++i) {
-            // one 512-byte row per warp step: 4 chunks x 8 units of 16 B
-            const int row = i, q4 = lane >> 3, u = lane & 7;
-            const int chunk = 4 * (q4 >> 1) + 2 * (int)rank + (q4 & 1);
-            const int srow = row + slot0;
-            const uint32_t d = dst + q4 * kChunk + row * 128 + ((u ^ (row & 7)) << 4);
-            if (slot0 < kPage && srow >= 0)
-              cp_async16(d, src + srow * (kD * 2) + chunk * 128 + u * 16);
-            else
-              st_shared_zero16(d);
-          }
-          if (slot0 != 0) fence_proxy_async_smem();
-          cp_async_arrive_noinc(smem_u32(&pv_full[s]));
-        }
-    }
-    asm volatile("cp.async.wait_all;" ::: "memory");
-  } else if (warp == 1 && lane == 0 && rank == 1) {
-    // ======  peer relay: forward landed PV stages to the leader's barriers  ======
-    const uint32_t lead0 = mapa_shared(smem_u32(&pv_full[0]), 0);
-    PieceIter pi;
-    pi.init(P.start, V, lo, hi);
-    int v, x0, x1;
-    uint32_t it = 0;
-    bool ok = true;
-    while (ok && pi.next(v, x0, x1)) {
-      for (int x = x0; x < x1 && ok; ++x)
-        for (int p = 0; p < 2; ++p, ++it) {
-          const int s = it % kPvStages;
-          if (!mbar_wait(smem_u32(&pv_full[s]), (it / kPvStages) & 1, abort_p, 14, it)) {
-            ok = false;
-            break;
-          }
-          fence_proxy_async_smem();
-          mbar_arrive_cluster(lead0 + s * 8);
-        }
-    }
-  } else if (warp == 1 && lane == 0 && rank == 0) {
-    // =================  MMA issuer (leader CTA)  =================
-    const uint32_t idesc_qk = idesc_bf16_f32(128, 128, false, false);
-    const uint32_t idesc_pv = idesc_bf16_f32(128, 256, false, true);
-    uint32_t itq = 0, itv = 0;
-    int j = 0;  // block counter of this worker
-    PieceIter pi;
-    pi.init(P.start, V, lo, hi);
-    int v, x0, x1, piece = 0;
-    bool ok = true;
-    int pend = -1;            // block whose PV is pending
-    bool pend_first = false;  // ... is the first block of its piece
-    int pend_piece = 0;
-    auto issue_pv = [&](int jb, bool first, int pc) -> bool {
-      if (!mbar_wait(smem_u32(&p_full), jb & 1, abort_p, 4, jb)) return false;
-      if (first && pc > 0 && !mbar_wait(smem_u32(&o_empty), (pc - 1) & 1, abort_p, 5, pc))
-        return false;
-      tc_fence_after();
-      for (int p = 0; p < 2; ++p, ++itv) {
-        const int s = itv % kPvStages;
-        if (!mbar_wait(smem_u32(&pv_full[s]), (itv / kPvStages) & 1, abort_p, 12, itv))
-          return false;
-        // The stage was written by cp.async and st.shared (generic proxy);
-        // the MMA reads it through the async proxy.  The writes are ordered
-        // before this thread by the barrier; the proxy fence makes them
-        // visible to the MMAs this thread issues next.  (The peer's half
-        // is fenced the same way by its relay lane.)
-        fence_proxy_async_smem();
-        tc_fence_after();
-        const uint32_t st = sPv + s * kPvStageBytes;
-        for (int n = 0; n < 2; ++n) {
-#pragma unroll
-          for (int kk = 0; kk < 4; ++kk) {
-            const uint64_t ad = sw128_desc(sP + p * kChunk + kk * 32, 16, 1024);
-            const uint64_t bd = sw128_desc(st + n * 2 * kChunk + kk * 2048, kChunk, 1024);
-            const uint32_t acc = (first && p == 0 && kk == 0) ? 0u : 1u;
-            mma_bf16_ss<2>(tmem + kTmemO + 128 * n, ad, bd, idesc_pv, acc);
-          }
-        }
-        mma_commit_2_mc(smem_u32(&pv_empty[s]), 3);
+    } else if (warp == 2 || warp == 3) {
+      // ======  PV loader warps (cp.async): this CTA's latent half  ======
+      // Stage order per block: page p = 0..3, latent half n = 0..1; warp 2
+      // fills the even stages, warp 3 the odd ones.  A stage lands as
+      // [2 chunks][64 slots][128 B] for latent chunks 4n + 2r + {0, 1} of
+      // page p; rows past the sequence and pages past it are zeros.
+      const int mine = warp - 2;
+      uint32_t it = 0;
+      PieceIter pi;
+      pi.init(P.start, V, lo, hi);
+      int v, x0, x1;
+      bool ok = true;
+      const int rsub = lane >> 4, cc = (lane >> 3) & 1, u = lane & 7;
+      while (ok && pi.next(v, x0, x1)) {
+        const int b = v / P.R;
+        const int L = P.seq_lens[b];
+        for (int x = x0; x < x1 && ok; ++x)
+          for (int p = 0; p < 4 && ok; ++p)
+            for (int n = 0; n < 2; ++n, ++it) {
+              if ((int)(it & 1) != mine) continue;
+              const int pg = page_of(P, b, L, x, p);
+              const int valid = pg < 0 ? 0 : min(L - (x * kBlk + p * kPage), kPage);
+              const int s = it % kPvStages;
+              const bool got = mbar_wait(smem_u32(&pv_empty[s]), ((it / kPvStages) & 1) ^ 1,
+                                         abort_p, 11, it);
+              if (!__all_sync(0xffffffffu, got)) { ok = false; break; }
+              const uint8_t* src = P.pool + (size_t)(pg < 0 ? 0 : pg) * kPageBytes +
+                                   (4 * n + 2 * (int)rank + cc) * 128 + u * 16;
+              const uint32_t dst = sPv + s * kPvStageBytes + cc * kChunk + (u << 4);
+  #pragma unroll 8
+              for (int i = 0; i < kPage; i += 2) {
+                const int row = i + rsub;
+                const uint32_t d = dst + row * 128;
+                const uint32_t dsw = d ^ ((uint32_t)(row & 7) << 4);
+                if (row < valid)
+                  cp_async16(dsw, src + (size_t)row * (kD * 2));
+                else
+                  st_shared_zero16(dsw);
+              }
+              if (valid < kPage) fence_proxy_async_smem();
+              cp_async_arrive_noinc(smem_u32(&pv_full[s]));
+            }
       }
-      mma_commit_2_mc(smem_u32(&pv_done), 3);
-      return true;
-    };
-    while (ok && pi.next(v, x0, x1)) {
-      if (!mbar_wait(smem_u32(&q_full), piece & 1, abort_p, 6, piece)) { ok = false; break; }
-      tc_fence_after();
-      for (int x = x0; x < x1 && ok; ++x, ++j) {
-        // QK(j) into S[j & 1]
-        const uint32_t sd = tmem + kTmemS + 64 * (j & 1);
-        for (int k = 0; k < 9 / kQkChunks; ++k, ++itq) {
+      asm volatile("cp.async.wait_all;" ::: "memory");
+    } else if (warp == 1 && lane == 0 && rank == 1) {
+      // ======  peer relay: forward landed PV stages to the leader's barriers  ======
+      const uint32_t lead0 = mapa_shared(smem_u32(&pv_full[0]), 0);
+      PieceIter pi;
+      pi.init(P.start, V, lo, hi);
+      int v, x0, x1;
+      uint32_t it = 0;
+      bool ok = true;
+      while (ok && pi.next(v, x0, x1)) {
+        for (int x = x0; x < x1 && ok; ++x)
+          for (int k = 0; k < kPvStagesPerBlock; ++k, ++it) {
+            const int s = it % kPvStages;
+            if (!mbar_wait(smem_u32(&pv_full[s]), (it / kPvStages) & 1, abort_p, 14, it)) {
+              ok = false;
+              break;
+            }
+            fence_proxy_async_smem();
+            mbar_arrive_cluster(lead0 + s * 8);
+          }
+      }
+    } else if (warp == 1 && lane == 0 && rank == 0) {
+      // =================  MMA issuer (leader CTA)  =================
+      // Two streams share the tensor pipe: QK of block jq and PV of an
+      // earlier block jp.  Each turn issues at most one QK stage and one PV
+      // stage, each only if its operands have landed, so both rings drain
+      // steadily and the loads of each ring overlap the other stream's MMAs.
+      // QK(jq) writes S buffer jq & 1, which the softmax of block jq - 2
+      // releases when it hands over P(jq - 2): QK(jq) waits until PV(jq - 2)
+      // has begun.  PV(jp) begins once P(jp) is in and, for the first block
+      // of a piece, once the previous piece's epilogue has released O.
+      const uint32_t idesc_qk = idesc_bf16_f32(128, 256, false, false);
+      const uint32_t idesc_pv = idesc_bf16_f32(128, 256, false, true);
+      PieceIter qi, vi;
+      qi.init(P.start, V, lo, hi);
+      vi.init(P.start, V, lo, hi);
+      int qv, qx0 = 0, qx1 = 0, vv, vx0 = 0, vx1 = 0;
+      bool q_more = qi.next(qv, qx0, qx1), v_more = vi.next(vv, vx0, vx1);
+      int qx = qx0, q_piece = 0, jq = 0, kq = 0;   // QK: block, piece, stage
+      bool q_in = false;                           // Q of this QK piece landed
+      int vx = vx0, v_piece = 0, jp = 0, tp = 0;   // PV: block, piece, stage 0..7
+      bool p_in = false;                           // P of block jp in (and O free)
+      uint32_t itq = 0, itv = 0;
+      bool ok = true;
+      uint64_t t_stall = 0;                        // start of the current idle spell
+      uint32_t spins = 0;
+      while (ok && (q_more || v_more)) {
+        bool progressed = false;
+        // ---------------- one QK stage ----------------
+        if (q_more && jq <= jp + (p_in ? 1 : 0) + 1) {
+          bool ready = true;
+          if (!q_in) {
+            ready = mbar_try_wait(smem_u32(&q_full), q_piece & 1);
+            if (ready) q_in = true;
+          }
           const int s = itq % kQkStages;
-          if (!mbar_wait(smem_u32(&qk_full[s]), (itq / kQkStages) & 1, abort_p, 3, itq)) {
-            ok = false;
-            break;
-          }
-          tc_fence_after();
-          const uint32_t st = sQk + s * kQkStageBytes;
-          for (int cc = 0; cc < kQkChunks; ++cc) {
-            const int c = kQkChunks * k + cc;  // 64-column chunk of the 576
+          if (ready && mbar_try_wait(smem_u32(&qk_full[s]), (itq / kQkStages) & 1)) {
+            tc_fence_after();
+            const uint32_t sd = tmem + kTmemS + 128 * (jq & 1);
+            const uint32_t st = sQk + s * kQkStageBytes;
+            const int ncc = (kq == kQkStagesPerBlock - 1) ? 1 : 2;
+            for (int cc = 0; cc < ncc; ++cc) {
+              const int c = 2 * kq + cc;  // 64-column chunk of the 576
 #pragma unroll
-            for (int kk = 0; kk < 4; ++kk) {
-              const uint64_t ad = sw128_desc(sQ + c * kChunk + kk * 32, 16, 1024);
-              const uint64_t bd = sw128_desc(st + cc * kChunk + kk * 32, 16, 1024);
-              mma_bf16_ss<2>(sd, ad, bd, idesc_qk, (c | kk) ? 1u : 0u);
+              for (int kk = 0; kk < 4; ++kk) {
+                const uint64_t ad = sw128_desc(sQ + c * kChunk + kk * 32, 16, 1024);
+                // 16 slot groups (8 per page) 2 KB apart
+                const uint64_t bd = sw128_desc(st + cc * 1024 + kk * 32, 16, 2048);
+                mma_bf16_ss<2>(sd, ad, bd, idesc_qk, (c | kk) ? 1u : 0u);
+              }
+            }
+            mma_commit_2_mc(smem_u32(&qk_empty[s]), 3);
+            ++itq;
+            progressed = true;
+            if (++kq == kQkStagesPerBlock) {
+              kq = 0;
+              mma_commit_2_mc(smem_u32(&s_full[jq & 1]), 3);
+              ++jq;
+              if (++qx == qx1) {
+                mma_commit_2_mc(smem_u32(&q_empty), 3);
+                q_more = qi.next(qv, qx0, qx1);
+                qx = qx0;
+                ++q_piece;
+                q_in = false;
+              }
             }
           }
-          mma_commit_2_mc(smem_u32(&qk_empty[s]), 3);
         }
-        if (!ok) break;
-        mma_commit_2_mc(smem_u32(&s_full[j & 1]), 3);
-        if (x == x1 - 1) mma_commit_2_mc(smem_u32(&q_empty), 3);
-        if (pend >= 0 && !issue_pv(pend, pend_first, pend_piece)) { ok = false; break; }
-        pend = j; pend_first = (x == x0); pend_piece = piece;
+        // ---------------- one PV stage ----------------
+        if (v_more && jp < jq) {
+          if (!p_in) {
+            p_in = mbar_try_wait(smem_u32(&p_full), jp & 1) &&
+                   (vx != vx0 || v_piece == 0 ||
+                    mbar_try_wait(smem_u32(&o_empty), (v_piece - 1) & 1));
+            if (p_in) tc_fence_after();
+          }
+          const int s = itv % kPvStages;
+          if (p_in && mbar_try_wait(smem_u32(&pv_full[s]), (itv / kPvStages) & 1)) {
+            // The stage was written by cp.async and st.shared (generic
+            // proxy); the MMA reads it through the async proxy.  The writes
+            // are ordered before this thread by the barrier; the proxy fence
+            // makes them visible to the MMAs issued next.  (The peer's half
+            // is fenced the same way by its relay lane.)
+            fence_proxy_async_smem();
+            tc_fence_after();
+            const int p = tp >> 1, n = tp & 1;
+            const bool first = (vx == vx0);
+            const uint32_t st = sPv + s * kPvStageBytes;
+#pragma unroll
+            for (int kk = 0; kk < 4; ++kk) {
+              const uint64_t ad = sw128_desc(sP + p * kChunk + kk * 32, 16, 1024);
+              const uint64_t bd = sw128_desc(st + kk * 2048, kChunk, 1024);
+              const uint32_t acc = (first && p == 0 && kk == 0) ? 0u : 1u;
+              mma_bf16_ss<2>(tmem + kTmemO + 128 * n, ad, bd, idesc_pv, acc);
+            }
+            mma_commit_2_mc(smem_u32(&pv_empty[s]), 3);
+            ++itv;
+            progressed = true;
+            if (++tp == kPvStagesPerBlock) {
+              tp = 0;
+              mma_commit_2_mc(smem_u32(&pv_done), 3);
+              ++jp;
+              p_in = false;
+              if (++vx == vx1) {
+                v_more = vi.next(vv, vx0, vx1);
+                vx = vx0;
+                ++v_piece;
+              }
+            }
+          }
+        }
+        // ---------------- bounded idle ----------------
+        if (progressed) {
+          spins = 0;
+        } else if ((++spins & 63u) == 0) {
+          const uint64_t now = globaltimer();
+          if (spins == 64) t_stall = now;
+          if (*abort_p) {
+            ok = false;
+          } else if (now - t_stall > MLA_WAIT_NS) {
+            raise_flag(kFlagTimeout);
+            record_timeout(3, (uint32_t)jq, (uint32_t)jp);
+            *abort_p = 1;
+            ok = false;
+          }
+        }
       }
-      ++piece;
+      if (!ok) {
+        // Leaving early: one more commit tracks every MMA issued so far; wait
+        // (bounded) for it, so that no MMA still reads shared memory or writes
+        // TMEM when the pair frees them.
+        mma_commit_2_mc(smem_u32(&mma_drain), 1);
+        mbar_wait_bounded(smem_u32(&mma_drain), 0, kDrainNs);
+      }
     }
-    if (ok && pend >= 0) ok = issue_pv(pend, pend_first, pend_piece);
-    if (!ok) {
-      // Leaving early: one more commit tracks every MMA issued so far; wait
-      // (bounded) for it, so that no MMA still reads shared memory or writes
-      // TMEM when the pair frees them.
-      mma_commit_2_mc(smem_u32(&mma_drain), 1);
-      mbar_wait_bounded(smem_u32(&mma_drain), 0, kDrainNs);
-    }
-  } else if (warp >= kSoftmaxWarp0) {
+  } else {
+    setmaxnreg_inc<kRegsSoftmax>();
     // =================  softmax + epilogue (both CTAs)  =================
-    const int tid = threadIdx.x - kSoftmaxWarp0 * 32;  // = TMEM lane
-    const int h = tid & 63, half = tid >> 6;
-    const uint32_t lane_addr = (uint32_t)(32 * (warp - kSoftmaxWarp0)) << 16;
+    const int sw = warp - kSoftmaxWarp0;
+    const int quad = sw & 3, ch = sw >> 2;           // TMEM lane quadrant, column half
+    const int tl = 32 * quad + lane;                 // TMEM lane
+    const int h = tl & 63, hh = tl >> 6;             // row of this CTA, token half
+    const int pb = 2 * hh + ch;                      // page of the block this thread scores
+    const uint32_t lane_addr = (uint32_t)(32 * quad) << 16;
     const uint32_t lead_pfull = mapa_shared(smem_u32(&p_full), 0);
     const uint32_t lead_oempty = mapa_shared(smem_u32(&o_empty), 0);
-    const uint32_t prow = sP + half * kChunk + h * 128;
+    const uint32_t prow = sP + pb * kChunk + h * 128;
     PieceIter pi;
     pi.init(P.start, V, lo, hi);
     int v, x0, x1;
@@ -457,35 +529,33 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(dtc::kThreads, 1)
       const int b = v / P.R, rb = v % P.R;
       const int L = P.seq_lens[b];
       const int grow = rb * 128 + 64 * (int)rank + h;      // row within the sequence
-      const int tl = P.tail != nullptr ? P.tail[b] : 0;
-      const int limit = L + tl - P.S_q + grow / P.H + 1;    // visible tokens t < limit
+      const int tail = P.tail != nullptr ? P.tail[b] : 0;
+      const int limit = min(L, L + tail - P.S_q + grow / P.H + 1);  // visible tokens t < limit
       float m = -INFINITY, l = 0.f;
       bool o_started = false;
       for (int x = x0; x < x1; ++x, ++j) {
         const bool got = mbar_wait(smem_u32(&s_full[j & 1]), (j >> 1) & 1, abort_p, 7, j);
         uint32_t s_raw[64];
         float mx = -INFINITY;
-        // token t of this lane's page: first + c - shift, valid if c >= shift
-        const int first = x * kBlk + half * kPage;
-        const int valid = min(L - first, kPage);
-        const int shift = valid > 0 ? kPage - valid : kPage;
-        const int cmax = limit - first + shift;  // columns c < cmax are visible
+        const int cmax = limit - (x * kBlk + pb * kPage);  // columns c < cmax are visible
         if (__all_sync(0xffffffffu, got)) {
           tc_fence_after();
           uint32_t (&a)[32] = *reinterpret_cast<uint32_t(*)[32]>(&s_raw[0]);
           uint32_t (&c2)[32] = *reinterpret_cast<uint32_t(*)[32]>(&s_raw[32]);
-          const uint32_t sa = tmem + lane_addr + kTmemS + 64 * (j & 1);
+          const uint32_t sa = tmem + lane_addr + kTmemS + 128 * (j & 1) + 64 * ch;
           tmem_ld32(sa, a);
           tmem_ld32(sa + 32, c2);
           tmem_wait_ld();
 #pragma unroll
           for (int c = 0; c < 64; ++c)
-            if (c >= shift && c < cmax) mx = fmaxf(mx, __uint_as_float(s_raw[c]));
+            if (c < cmax) mx = fmaxf(mx, __uint_as_float(s_raw[c]));
         }
-        red_max[j & 1][half][h] = mx;
-        // one barrier: partner's max visible, and everyone agrees to go on
-        if (named_bar_or(1, 128, !got || *abort_p)) { dead = true; break; }
-        mx = fmaxf(mx, red_max[j & 1][half ^ 1][h]);
+        red_max[j & 1][pb][h] = mx;
+        // one barrier: the other pages' maxima visible, and everyone agrees
+        // to go on
+        if (named_bar_or(1, kSoftmaxThreads, !got || *abort_p)) { dead = true; break; }
+#pragma unroll
+        for (int q2 = 0; q2 < 4; ++q2) mx = fmaxf(mx, red_max[j & 1][q2][h]);
         const float m_blk = mx * P.scale_log2;
         // Lazy rescale: a row moves its running max only when the block max
         // exceeds it by more than 2^kRescaleLog2.  TMEM loads/stores are
@@ -499,10 +569,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(dtc::kThreads, 1)
 #pragma unroll
         for (int e = 0; e < 32; ++e) {
           const int c0 = 2 * e;
-          const float p0 = (c0 >= shift && c0 < cmax)
+          const float p0 = c0 < cmax
                                ? ex2_approx(fmaf(__uint_as_float(s_raw[c0]), P.scale_log2, -m_use))
                                : 0.f;
-          const float p1 = (c0 + 1 >= shift && c0 + 1 < cmax)
+          const float p1 = c0 + 1 < cmax
                                ? ex2_approx(fmaf(__uint_as_float(s_raw[c0 + 1]), P.scale_log2,
                                                  -m_use))
                                : 0.f;
@@ -515,17 +585,16 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(dtc::kThreads, 1)
         if (__all_sync(0xffffffffu, ok)) {
           if (o_started && __any_sync(0xffffffffu, need)) {
             tc_fence_after();
-            for (int n = 0; n < 2; ++n)
-              for (int cc = 0; cc < 4; ++cc) {
-                uint32_t r[32];
-                const uint32_t oa = tmem + lane_addr + kTmemO + 128 * n + 32 * cc;
-                tmem_ld32(oa, r);
-                tmem_wait_ld();
+            for (int cc = 0; cc < 4; ++cc) {
+              uint32_t r[32];
+              const uint32_t oa = tmem + lane_addr + kTmemO + 128 * ch + 32 * cc;
+              tmem_ld32(oa, r);
+              tmem_wait_ld();
 #pragma unroll
-                for (int i = 0; i < 32; ++i)
-                  r[i] = __float_as_uint(__uint_as_float(r[i]) * alpha);
-                tmem_st32(oa, r);
-              }
+              for (int i = 0; i < 32; ++i)
+                r[i] = __float_as_uint(__uint_as_float(r[i]) * alpha);
+              tmem_st32(oa, r);
+            }
             tmem_wait_st();
           }
 #pragma unroll
@@ -549,29 +618,30 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(dtc::kThreads, 1)
       // ---------------- epilogue of the piece ----------------
       const int jl = j - 1;
       const bool got = mbar_wait(smem_u32(&pv_done), jl & 1, abort_p, 10, jl);
-      red_sum[half][h] = l;
-      if (named_bar_or(1, 128, !got || *abort_p)) { dead = true; break; }
+      red_sum[pb][h] = l;
+      if (named_bar_or(1, kSoftmaxThreads, !got || *abort_p)) { dead = true; break; }
       tc_fence_after();
-      const float lt = l + red_sum[half ^ 1][h];
+      const float lt = red_sum[0][h] + red_sum[1][h] + red_sum[2][h] + red_sum[3][h];
       const float inv = lt > 0.f ? 1.f / lt : 0.f;
       const long long slot = (long long)worker + v;
       const long long row = slot * 128 + 64 * (int)rank + h;
-      float* dst = P.ws_o + row * kDC;
-      for (int n = 0; n < 2; ++n)
-        for (int cc = 0; cc < 4; ++cc) {
-          uint32_t r[32];
-          tmem_ld32(tmem + lane_addr + kTmemO + 128 * n + 32 * cc, r);
-          tmem_wait_ld();
-          float4* d4 = reinterpret_cast<float4*>(dst + 256 * n + 128 * half + 32 * cc);
+      // this warp writes latent half n = ch of its lanes: columns
+      // 256n + 128hh + [0, 128)
+      float* dst = P.ws_o + row * kDC + 256 * ch + 128 * hh;
+      for (int cc = 0; cc < 4; ++cc) {
+        uint32_t r[32];
+        tmem_ld32(tmem + lane_addr + kTmemO + 128 * ch + 32 * cc, r);
+        tmem_wait_ld();
+        float4* d4 = reinterpret_cast<float4*>(dst + 32 * cc);
 #pragma unroll
-          for (int i = 0; i < 8; ++i)
-            d4[i] = make_float4(__uint_as_float(r[4 * i]) * inv, __uint_as_float(r[4 * i + 1]) * inv,
-                                __uint_as_float(r[4 * i + 2]) * inv,
-                                __uint_as_float(r[4 * i + 3]) * inv);
-        }
-      if (half == 0)
+        for (int i = 0; i < 8; ++i)
+          d4[i] = make_float4(__uint_as_float(r[4 * i]) * inv, __uint_as_float(r[4 * i + 1]) * inv,
+                              __uint_as_float(r[4 * i + 2]) * inv,
+                              __uint_as_float(r[4 * i + 3]) * inv);
+      }
+      if (pb == 0)
         P.ws_lse[row] = lt > 0.f ? (m + log2f(lt)) * 0.69314718055994531f : -INFINITY;
-      named_bar_sync(1, 128);  // red_sum is rewritten by the next piece
+      named_bar_sync(1, kSoftmaxThreads);  // red_sum is rewritten by the next piece
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive_cluster(lead_oempty);
@@ -601,13 +671,16 @@ inline mla_status launch_decode_tc_impl(
     const uint32_t box[2] = {64, 64};
     if (!make_tmap(&tQ, qbuf, 2, dims, strides, box)) return MLA_ERR_CUDA;
   }
-  // The pool [n_pages][64 slots][576] seen as 64-column chunks: element
-  // (col, slot, chunk, page) at page*73728 + slot*1152 + chunk*128 + col*2 bytes.
+  // The pool [n_pages][64 slots][576] seen as (64 columns, 8 slots, 9
+  // chunks, 8 slot groups, pages): element (col, s, chunk, g, page) at
+  // page*73728 + (8g + s)*1152 + chunk*128 + col*2 bytes.  A box of two
+  // chunks of one page lands as [g][chunk][s][64 columns].
   {
-    const uint64_t dims[4] = {64, (uint64_t)kPage, 9, (uint64_t)n_pages};
-    const uint64_t strides[3] = {(uint64_t)kD * 2, 128, (uint64_t)kD * 2 * kPage};
-    const uint32_t box[4] = {64, 64, (uint32_t)kQkChunks, 1};
-    if (!make_tmap(&tQK, pool, 4, dims, strides, box)) return MLA_ERR_CUDA;
+    const uint64_t dims[5] = {64, 8, 9, 8, (uint64_t)n_pages};
+    const uint64_t strides[4] = {(uint64_t)kD * 2, 128, (uint64_t)kD * 2 * 8,
+                                 (uint64_t)kPageBytes};
+    const uint32_t box[5] = {64, 8, 2, 8, 1};
+    if (!make_tmap(&tQK, pool, 5, dims, strides, box)) return MLA_ERR_CUDA;
   }
   DecodeTcParams p;
   p.pool = static_cast<const uint8_t*>(pool);
@@ -622,7 +695,7 @@ inline mla_status launch_decode_tc_impl(
   p.B = B;
   p.S_q = S_q;
   p.H = H;
-  p.R = (S_q * H) / 128;
+  p.R = (S_q * H + 127) / 128;  // the last row block may be padded
   p.G = G;
   p.scale_log2 = scale * 1.4426950408889634f;
   if (cudaFuncSetAttribute(decode_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,

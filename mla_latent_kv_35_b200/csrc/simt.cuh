@@ -274,18 +274,21 @@ __global__ void __launch_bounds__(256) decode_simt_kernel(
 // ---------------------------------------------------------------------------
 // Log-sum-exp combine of the pieces of every virtual sequence.
 //   o = sum_k w_k o_k / sum_k w_k, w_k = exp(lse_k - max lse), lse = max + ln sum w
-// Grid (V, ceil(rows_per_v / 8)), one warp per row.
+// Grid (V, ceil(rows_per_v / 8)), one warp per row.  Virtual sequence v is
+// row block v % R of sequence v / R: rows_per_v workspace rows, of which the
+// ones past the sequence's rows_seq query rows are padding and skipped.
 // ---------------------------------------------------------------------------
 __global__ void __launch_bounds__(256) combine_kernel(const float* ws_lse, const float* ws_o,
                                                       const int32_t* start, int V, int R, int G,
-                                                      int rows_per_v, int d_c, float* o_lat,
-                                                      float* lse) {
+                                                      int rows_per_v, int rows_seq, int d_c,
+                                                      float* o_lat, float* lse) {
   const int v = blockIdx.x;
   const int r = blockIdx.y * 8 + (threadIdx.x >> 5);
   const int lane = threadIdx.x & 31;
-  if (r >= rows_per_v) return;
+  const int row_in_seq = (v % R) * rows_per_v + r;
+  if (r >= rows_per_v || row_in_seq >= rows_seq) return;
   const int total = start[V];
-  const long long out_row = (long long)(v / R) * R * rows_per_v + (long long)(v % R) * rows_per_v + r;
+  const long long out_row = (long long)(v / R) * rows_seq + row_in_seq;
   float* dst = o_lat + out_row * d_c;
   if (start[v + 1] == start[v]) {
     for (int c = lane; c < d_c; c += 32) dst[c] = 0.f;

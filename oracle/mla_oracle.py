@@ -384,3 +384,77 @@ def combine_splits(o_parts, lse_parts):
     z = w.sum(axis=0)
     o = (w[..., None] * o_parts).sum(axis=0) / z[..., None]
     return o, m + np.log(z)
+
+
+# ---------------------------------------------------------------------------
+# 8-bit latent cache (deepforge page, §4 "Build it yourself", stretch goals:
+# quantize the latent to 8 bits and measure the extra error a production
+# cache would pay).  The pages fix neither the format nor the scale; the
+# reading used here (R16): each token's 512-number latent is stored in the
+# 8-bit float format E4M3 (1 sign, 4 exponent bits with bias 7, 3 mantissa
+# bits, largest finite value 448, no infinities) after division by one
+# per-token scale s = max|c| / 448; the 64-number RoPE key is kept in a
+# 16-bit float.  The scale and the division are single-precision steps (the
+# precision the GPU quantizer takes the decision in), so both sides produce
+# the same codes.
+# ---------------------------------------------------------------------------
+
+E4M3_MAX = 448.0
+
+
+def round_to_grid(x, mant_bits: int, emin: int, max_value: float):
+    """Round x to the nearest number of a binary floating-point format with
+    `mant_bits` stored mantissa bits and smallest normal exponent `emin`
+    (subnormals below 2^emin), ties to even, saturating at +-max_value.
+
+    Inside binade [2^e, 2^(e+1)) the representable numbers are multiples of
+    2^(e - mant_bits); below 2^emin they are multiples of 2^(emin - mant_bits).
+    """
+    x = np.asarray(x, dtype=F64)
+    a = np.abs(x)
+    e = np.floor(np.log2(np.where(a > 0, a, 1.0)))
+    e = np.maximum(e, emin)
+    quantum = np.exp2(e - mant_bits)
+    q = np.round(a / quantum) * quantum          # numpy rounds halves to even
+    q = np.minimum(q, max_value)
+    return np.sign(x) * q
+
+
+def e4m3_round(x):
+    """Nearest E4M3 value (3 mantissa bits, normals from 2^-6, max 448)."""
+    return round_to_grid(x, 3, -6, E4M3_MAX)
+
+
+def bf16_round(x):
+    """Nearest bfloat16 value (7 stored mantissa bits, 8 exponent bits)."""
+    return round_to_grid(x, 7, -126, 3.3895313892515355e38)
+
+
+def f16_round(x):
+    """Nearest IEEE half-precision value (10 stored mantissa bits, normals
+    from 2^-14, largest finite 65504)."""
+    return round_to_grid(x, 10, -14, 65504.0)
+
+
+def quantize_latent_fp8(C, KR):
+    """8-bit cache rows of tokens C [L, d_c], KR [L, d_r] (reading R16).
+
+    Per token t, in single precision: s_t = max_k |C[t, k]| / 448 (1 for an
+    all-zero latent) and x = C[t] / s_t, then c8_t = E4M3(x); the RoPE key is
+    stored as half precision, kr8_t = f16(KR[t]).  Returns (s [L],
+    c8 [L, d_c] E4M3 values, kr8 [L, d_r]); the cache the attention sees is
+    [s_t c8_t ; kr8_t] (dequantize_fp8).
+    """
+    C32 = np.asarray(C, dtype=np.float32)
+    m = np.abs(C32).max(axis=1) if C32.shape[1] else np.zeros(C32.shape[0], np.float32)
+    s = np.where(m > 0, m / np.float32(E4M3_MAX), np.float32(1.0)).astype(np.float32)
+    x = (C32 / s[:, None]).astype(np.float32)
+    c8 = e4m3_round(x.astype(F64))
+    kr8 = f16_round(np.asarray(KR, dtype=F64))
+    return s.astype(F64), c8, kr8
+
+
+def dequantize_fp8(s, c8, kr8):
+    """The cache numbers an 8-bit row stands for: (s c8, kr8)."""
+    s = np.asarray(s, dtype=F64)[:, None]
+    return s * np.asarray(c8, dtype=F64), np.asarray(kr8, dtype=F64)

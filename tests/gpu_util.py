@@ -62,5 +62,27 @@ def check(got, ref, dtype, what="", tol=None):
     return mx, mean, rel
 
 
+def check_stored_bf16(got, ref, what="", rotated=False):
+    """A value the GPU stores in bf16 against the oracle's fp64 value.
+
+    A bf16 store rounds to nearest: |error| <= u |ref| with the unit roundoff
+    u = 2^-8 of 8 significant bits.  A RoPE-rotated key (rotated=True) is
+    rounded twice: its pre-RoPE input is a bf16 projection output, and
+    rotating a pair mixes the two rounded inputs, so element e of pair (x, y)
+    may be off by u (|x_in| + |y_in|) <= u sqrt(2) |pair| before the final
+    rounding of u |ref_e|.  A little fp32 slack is added to both bounds."""
+    got = np.asarray(got, np.float64)
+    ref = np.asarray(ref, np.float64)
+    u = 2.0 ** -8
+    bound = u * np.abs(ref)
+    if rotated:
+        pair = np.sqrt(ref[0::2] ** 2 + ref[1::2] ** 2)
+        bound = bound + u * np.sqrt(2.0) * np.repeat(pair, 2)
+    bound = bound * (1 + 1e-3) + 1e-6
+    err = np.abs(got - ref)
+    assert (err <= bound).all(), \
+        f"{what}: worst error {err.max():.3e} (bound there {bound[np.argmax(err - bound)]:.3e})"
+
+
 def status():
     return B.mla_get_device_status()

@@ -245,11 +245,9 @@ def _run_decode(d, c, S_q, workers=0):
 
 
 def _expected_kernel(dtype, H, S_q):
-    """The split kernel mla_decode should pick: tensor cores for bf16 query
-    blocks of a multiple of 128 rows, CUDA cores otherwise."""
-    if dtype == "bf16" and (S_q * H) % 128 == 0:
-        return B.DECODE_KERNEL_TC
-    return B.DECODE_KERNEL_SIMT
+    """The split kernel mla_decode should pick: tensor cores for every bf16
+    shape (query blocks under 128 rows are padded), CUDA cores for fp32."""
+    return B.DECODE_KERNEL_TC if dtype == "bf16" else B.DECODE_KERNEL_SIMT
 
 
 def _decode_ref(d, c, b):
@@ -268,6 +266,8 @@ def _decode_ref(d, c, b):
     ("bf16", 16, 1, [40, 300]),
     ("bf16", 32, 1, [33, 200, 129]),
     ("bf16", 64, 1, [1, 190, 64]),
+    ("bf16", 96, 2, [3, 300, 257]),
+    ("bf16", 8, 2, [2, 70]),
 ])
 def test_decode_matches_oracle(dtype, H, S_q, lens):
     dc, dr = (64, 16) if dtype == "f32" else (512, 64)
