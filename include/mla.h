@@ -16,6 +16,9 @@
  *           their values are mixed (softmax attention over the cache).
  *   [CA-1]  crackai.dev "DeepSeek-V2", "How It Works": up-projections differ
  *           per head; the decoupled RoPE keys carry position separately.
+ *   [DF-4]  deepforge "DeepSeek-V2", §4 "Build it yourself", stretch goals:
+ *           quantize the latent to 8 bits and measure how much extra error a
+ *           production cache would pay.
  *
  * Conventions shared by every call
  *   - All pointers named "device" are CUDA device pointers owned by the
@@ -127,6 +130,62 @@ mla_status mla_cache_append(const mla_dims* dims, const void* c, int cs_tok,
                             const int32_t* batch_idx, const int32_t* pos,
                             const int32_t* page_table, int max_pages,
                             void* pool, int n_pages, int T, void* stream);
+
+/* 8-bit latent cache ([DF-4]: the stretch goal of quantizing the latent to
+ * 8 bits).  One 656-byte row per token:
+ *   bytes [0, 512)    c / s in E4M3 (1 sign, 4 exponent bits, bias 7, 3
+ *                     mantissa bits; largest finite 448), nearest even,
+ *                     saturating
+ *   bytes [512, 640)  k_rope / s in IEEE half precision
+ *   bytes [640, 644)  s = max(max|c| / 448, max|k_rope| / 65504) as fp32
+ *                     (1 for an all-zero row)
+ *   bytes [644, 656)  zero
+ * s and the quotients are correctly rounded single-precision divisions.  The
+ * cache numbers a row stands for are s * [c8 ; k16].  An 8-bit pool is
+ * [n_pages][page_size][656] bytes; page tables index it as the bf16 pool.
+ * Both calls need dtype MLA_BF16 (their inputs are bf16), d_latent == 512
+ * and d_rope == 64 (else MLA_ERR_UNSUPPORTED), and 16-byte aligned buffers. */
+#define MLA_FP8_ROW_BYTES 656
+
+/* A3 for the 8-bit cache: quantize each new token's [c ; k_rope] (bf16, as
+ * for mla_cache_append, row strides cs_tok and ks_tok multiples of 8) into
+ * the slot of (batch_idx[t], pos[t]) of pool8.  A page id outside
+ * [0, n_pages) skips the token and raises MLA_ERR_BOUNDS. */
+mla_status mla_cache_append_fp8(const mla_dims* dims, const void* c, int cs_tok,
+                                const void* kr, int ks_tok,
+                                const int32_t* batch_idx, const int32_t* pos,
+                                const int32_t* page_table, int max_pages,
+                                void* pool8, int n_pages, int T, void* stream);
+
+/* Quantize a whole bf16 pool [n_pages][page_size][576] into the 8-bit pool
+ * [n_pages][page_size][656] row by row (same pages and slots).  Slots that
+ * hold no token are converted too; their bytes are never read as cache. */
+mla_status mla_cache_quantize_fp8(const mla_dims* dims, const void* pool, void* pool8,
+                                  int n_pages, void* stream);
+
+/* Workspace bytes mla_decode_fp8 needs (mla_decode's, plus a half copy of
+ * the query); 0 for dims the 8-bit cache does not cover. */
+size_t mla_decode_fp8_workspace_size(const mla_dims* dims, int B, int S_q,
+                                     int num_workers);
+
+/* A4 + A5 on the 8-bit cache: the attention of mla_decode over the cache
+ * numbers the 8-bit rows stand for, s * [c8 ; k16] ([DF-0], [DF-1],
+ * [DF-4]).  qbuf, page_table, seq_lens, o_lat, lse and the split planning
+ * as for mla_decode; pool8 is the 8-bit pool [n_pages][64][656] bytes.  The
+ * tensor cores compute in IEEE half precision on the stored numbers: the
+ * query is converted to half (exact within half's range), the 8-bit codes
+ * to half (exact), each score is the fp32 product of s and the fp32 dot
+ * product, and the value product takes 64 * p * s rounded to half as its
+ * weights (the 64 keeps them in half's normal range; it is divided out);
+ * accumulation is fp32.  Needs dtype MLA_BF16, d_latent == 512, d_rope == 64, page_size ==
+ * 64 (else MLA_ERR_UNSUPPORTED), 1 <= S_q <= 2, a 256-byte aligned workspace
+ * of mla_decode_fp8_workspace_size bytes, and 16-byte aligned qbuf and
+ * pool8.  Device-side errors as for mla_decode. */
+mla_status mla_decode_fp8(const mla_dims* dims, const void* qbuf, const void* pool8,
+                          int n_pages, const int32_t* page_table, int max_pages,
+                          const int32_t* seq_lens, int B, int S_q, int num_workers,
+                          void* workspace, size_t ws_bytes, float* o_lat,
+                          float* lse, void* stream);
 
 /* A1 + A2 + A3 in one call: everything between the projection and the
  * decode ([DF-1]; the pages describe the steps, not this grouping).

@@ -27,7 +27,9 @@ EXPORTS = ("mla_project", "mla_absorb_q", "mla_rope", "mla_cache_append",
            "mla_out_proj", "mla_get_device_status", "mla_status_string",
            "mla_launch_count", "mla_selftest_wait_timeout", "mla_get_wait_diag",
            "mla_decode_noalloc", "mla_pre_attention", "mla_decode_partial",
-           "mla_combine_parts", "mla_decode_config", "mla_decode_noalloc_scratch_bytes")
+           "mla_combine_parts", "mla_decode_config", "mla_decode_noalloc_scratch_bytes",
+           "mla_cache_append_fp8", "mla_cache_quantize_fp8", "mla_decode_fp8",
+           "mla_decode_fp8_workspace_size")
 
 
 class MLAError(RuntimeError):
@@ -102,7 +104,15 @@ _SIGS = {
     "mla_decode_config": ([ctypes.POINTER(Dims), _I, _I, ctypes.POINTER(_I),
                            ctypes.POINTER(_I), ctypes.POINTER(_I)], _I),
     "mla_decode_noalloc_scratch_bytes": ([], _Z),
+    "mla_cache_append_fp8": ([ctypes.POINTER(Dims), _P, _I, _P, _I, _P, _P, _P, _I, _P,
+                              _I, _I, _P], _I),
+    "mla_cache_quantize_fp8": ([ctypes.POINTER(Dims), _P, _P, _I, _P], _I),
+    "mla_decode_fp8_workspace_size": ([ctypes.POINTER(Dims), _I, _I, _I], _Z),
+    "mla_decode_fp8": ([ctypes.POINTER(Dims), _P, _P, _I, _P, _I, _P, _I, _I, _I, _P, _Z,
+                        _P, _P, _P], _I),
 }
+
+FP8_ROW_BYTES = 656
 
 DECODE_KERNEL_SIMT, DECODE_KERNEL_TC = 0, 1
 
@@ -171,6 +181,34 @@ def mla_cache_append(dims: MLADims, c, cs_tok, kr, ks_tok, batch_idx, pos, page_
     _check("mla_cache_append", lib().mla_cache_append(
         ctypes.byref(dims.c()), _ptr(c), cs_tok, _ptr(kr), ks_tok, _ptr(batch_idx), _ptr(pos),
         _ptr(page_table), max_pages, _ptr(pool), n_pages, T, _stream()))
+
+
+def mla_cache_append_fp8(dims: MLADims, c, cs_tok, kr, ks_tok, batch_idx, pos, page_table,
+                         max_pages, pool8, n_pages, T):
+    _dev(c, kr, batch_idx, pos, page_table, pool8)
+    _check("mla_cache_append_fp8", lib().mla_cache_append_fp8(
+        ctypes.byref(dims.c()), _ptr(c), cs_tok, _ptr(kr), ks_tok, _ptr(batch_idx), _ptr(pos),
+        _ptr(page_table), max_pages, _ptr(pool8), n_pages, T, _stream()))
+
+
+def mla_cache_quantize_fp8(dims: MLADims, pool, pool8, n_pages):
+    _dev(pool, pool8)
+    _check("mla_cache_quantize_fp8", lib().mla_cache_quantize_fp8(
+        ctypes.byref(dims.c()), _ptr(pool), _ptr(pool8), n_pages, _stream()))
+
+
+def mla_decode_fp8_workspace_size(dims: MLADims, B: int, S_q: int, num_workers: int = 0) -> int:
+    return int(lib().mla_decode_fp8_workspace_size(ctypes.byref(dims.c()), B, S_q, num_workers))
+
+
+def mla_decode_fp8(dims: MLADims, qbuf, pool8, n_pages, page_table, max_pages, seq_lens, B, S_q,
+                   num_workers, workspace, o_lat, lse):
+    _dev(qbuf, pool8, page_table, seq_lens, workspace, o_lat, lse)
+    ws_bytes = workspace.numel() * workspace.element_size()
+    _check("mla_decode_fp8", lib().mla_decode_fp8(
+        ctypes.byref(dims.c()), _ptr(qbuf), _ptr(pool8), n_pages, _ptr(page_table), max_pages,
+        _ptr(seq_lens), B, S_q, num_workers, _ptr(workspace), ws_bytes, _ptr(o_lat), _ptr(lse),
+        _stream()))
 
 
 def mla_pre_attention(dims: MLADims, y, y_stride_tok, w_uk, qbuf, batch_idx, pos, page_table,

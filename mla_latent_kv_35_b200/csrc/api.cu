@@ -12,7 +12,9 @@
 
 #include "../../include/mla.h"
 #include "common.cuh"
+#include "decode_fp8.cuh"
 #include "decode_tc.cuh"
+#include "fp8.cuh"
 #include "gemm_tc.cuh"
 #include "simt.cuh"
 
@@ -74,8 +76,8 @@ EncodeTiledFn encode_fn() {
 
 // bf16 tensor of rank `rank` (<= 5), dims innermost first, byte strides of
 // dims 1.., 128-byte swizzle, zero fill out of bounds.
-bool make_tmap_bf16(CUtensorMap* m, const void* ptr, int rank, const uint64_t* dims,
-                    const uint64_t* strides_bytes, const uint32_t* box) {
+bool make_tmap_typed(CUtensorMapDataType type, CUtensorMap* m, const void* ptr, int rank,
+                     const uint64_t* dims, const uint64_t* strides_bytes, const uint32_t* box) {
   EncodeTiledFn fn = encode_fn();
   if (fn == nullptr) return false;
   cuuint64_t d[5], s[4];
@@ -86,10 +88,20 @@ bool make_tmap_bf16(CUtensorMap* m, const void* ptr, int rank, const uint64_t* d
     es[i] = 1;
   }
   for (int i = 0; i + 1 < rank; ++i) s[i] = strides_bytes[i];
-  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, rank, const_cast<void*>(ptr), d, s, bx, es,
+  CUresult r = fn(m, type, rank, const_cast<void*>(ptr), d, s, bx, es,
                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS;
+}
+
+bool make_tmap_bf16(CUtensorMap* m, const void* ptr, int rank, const uint64_t* dims,
+                    const uint64_t* strides_bytes, const uint32_t* box) {
+  return make_tmap_typed(CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, m, ptr, rank, dims, strides_bytes, box);
+}
+
+bool make_tmap_f16(CUtensorMap* m, const void* ptr, int rank, const uint64_t* dims,
+                   const uint64_t* strides_bytes, const uint32_t* box) {
+  return make_tmap_typed(CU_TENSOR_MAP_DATA_TYPE_FLOAT16, m, ptr, rank, dims, strides_bytes, box);
 }
 
 // ---------------------------------------------------------------------------
@@ -131,16 +143,20 @@ TcGemmPlan plan_tc_gemm(int M, int N, int K, int batch, bool allow_split) {
 // A: [batch][M][K] K-major (a_mn = false) or [batch][K][M] (a_mn = true);
 // X: [batch][N][K] with row stride xs_n and batch stride xs_b (elements).
 // out element (b, n, m) at ob*b + on*n + om*m.
+// kOutF32Split: the partial of split s goes to out + s * M * N (elements),
+// laid out by (ob, on, om) within the slice; *splits_out receives the split
+// count (the caller sums the slices).
 mla_status launch_tc_gemm(const void* A, bool a_mn, long long as_b, const void* X, long long xs_n,
                           long long xs_b, int M, int N, int K, int batch, void* out, long long ob,
                           long long on, long long om, int out_kind, cudaStream_t st,
-                          const PreAttnAux* aux = nullptr) {
+                          const PreAttnAux* aux = nullptr, int* splits_out = nullptr) {
   if (M <= 0 || N <= 0 || batch <= 0) return MLA_OK;
   if (!aligned16(A) || !aligned16(X) || (K % 8) != 0 || (xs_n % 8) != 0 || (xs_b % 8) != 0 ||
       (as_b % 8) != 0)
     return MLA_ERR_INVALID_ARG;
   if (a_mn && (M % 8) != 0) return MLA_ERR_INVALID_ARG;
-  TcGemmPlan p = plan_tc_gemm(M, N, K, batch, out_kind == kOutF32Atomic);
+  TcGemmPlan p = plan_tc_gemm(M, N, K, batch, out_kind == kOutF32Split);
+  if (splits_out) *splits_out = p.splits;
   CUtensorMap tA, tX;
   {
     uint64_t dims[3], strides[2];
@@ -170,6 +186,7 @@ mla_status launch_tc_gemm(const void* A, bool a_mn, long long as_b, const void* 
   g.k_chunks_per_split = p.k_chunks_per_split;
   g.stages = p.stages;
   g.out = out; g.ob = ob; g.on = on; g.om = om;
+  g.os = (long long)M * N;
   g.batch = batch;
   g.aux = PreAttnAux{};
   int aux_z = 0;
@@ -192,11 +209,11 @@ mla_status launch_tc_gemm(const void* A, bool a_mn, long long as_b, const void* 
   if (a_mn) {
     if (out_kind == kOutBf16) MLA_GEMM_LAUNCH(true, kOutBf16);
     else if (out_kind == kOutF32) MLA_GEMM_LAUNCH(true, kOutF32);
-    else MLA_GEMM_LAUNCH(true, kOutF32Atomic);
+    else MLA_GEMM_LAUNCH(true, kOutF32Split);
   } else {
     if (out_kind == kOutBf16) MLA_GEMM_LAUNCH(false, kOutBf16);
     else if (out_kind == kOutF32) MLA_GEMM_LAUNCH(false, kOutF32);
-    else MLA_GEMM_LAUNCH(false, kOutF32Atomic);
+    else MLA_GEMM_LAUNCH(false, kOutF32Split);
   }
 #undef MLA_GEMM_LAUNCH
   return check_launch();
@@ -369,6 +386,40 @@ mla_status mla_cache_append(const mla_dims* dims, const void* c, int cs_tok, con
   return check_launch();
 }
 
+static bool fp8_dims_ok(const mla_dims* d) {
+  return d->dtype == MLA_BF16 && d->d_latent == fp8::kDC && d->d_rope == fp8::kDR;
+}
+
+mla_status mla_cache_append_fp8(const mla_dims* dims, const void* c, int cs_tok, const void* kr,
+                                int ks_tok, const int32_t* batch_idx, const int32_t* pos,
+                                const int32_t* page_table, int max_pages, void* pool8,
+                                int n_pages, int T, void* stream) {
+  if (!dims_ok(dims) || T < 0 || max_pages < 1 || n_pages < 1) return MLA_ERR_INVALID_ARG;
+  if (!fp8_dims_ok(dims)) return MLA_ERR_UNSUPPORTED;
+  if (T == 0) return MLA_OK;
+  if (!c || !kr || !batch_idx || !pos || !page_table || !pool8) return MLA_ERR_INVALID_ARG;
+  if (!aligned16(c) || !aligned16(kr) || !aligned16(pool8) || (cs_tok % 8) != 0 ||
+      (ks_tok % 8) != 0)
+    return MLA_ERR_INVALID_ARG;
+  append_fp8_kernel<<<(T + 7) / 8, 256, 0, as_stream(stream)>>>(
+      static_cast<const uint16_t*>(c), cs_tok, static_cast<const uint16_t*>(kr), ks_tok,
+      batch_idx, pos, page_table, max_pages, static_cast<uint8_t*>(pool8), n_pages,
+      dims->page_size, T);
+  return check_launch();
+}
+
+mla_status mla_cache_quantize_fp8(const mla_dims* dims, const void* pool, void* pool8,
+                                  int n_pages, void* stream) {
+  if (!dims_ok(dims) || n_pages < 0) return MLA_ERR_INVALID_ARG;
+  if (!fp8_dims_ok(dims)) return MLA_ERR_UNSUPPORTED;
+  if (n_pages == 0) return MLA_OK;
+  if (!pool || !pool8 || !aligned16(pool) || !aligned16(pool8)) return MLA_ERR_INVALID_ARG;
+  const long long rows = (long long)n_pages * dims->page_size;
+  quantize_pool_fp8_kernel<<<(unsigned)((rows + 7) / 8), 256, 0, as_stream(stream)>>>(
+      static_cast<const uint16_t*>(pool), static_cast<uint8_t*>(pool8), rows);
+  return check_launch();
+}
+
 mla_status mla_pre_attention(const mla_dims* dims, void* y, int y_stride_tok, const void* w_uk,
                              void* qbuf, const int32_t* batch_idx, const int32_t* pos,
                              const int32_t* page_table, int max_pages, void* pool, int n_pages,
@@ -503,6 +554,59 @@ mla_status mla_decode(const mla_dims* dims, const void* qbuf, const void* pool, 
                      num_workers, workspace, ws_bytes, o_lat, lse, stream);
 }
 
+// Workspace of mla_decode_fp8: mla_decode's layout (same split planning),
+// then the half copy of the query, [B][S_q][H][576].
+static size_t fp8_q16_offset(const mla_dims* dims, int B, int S_q, int num_workers) {
+  return decode_layout(dims, B, S_q, num_workers).total;
+}
+
+size_t mla_decode_fp8_workspace_size(const mla_dims* dims, int B, int S_q, int num_workers) {
+  if (!dims_ok(dims) || B < 0 || S_q < 1 || num_workers < 0 || !fp8_dims_ok(dims)) return 0;
+  return fp8_q16_offset(dims, B, S_q, num_workers) +
+         (((size_t)B * S_q * dims->n_heads * 576 * 2 + 255) & ~(size_t)255);
+}
+
+mla_status mla_decode_fp8(const mla_dims* dims, const void* qbuf, const void* pool8,
+                          int n_pages, const int32_t* page_table, int max_pages,
+                          const int32_t* seq_lens, int B, int S_q, int num_workers,
+                          void* workspace, size_t ws_bytes, float* o_lat, float* lse,
+                          void* stream) {
+  if (!dims_ok(dims) || B < 0 || S_q < 1 || S_q > 2 || num_workers < 0 || n_pages < 1 ||
+      max_pages < 1)
+    return MLA_ERR_INVALID_ARG;
+  if (!fp8_dims_ok(dims) || dims->page_size != 64) return MLA_ERR_UNSUPPORTED;
+  if (B == 0) return MLA_OK;
+  if (!qbuf || !pool8 || !page_table || !seq_lens || !workspace || !o_lat || !lse)
+    return MLA_ERR_INVALID_ARG;
+  if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0 || !aligned16(qbuf) ||
+      !aligned16(pool8))
+    return MLA_ERR_INVALID_ARG;
+  if (ws_bytes < mla_decode_fp8_workspace_size(dims, B, S_q, num_workers))
+    return MLA_ERR_INVALID_ARG;
+  const DecodeLayout L = decode_layout(dims, B, S_q, num_workers);
+  cudaStream_t st = as_stream(stream);
+  char* ws = static_cast<char*>(workspace);
+  int32_t* start = reinterpret_cast<int32_t*>(ws + L.off_start);
+  float* ws_lse = reinterpret_cast<float*>(ws + L.off_lse);
+  float* ws_o = reinterpret_cast<float*>(ws + L.off_o);
+  uint16_t* q16 = reinterpret_cast<uint16_t*>(ws + fp8_q16_offset(dims, B, S_q, num_workers));
+  const long long nq = (long long)B * S_q * dims->n_heads * 576;
+  bf16_to_f16_kernel<<<(unsigned)((nq / 8 + 255) / 256 + 1), 256, 0, st>>>(
+      static_cast<const uint16_t*>(qbuf), q16, nq);
+  MLA_TRY(check_launch());
+  plan_kernel<<<1, 1024, 0, st>>>(seq_lens, nullptr, B, L.R, S_q, max_pages * dims->page_size,
+                                  dfp::kBlk, start);
+  MLA_TRY(check_launch());
+  MLA_TRY(launch_decode_fp8_impl(make_tmap_f16, q16, pool8, n_pages, page_table, max_pages,
+                                 seq_lens, nullptr, B, S_q, dims->n_heads, dims->scale, L.G,
+                                 start, ws_lse, ws_o, st));
+  g_launches.fetch_add(1, std::memory_order_relaxed);
+  dim3 cgrid(L.V, (L.rows_per_v + 7) / 8);
+  combine_kernel<<<cgrid, 256, 0, st>>>(ws_lse, ws_o, start, L.V, L.R, L.G, L.rows_per_v,
+                                        S_q * dims->n_heads, dims->d_latent, o_lat, lse);
+  return check_launch();
+}
+
 mla_status mla_decode_partial(const mla_dims* dims, const void* qbuf, const void* pool,
                               int n_pages, const int32_t* page_table, int max_pages,
                               const int32_t* seq_lens, const int32_t* seq_tail, int B, int S_q,
@@ -524,12 +628,19 @@ mla_status mla_combine_parts(const mla_dims* dims, const float* o_parts, const f
   return check_launch();
 }
 
+// Split count of the W_O GEMM for T tokens (its fp32 partials live in the
+// scratch).
+static int w_o_splits(const mla_dims* d, int T) {
+  return plan_tc_gemm(d->d_model, T, d->n_heads * d->d_v, 1, true).splits;
+}
+
 size_t mla_out_proj_scratch_size(const mla_dims* dims, int T) {
   if (!dims_ok(dims) || T < 0) return 0;
   auto up = [](size_t x) { return (x + 255) & ~(size_t)255; };
   const size_t H = dims->n_heads;
   if (dims->dtype == MLA_F32) return up((size_t)T * H * dims->d_v * 4);
-  return up((size_t)T * H * dims->d_latent * 2) + up((size_t)T * H * dims->d_v * 2);
+  return up((size_t)T * H * dims->d_latent * 2) + up((size_t)T * H * dims->d_v * 2) +
+         up((size_t)w_o_splits(dims, T) * T * dims->d_model * 4);
 }
 
 mla_status mla_out_proj(const mla_dims* dims, const float* o_lat, const void* w_uv,
@@ -563,11 +674,16 @@ mla_status mla_out_proj(const mla_dims* dims, const float* o_lat, const void* w_
   // o[t, i, :] = W_UV[i] o_lat[t, i, :]
   MLA_TRY(launch_tc_gemm(w_uv, false, (long long)dv * dc, olb, (long long)H * dc, dc, dv, T, dc, H,
                          o, dv, (long long)H * dv, 1, kOutBf16, st));
-  // out[t, :] = W_O o[t, :]
-  if (cudaMemsetAsync(out, 0, sizeof(float) * (size_t)T * dm, st) != cudaSuccess)
-    return MLA_ERR_CUDA;
-  return launch_tc_gemm(w_o, false, 0, o, (long long)H * dv, 0, dm, T, H * dv, 1, out, 0, dm, 1,
-                        kOutF32Atomic, st);
+  // out[t, :] = W_O o[t, :]: split-K partials into the scratch, then their
+  // ordered sum (deterministic: no atomics)
+  float* parts = reinterpret_cast<float*>(reinterpret_cast<char*>(o) + up((size_t)T * H * dv * 2));
+  int splits = 1;
+  MLA_TRY(launch_tc_gemm(w_o, false, 0, o, (long long)H * dv, 0, dm, T, H * dv, 1, parts, 0, dm, 1,
+                         kOutF32Split, st, nullptr, &splits));
+  const long long n_out = (long long)T * dm;
+  sum_splits_kernel<<<(unsigned)((n_out / 4 + 255) / 256 + 1), 256, 0, st>>>(parts, splits, n_out,
+                                                                             out);
+  return check_launch();
 }
 
 }  // extern "C"

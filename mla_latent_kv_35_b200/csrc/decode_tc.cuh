@@ -31,11 +31,11 @@
 //     [slot group][chunk][8 slots][128 B], so the two pages' slot groups of a
 //     chunk sit at one uniform stride (2 KB) and form the 128-row K-major B
 //     operand.  Only the leader arms each stage barrier, for both CTAs' bytes.
-//     The same lane prefetches the next block's pages into L2 (bulk
-//     prefetch, one request per page), so the boxes are served from L2.
+//     (An L2 bulk prefetch of the next block's pages was tried: 10% slower;
+//     the prefetches queue in the same copy engine as the boxes.)
 //   * PV loads.  Warps 2 and 3 fill a ring of three 16 KB stages (one page x
 //     128 latent columns) with 16-byte cp.async into the 128-byte-swizzled
-//     layout; they read the same pages the QK boxes just brought into L2.
+//     layout; they read the same pages the QK boxes bring into L2.
 //     In the peer CTA, warp 1 lane 0 relays each landed stage to the
 //     leader's barrier.
 //   * Softmax: eight warps per CTA.  Warps w and w + 4 share TMEM lane
@@ -98,8 +98,8 @@ constexpr int kSoftmaxThreads = 256;
 // registers per thread: at launch (65536 / 384, rounded down to 8), then
 // after the split of the control warpgroup and the softmax warpgroups
 constexpr int kRegsLaunch = 168;
-constexpr int kRegsControl = 72;
-constexpr int kRegsSoftmax = 216;
+constexpr int kRegsControl = 136;
+constexpr int kRegsSoftmax = 184;
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kTmemO = 0;       // O_n at columns [128n, 128n + 128)
 constexpr uint32_t kTmemS = 256;     // S_b at columns [256 + 128b, +128)
@@ -240,26 +240,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(dtc::kThreads, 1)
     // (the register budget applies to the code it dominates)
     setmaxnreg_dec<kRegsControl>();
     if (warp == 0 && lane == 0) {
-      // ==========  QK producer: Q slices, QK boxes, L2 prefetch  ==========
+      // ==========  QK producer: Q slices and QK boxes  ==========
       const uint32_t lead_full0 = mapa_shared(smem_u32(&qk_full[0]), 0);
       const uint32_t lead_qfull = mapa_shared(smem_u32(&q_full), 0);
       uint32_t it = 0, q_issued = 0;
       PieceIter pi;
       pi.init(P.start, V, lo, hi);
-      // cursor of the next block to prefetch into L2 (global block index)
-      int pf_g = lo, pf_v = lo < hi ? seq_of_block(P.start, V, lo) : V;
-      auto prefetch_upto = [&](int g_end) {
-        for (; pf_g < min(g_end, hi); ++pf_g) {
-          while (P.start[pf_v + 1] <= pf_g) ++pf_v;
-          const int b = pf_v / P.R;
-          const int L = P.seq_lens[b];
-          const int x = pf_g - P.start[pf_v];
-          for (int i = 0; i < 2; ++i) {
-            const int pg = page_of(P, b, L, x, 2 * (int)rank + i);
-            if (pg >= 0) prefetch_l2_bulk(P.pool + (size_t)pg * kPageBytes, kPageBytes);
-          }
-        }
-      };
       int v, x0, x1, piece = 0;
       bool ok = true;
       while (ok && pi.next(v, x0, x1)) {
@@ -276,8 +262,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(dtc::kThreads, 1)
           tma_load_2d_pair(sQ + c * kChunk, &tmQ, c * 64, row0, lead_qfull);
         ++q_issued;
         for (int x = x0; x < x1 && ok; ++x) {
-          // this block and the next one go to L2 ahead of the boxes
-          prefetch_upto(P.start[v] + x + 2);
           int pg[2];
           for (int i = 0; i < 2; ++i) {
             pg[i] = page_of(P, b, L, x, 2 * (int)rank + i);
@@ -386,6 +370,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(dtc::kThreads, 1)
       // of a piece, once the previous piece's epilogue has released O.
       const uint32_t idesc_qk = idesc_bf16_f32(128, 256, false, false);
       const uint32_t idesc_pv = idesc_bf16_f32(128, 256, false, true);
+      // Operand descriptors are formed once; an MMA only adds its tile's
+      // offset (in 16-byte units) to the start-address field, which keeps
+      // the issuing thread's work per MMA to a few integer adds.
+      const uint64_t q_desc = sw128_desc(sQ, 16, 1024);
+      const uint64_t p_desc = sw128_desc(sP, 16, 1024);
+      const uint64_t qk_desc = sw128_desc(sQk, 16, 2048);  // 16 slot groups 2 KB apart
+      const uint64_t pv_desc = sw128_desc(sPv, kChunk, 1024);
       PieceIter qi, vi;
       qi.init(P.start, V, lo, hi);
       vi.init(P.start, V, lo, hi);
@@ -405,24 +396,23 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(dtc::kThreads, 1)
         if (q_more && jq <= jp + (p_in ? 1 : 0) + 1) {
           bool ready = true;
           if (!q_in) {
-            ready = mbar_try_wait(smem_u32(&q_full), q_piece & 1);
+            ready = mbar_test_wait(smem_u32(&q_full), q_piece & 1);
             if (ready) q_in = true;
           }
           const int s = itq % kQkStages;
-          if (ready && mbar_try_wait(smem_u32(&qk_full[s]), (itq / kQkStages) & 1)) {
+          if (ready && mbar_test_wait(smem_u32(&qk_full[s]), (itq / kQkStages) & 1)) {
             tc_fence_after();
             const uint32_t sd = tmem + kTmemS + 128 * (jq & 1);
-            const uint32_t st = sQk + s * kQkStageBytes;
             const int ncc = (kq == kQkStagesPerBlock - 1) ? 1 : 2;
+            const uint64_t a0 = q_desc + (uint64_t)((2 * kq * kChunk) >> 4);
+            const uint64_t b0 = qk_desc + (uint64_t)s * (kQkStageBytes >> 4);
             for (int cc = 0; cc < ncc; ++cc) {
               const int c = 2 * kq + cc;  // 64-column chunk of the 576
 #pragma unroll
-              for (int kk = 0; kk < 4; ++kk) {
-                const uint64_t ad = sw128_desc(sQ + c * kChunk + kk * 32, 16, 1024);
-                // 16 slot groups (8 per page) 2 KB apart
-                const uint64_t bd = sw128_desc(st + cc * 1024 + kk * 32, 16, 2048);
-                mma_bf16_ss<2>(sd, ad, bd, idesc_qk, (c | kk) ? 1u : 0u);
-              }
+              for (int kk = 0; kk < 4; ++kk)
+                mma_bf16_ss<2>(sd, a0 + (uint64_t)((cc * kChunk + kk * 32) >> 4),
+                               b0 + (uint64_t)((cc * 1024 + kk * 32) >> 4), idesc_qk,
+                               (c | kk) ? 1u : 0u);
             }
             mma_commit_2_mc(smem_u32(&qk_empty[s]), 3);
             ++itq;
@@ -444,13 +434,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(dtc::kThreads, 1)
         // ---------------- one PV stage ----------------
         if (v_more && jp < jq) {
           if (!p_in) {
-            p_in = mbar_try_wait(smem_u32(&p_full), jp & 1) &&
+            p_in = mbar_test_wait(smem_u32(&p_full), jp & 1) &&
                    (vx != vx0 || v_piece == 0 ||
-                    mbar_try_wait(smem_u32(&o_empty), (v_piece - 1) & 1));
+                    mbar_test_wait(smem_u32(&o_empty), (v_piece - 1) & 1));
             if (p_in) tc_fence_after();
           }
           const int s = itv % kPvStages;
-          if (p_in && mbar_try_wait(smem_u32(&pv_full[s]), (itv / kPvStages) & 1)) {
+          if (p_in && mbar_test_wait(smem_u32(&pv_full[s]), (itv / kPvStages) & 1)) {
             // The stage was written by cp.async and st.shared (generic
             // proxy); the MMA reads it through the async proxy.  The writes
             // are ordered before this thread by the barrier; the proxy fence
@@ -460,13 +450,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(dtc::kThreads, 1)
             tc_fence_after();
             const int p = tp >> 1, n = tp & 1;
             const bool first = (vx == vx0);
-            const uint32_t st = sPv + s * kPvStageBytes;
+            const uint64_t a0 = p_desc + (uint64_t)((p * kChunk) >> 4);
+            const uint64_t b0 = pv_desc + (uint64_t)s * (kPvStageBytes >> 4);
 #pragma unroll
             for (int kk = 0; kk < 4; ++kk) {
-              const uint64_t ad = sw128_desc(sP + p * kChunk + kk * 32, 16, 1024);
-              const uint64_t bd = sw128_desc(st + kk * 2048, kChunk, 1024);
               const uint32_t acc = (first && p == 0 && kk == 0) ? 0u : 1u;
-              mma_bf16_ss<2>(tmem + kTmemO + 128 * n, ad, bd, idesc_pv, acc);
+              mma_bf16_ss<2>(tmem + kTmemO + 128 * n, a0 + (uint64_t)((kk * 32) >> 4),
+                             b0 + (uint64_t)((kk * 2048) >> 4), idesc_pv, acc);
             }
             mma_commit_2_mc(smem_u32(&pv_empty[s]), 3);
             ++itv;
@@ -535,20 +525,26 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(dtc::kThreads, 1)
       bool o_started = false;
       for (int x = x0; x < x1; ++x, ++j) {
         const bool got = mbar_wait(smem_u32(&s_full[j & 1]), (j >> 1) & 1, abort_p, 7, j);
-        uint32_t s_raw[64];
         float mx = -INFINITY;
         const int cmax = limit - (x * kBlk + pb * kPage);  // columns c < cmax are visible
-        if (__all_sync(0xffffffffu, got)) {
+        // this thread's 64 scores, read from TMEM 32 at a time (twice: for
+        // the max, then for the exponentials), which keeps half the
+        // registers of holding all 64 across the max exchange; invisible
+        // columns (past the context, causally hidden, or slots of a partial
+        // page whose contents are not cache) count as -inf
+        const uint32_t sa = tmem + lane_addr + kTmemS + 128 * (j & 1) + 64 * ch;
+        const bool all_got = __all_sync(0xffffffffu, got);
+        if (all_got) {
           tc_fence_after();
-          uint32_t (&a)[32] = *reinterpret_cast<uint32_t(*)[32]>(&s_raw[0]);
-          uint32_t (&c2)[32] = *reinterpret_cast<uint32_t(*)[32]>(&s_raw[32]);
-          const uint32_t sa = tmem + lane_addr + kTmemS + 128 * (j & 1) + 64 * ch;
-          tmem_ld32(sa, a);
-          tmem_ld32(sa + 32, c2);
-          tmem_wait_ld();
 #pragma unroll
-          for (int c = 0; c < 64; ++c)
-            if (c < cmax) mx = fmaxf(mx, __uint_as_float(s_raw[c]));
+          for (int hf = 0; hf < 2; ++hf) {
+            uint32_t r[32];
+            tmem_ld32(sa + 32 * hf, r);
+            tmem_wait_ld();
+#pragma unroll
+            for (int c = 0; c < 32; ++c)
+              if (32 * hf + c < cmax) mx = fmaxf(mx, __uint_as_float(r[c]));
+          }
         }
         red_max[j & 1][pb][h] = mx;
         // one barrier: the other pages' maxima visible, and everyone agrees
@@ -567,17 +563,23 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(dtc::kThreads, 1)
         uint32_t pk[32];
         float lsum = 0.f;
 #pragma unroll
-        for (int e = 0; e < 32; ++e) {
-          const int c0 = 2 * e;
-          const float p0 = c0 < cmax
-                               ? ex2_approx(fmaf(__uint_as_float(s_raw[c0]), P.scale_log2, -m_use))
-                               : 0.f;
-          const float p1 = c0 + 1 < cmax
-                               ? ex2_approx(fmaf(__uint_as_float(s_raw[c0 + 1]), P.scale_log2,
-                                                 -m_use))
-                               : 0.f;
-          lsum += p0 + p1;
-          pk[e] = pack_bf16x2(p0, p1);
+        for (int hf = 0; hf < 2; ++hf) {
+          uint32_t r[32];
+          tmem_ld32(sa + 32 * hf, r);
+          tmem_wait_ld();
+#pragma unroll
+          for (int e = 0; e < 16; ++e) {
+            const int c0 = 32 * hf + 2 * e;
+            const float p0 =
+                c0 < cmax ? ex2_approx(fmaf(__uint_as_float(r[2 * e]), P.scale_log2, -m_use))
+                          : 0.f;
+            const float p1 =
+                c0 + 1 < cmax
+                    ? ex2_approx(fmaf(__uint_as_float(r[2 * e + 1]), P.scale_log2, -m_use))
+                    : 0.f;
+            lsum += p0 + p1;
+            pk[16 * hf + e] = pack_bf16x2(p0, p1);
+          }
         }
         // PV(j-1) must be done before P is overwritten and before O is rescaled
         bool ok = true;

@@ -9,7 +9,9 @@
 // below 128, so putting the weights on M keeps the MMA at full height.
 // A may be K-major ([M][K], the usual [out, in] weight) or MN-major ([K][M],
 // e.g. W_UK[i] read as its transpose).  X is always K-major.  Split-K over
-// grid.y accumulates fp32 outputs with atomics.
+// grid.y writes each split's fp32 partial to its own slice of the output
+// (split s at out + s * os); an ordered sum of the slices follows, so the
+// result does not depend on the order the splits finish in.
 //
 // Warp roles (128 threads): warp 0 lane 0 issues TMA loads into an
 // S-stage ring; warp 1 allocates TMEM and its lane 0 issues the MMAs; after
@@ -22,7 +24,7 @@
 
 namespace mla {
 
-enum GemmOut : int { kOutBf16 = 0, kOutF32 = 1, kOutF32Atomic = 2 };
+enum GemmOut : int { kOutBf16 = 0, kOutF32 = 1, kOutF32Split = 2 };
 
 struct GemmTcArgs {
   int M, N, K;           // per batch entry
@@ -32,6 +34,7 @@ struct GemmTcArgs {
   int stages;
   void* out;
   long long ob, on, om;  // output strides in elements
+  long long os;          // kOutF32Split: elements between the splits' slices
   int batch;             // GEMM batch entries
   int aux_z;             // grid.z slices [0, aux_z) run `aux`; GEMM entry b is slice aux_z + b
   PreAttnAux aux;
@@ -174,12 +177,12 @@ __global__ void __launch_bounds__(128, 1) gemm_tc_kernel(const __grid_constant__
             else if constexpr (kOut == kOutF32)
               static_cast<float*>(g.out)[o] = v;
             else
-              atomicAdd(static_cast<float*>(g.out) + o, v);
+              static_cast<float*>(g.out)[o + split * g.os] = v;
           }
         }
       }
     }
-  } else if (nk == 0 && kOut != kOutF32Atomic) {
+  } else if (nk == 0) {
     // empty K range: the product is zero
     const int m = m0 + warp * 32 + lane;
     if (m < g.M)
@@ -189,14 +192,35 @@ __global__ void __launch_bounds__(128, 1) gemm_tc_kernel(const __grid_constant__
           const long long o = (long long)b * g.ob + (long long)n * g.on + (long long)m * g.om;
           if constexpr (kOut == kOutBf16)
             static_cast<__nv_bfloat16*>(g.out)[o] = __float2bfloat16_rn(0.f);
-          else
+          else if constexpr (kOut == kOutF32)
             static_cast<float*>(g.out)[o] = 0.f;
+          else
+            static_cast<float*>(g.out)[o + split * g.os] = 0.f;
         }
       }
   }
   tc_fence_before();
   __syncthreads();
   if (warp == 1) tmem_dealloc<1>(tmem, tmem_cols);
+}
+
+// out[i] = sum over s = 0 .. splits-1 of parts[s * n + i], in that order.
+__global__ void sum_splits_kernel(const float* parts, int splits, long long n, float* out) {
+  const long long i = ((long long)blockIdx.x * blockDim.x + threadIdx.x) * 4;
+  if (i + 3 < n) {
+    float4 acc = *reinterpret_cast<const float4*>(parts + i);
+    for (int s = 1; s < splits; ++s) {
+      const float4 v = *reinterpret_cast<const float4*>(parts + s * n + i);
+      acc.x += v.x; acc.y += v.y; acc.z += v.z; acc.w += v.w;
+    }
+    *reinterpret_cast<float4*>(out + i) = acc;
+  } else {
+    for (long long k = i; k < n; ++k) {
+      float acc = parts[k];
+      for (int s = 1; s < splits; ++s) acc += parts[s * n + k];
+      out[k] = acc;
+    }
+  }
 }
 
 }  // namespace mla

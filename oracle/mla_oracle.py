@@ -393,10 +393,10 @@ def combine_splits(o_parts, lse_parts):
 # reading used here (R16): each token's 512-number latent is stored in the
 # 8-bit float format E4M3 (1 sign, 4 exponent bits with bias 7, 3 mantissa
 # bits, largest finite value 448, no infinities) after division by one
-# per-token scale s = max|c| / 448; the 64-number RoPE key is kept in a
-# 16-bit float.  The scale and the division are single-precision steps (the
-# precision the GPU quantizer takes the decision in), so both sides produce
-# the same codes.
+# per-token scale s (max|c| / 448, or more when the RoPE key needs it); the
+# 64-number RoPE key, divided by the same s, is kept in half precision.  The
+# scale and the divisions are single-precision steps (the precision the GPU
+# quantizer takes the decision in), so both sides produce the same codes.
 # ---------------------------------------------------------------------------
 
 E4M3_MAX = 448.0
@@ -436,25 +436,32 @@ def f16_round(x):
     return round_to_grid(x, 10, -14, 65504.0)
 
 
+F16_MAX = 65504.0
+
+
 def quantize_latent_fp8(C, KR):
     """8-bit cache rows of tokens C [L, d_c], KR [L, d_r] (reading R16).
 
-    Per token t, in single precision: s_t = max_k |C[t, k]| / 448 (1 for an
-    all-zero latent) and x = C[t] / s_t, then c8_t = E4M3(x); the RoPE key is
-    stored as half precision, kr8_t = f16(KR[t]).  Returns (s [L],
-    c8 [L, d_c] E4M3 values, kr8 [L, d_r]); the cache the attention sees is
-    [s_t c8_t ; kr8_t] (dequantize_fp8).
+    Per token t, in single precision: one scale for the whole row,
+    s_t = max(max_k |C[t, k]| / 448, max_r |KR[t, r]| / 65504) (1 for an
+    all-zero row), so that both parts divided by it fit their formats; then
+    c8_t = E4M3(C[t] / s_t) and the RoPE key is stored as the half-precision
+    number kr8_t = f16(KR[t] / s_t).  Returns (s [L], c8 [L, d_c] E4M3
+    values, kr8 [L, d_r] half values); the cache the attention sees is
+    s_t [c8_t ; kr8_t] (dequantize_fp8).
     """
     C32 = np.asarray(C, dtype=np.float32)
-    m = np.abs(C32).max(axis=1) if C32.shape[1] else np.zeros(C32.shape[0], np.float32)
-    s = np.where(m > 0, m / np.float32(E4M3_MAX), np.float32(1.0)).astype(np.float32)
-    x = (C32 / s[:, None]).astype(np.float32)
-    c8 = e4m3_round(x.astype(F64))
-    kr8 = f16_round(np.asarray(KR, dtype=F64))
+    K32 = np.asarray(KR, dtype=np.float32)
+    mc = np.abs(C32).max(axis=1) if C32.shape[1] else np.zeros(C32.shape[0], np.float32)
+    mk = np.abs(K32).max(axis=1) if K32.shape[1] else np.zeros(K32.shape[0], np.float32)
+    s = np.maximum(mc / np.float32(E4M3_MAX), mk / np.float32(F16_MAX)).astype(np.float32)
+    s = np.where(s > 0, s, np.float32(1.0)).astype(np.float32)
+    c8 = e4m3_round((C32 / s[:, None]).astype(np.float32).astype(F64))
+    kr8 = f16_round((K32 / s[:, None]).astype(np.float32).astype(F64))
     return s.astype(F64), c8, kr8
 
 
 def dequantize_fp8(s, c8, kr8):
-    """The cache numbers an 8-bit row stands for: (s c8, kr8)."""
+    """The cache numbers an 8-bit row stands for: (s c8, s kr8)."""
     s = np.asarray(s, dtype=F64)[:, None]
-    return s * np.asarray(c8, dtype=F64), np.asarray(kr8, dtype=F64)
+    return s * np.asarray(c8, dtype=F64), s * np.asarray(kr8, dtype=F64)

@@ -62,26 +62,42 @@ def check(got, ref, dtype, what="", tol=None):
     return mx, mean, rel
 
 
-def check_stored_bf16(got, ref, what="", rotated=False):
-    """A value the GPU stores in bf16 against the oracle's fp64 value.
+def check_stored_bf16(got, ref, what="", rotated=False, acc=None):
+    """A value the GPU computes in fp32 and stores in bf16, against the
+    oracle's fp64 value.
 
     A bf16 store rounds to nearest: |error| <= u |ref| with the unit roundoff
-    u = 2^-8 of 8 significant bits.  A RoPE-rotated key (rotated=True) is
-    rounded twice: its pre-RoPE input is a bf16 projection output, and
-    rotating a pair mixes the two rounded inputs, so element e of pair (x, y)
-    may be off by u (|x_in| + |y_in|) <= u sqrt(2) |pair| before the final
-    rounding of u |ref_e|.  A little fp32 slack is added to both bounds."""
+    u = 2^-8 of 8 significant bits.  `acc` (same shape) bounds the fp32
+    accumulation that produced the value before the store, elementwise.  A
+    RoPE-rotated key (rotated=True) is rounded twice: its pre-RoPE input is
+    a bf16 projection output, and rotating a pair mixes the two rounded
+    inputs, so element e of pair (x, y) may be off by u (|x_in| + |y_in|)
+    <= u sqrt(2) |pair| (plus both inputs' accumulation bounds) before the
+    final rounding of u |ref_e|."""
     got = np.asarray(got, np.float64)
     ref = np.asarray(ref, np.float64)
+    acc = np.zeros_like(ref) if acc is None else np.asarray(acc, np.float64)
     u = 2.0 ** -8
     bound = u * np.abs(ref)
     if rotated:
         pair = np.sqrt(ref[0::2] ** 2 + ref[1::2] ** 2)
+        acc = np.repeat(np.maximum(acc[0::2], acc[1::2]) * 2, 2)
         bound = bound + u * np.sqrt(2.0) * np.repeat(pair, 2)
-    bound = bound * (1 + 1e-3) + 1e-6
+    bound = (bound + acc) * (1 + 1e-3) + 1e-7
     err = np.abs(got - ref)
     assert (err <= bound).all(), \
         f"{what}: worst error {err.max():.3e} (bound there {bound[np.argmax(err - bound)]:.3e})"
+
+
+def fp32_accumulation_bound(x, w):
+    """Bound on the fp32 accumulation error of y = x . w[o] on the tensor
+    cores: each of the K/16 MMA steps adds one exactly formed partial product
+    sum to an fp32 accumulator, so the error is at most (K/16) 2^-24
+    sum_i |x_i w[o, i]|."""
+    x = np.abs(np.asarray(x, np.float64))
+    w = np.abs(np.asarray(w, np.float64))
+    K = x.shape[-1]
+    return (-(-K // 16)) * 2.0 ** -24 * (x @ w.T)
 
 
 def status():

@@ -20,7 +20,8 @@ from mla_latent_kv_35_b200.binding import MLADims
 from mla_latent_kv_35_b200.engine import MLADecodeLayer, build_pool_host, pool_to_device
 import oracle_pool
 from mla_latent_kv_35_b200 import binding as B
-from gpu_util import DEV, check, check_stored_bf16, ensure_lib, status, to_np
+from gpu_util import (DEV, check, check_stored_bf16, ensure_lib, fp32_accumulation_bound,
+                      status, to_np)
 
 gpu = pytest.mark.gpu
 
@@ -108,10 +109,13 @@ def _check_bf16_workload(name, sample, nonabs_sample, nonabs_heads=(0, 77, 127))
         check(lse[b], r["lse"], "bf16", f"{name} b={b} lse")
         check(out[b], r["out"], "bf16", f"{name} b={b} out")
         # the appended rows hold the new tokens' latent and rotated RoPE key
+        acc_c = fp32_accumulation_bound(h[b], W["W_DKV"])
+        acc_k = fp32_accumulation_bound(h[b], W["W_KR"])
         for j, row in enumerate(new_rows[b]):
             rowf = wl.bf16_to_f32(row).astype(np.float64)
-            check_stored_bf16(rowf[:w.d_latent], r["c_new"][j], "A3 c_new")
-            check_stored_bf16(rowf[w.d_latent:], r["kr_new"][j], "A3 kr_new", rotated=True)
+            check_stored_bf16(rowf[:w.d_latent], r["c_new"][j], "A3 c_new", acc=acc_c[j])
+            check_stored_bf16(rowf[w.d_latent:], r["kr_new"][j], "A3 kr_new", rotated=True,
+                              acc=acc_k[j])
     for b in nonabs_sample:
         c, kr = wl.draw_prior(w, b)
         na = oracle.decode_step(h[b:b + 1], [c], [kr], W["W_Q"], W["W_DKV"], W["W_KR"],

@@ -85,19 +85,24 @@ def test_quantize_latent_fp8_error_bound_and_worked_values():
     half = np.where(xs >= 2.0 ** -6, np.exp2(np.floor(np.log2(np.maximum(xs, 1e-300))) - 4),
                     2.0 ** -10)
     assert (np.abs(Cd - C) <= (half + xs * 2.0 ** -23) * s[:, None] * (1 + 1e-9)).all()
-    assert (np.abs(KRd - KR) <= 2.0 ** -11 * np.abs(KR) * (1 + 1e-12) + 2.0 ** -25).all()
+    # the RoPE key: half precision of KR / s (11 significant bits) times s
+    assert (np.abs(KRd - KR) <= (2.0 ** -11 + 2.0 ** -23) * np.abs(KR) * (1 + 1e-9)).all()
     # hand-worked token: max |c| = 896, so s = 2; 3 / 2 = 1.5 (exact), 1.1 / 2
     # = 0.55 -> 0.5625 (grid step 1/16 in [0.5, 1)), -896 / 2 = -448; RoPE
-    # key parts in [2, 4) sit on a grid of 2^-9: 3 + 2^-9 is kept and
-    # 3 + 2^-10, a tie, goes to the even neighbour 3
+    # parts / 2 in [1, 2) sit on a grid of 2^-10: 3 + 2^-9 -> 1.5 + 2^-10 is
+    # kept, 3 + 2^-10 -> 1.5 + 2^-11, a tie, goes to the even neighbour 1.5
     s1, c1, k1 = om.quantize_latent_fp8(np.array([[3.0, 1.1, -896.0]]),
                                         np.array([[3.001953125, 3.0009765625]]))
     assert s1[0] == 2.0
     np.testing.assert_array_equal(c1[0], [1.5, 0.5625, -448.0])
-    np.testing.assert_array_equal(k1[0], [3.001953125, 3.0])
-    # an all-zero latent keeps scale 1
-    s0, c0, _ = om.quantize_latent_fp8(np.zeros((1, 4)), np.ones((1, 2)))
-    assert s0[0] == 1.0 and (c0 == 0).all()
+    np.testing.assert_array_equal(k1[0], [1.5009765625, 1.5])
+    # a RoPE key too large for half precision at the latent's scale sets s
+    s2, c2, k2 = om.quantize_latent_fp8(np.array([[0.5, -0.25]]), np.array([[1.0e3, -2.0]]))
+    assert s2[0] == np.float32(np.float32(1.0e3) / np.float32(65504.0))
+    assert np.abs(k2).max() <= 65504.0
+    # an all-zero row keeps scale 1
+    s0, c0, k0 = om.quantize_latent_fp8(np.zeros((1, 4)), np.zeros((1, 2)))
+    assert s0[0] == 1.0 and (c0 == 0).all() and (k0 == 0).all()
 
 
 def test_planted_rounding_slips_are_caught(monkeypatch):
