@@ -91,19 +91,32 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
   return ok != 0;
 }
 
-// Non-blocking test of phase `parity` (try_wait may suspend the thread for a
-// while; a thread polling several barriers in turn uses this instead).
-__device__ __forceinline__ bool mbar_test_wait(uint32_t bar, uint32_t parity) {
+// try_wait by a whole warp with one answer for all lanes (a phase, once
+// complete, stays complete until the waiter releases the stage).
+__device__ __forceinline__ bool warp_try_wait(uint32_t bar, uint32_t parity) {
+  return __any_sync(0xffffffffu, mbar_try_wait(bar, parity));
+}
+
+// try_wait that may suspend the thread until the phase completes, for at
+// most about `ns` nanoseconds.
+__device__ __forceinline__ bool mbar_try_wait_suspend(uint32_t bar, uint32_t parity, uint32_t ns) {
   uint32_t ok;
   asm volatile(
       "{\n\t.reg .pred p;\n\t"
-      "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
       "selp.u32 %0, 1, 0, p;\n\t}"
       : "=r"(ok)
-      : "r"(bar), "r"(parity)
+      : "r"(bar), "r"(parity), "r"(ns)
       : "memory");
   return ok != 0;
 }
+
+// Suspend bound of one try_wait inside a waiting loop.  A waiting thread is
+// parked rather than spinning: spinning waiters share the issue slots and the
+// shared-memory pipe with the thread that issues the MMAs.
+#ifndef MLA_SUSPEND_NS
+#define MLA_SUSPEND_NS 1000u
+#endif
 
 // Wait for phase `parity` of the barrier to complete.  Gives up after
 // MLA_WAIT_NS (raising kFlagTimeout and setting *abort) or as soon as another
@@ -113,8 +126,8 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatil
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = globaltimer();
   for (uint32_t it = 1;; ++it) {
-    if (mbar_try_wait(bar, parity)) return true;
-    if ((it & 63u) == 0) {
+    if (mbar_try_wait_suspend(bar, parity, MLA_SUSPEND_NS)) return true;
+    if ((it & 3u) == 0) {
       if (abort != nullptr && *abort) return false;
       if (globaltimer() - t0 > MLA_WAIT_NS) {
         raise_flag(kFlagTimeout);
@@ -132,7 +145,7 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatil
 __device__ __forceinline__ bool mbar_wait_bounded(uint32_t bar, uint32_t parity, uint64_t ns) {
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = globaltimer();
-  while (!mbar_try_wait(bar, parity))
+  while (!mbar_try_wait_suspend(bar, parity, MLA_SUSPEND_NS))
     if (globaltimer() - t0 > ns) return false;
   return true;
 }

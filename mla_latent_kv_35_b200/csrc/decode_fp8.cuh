@@ -326,11 +326,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(dfp::kThreads, 1)
         if (q_more && jq <= jp + (p_in ? 1 : 0) + 1) {
           bool ready = true;
           if (!q_in) {
-            ready = mbar_test_wait(smem_u32(&q_full), q_piece & 1);
+            ready = mbar_try_wait(smem_u32(&q_full), q_piece & 1);
             if (ready) q_in = true;
           }
           const int s = itq % kQkStages;
-          if (ready && mbar_test_wait(smem_u32(&qk_full[s]), (itq / kQkStages) & 1)) {
+          if (ready && mbar_try_wait(smem_u32(&qk_full[s]), (itq / kQkStages) & 1)) {
             fence_proxy_async_smem();
             tc_fence_after();
             const uint32_t sd = tmem + kTmemS + 128 * (jq & 1);
@@ -364,13 +364,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(dfp::kThreads, 1)
         }
         if (v_more && jp < jq) {
           if (!p_in) {
-            p_in = mbar_test_wait(smem_u32(&p_full), jp & 1) &&
+            p_in = mbar_try_wait(smem_u32(&p_full), jp & 1) &&
                    (vx != vx0 || v_piece == 0 ||
-                    mbar_test_wait(smem_u32(&o_empty), (v_piece - 1) & 1));
+                    mbar_try_wait(smem_u32(&o_empty), (v_piece - 1) & 1));
             if (p_in) tc_fence_after();
           }
           const int s = itv % kPvStages;
-          if (p_in && mbar_test_wait(smem_u32(&pv_full[s]), (itv / kPvStages) & 1)) {
+          if (p_in && mbar_try_wait(smem_u32(&pv_full[s]), (itv / kPvStages) & 1)) {
             fence_proxy_async_smem();
             tc_fence_after();
             const int p = tp >> 1, n = tp & 1;

@@ -31,19 +31,29 @@
 //     [slot group][chunk][8 slots][128 B], so the two pages' slot groups of a
 //     chunk sit at one uniform stride (2 KB) and form the 128-row K-major B
 //     operand.  Only the leader arms each stage barrier, for both CTAs' bytes.
-//     (An L2 bulk prefetch of the next block's pages was tried: 10% slower;
-//     the prefetches queue in the same copy engine as the boxes.)
-//   * PV loads.  Warps 2 and 3 fill a ring of three 16 KB stages (one page x
-//     128 latent columns) with 16-byte cp.async into the 128-byte-swizzled
-//     layout; they read the same pages the QK boxes bring into L2.
-//     In the peer CTA, warp 1 lane 0 relays each landed stage to the
-//     leader's barrier.
+//     The page ids are read from the table two blocks ahead.  (L2 prefetch
+//     of later blocks' pages, by bulk prefetches or by line prefetches from
+//     the softmax warps, was measured slower; so were 16 KB stages.)
+//   * PV loads.  Lane 0 of warp 2 fills a ring of three 16 KB stages (one
+//     page x 128 latent columns) with one TMA box each from a 3-D view of
+//     the pool (64 columns, pool rows, 9 chunks), which lands in the
+//     MN-major operand layout; it reads the same pages the QK boxes brought
+//     into L2.  The partial last page of a sequence is copied by the whole
+//     warp with cp.async instead, with zeros for the slots past the end.
 //   * Softmax: eight warps per CTA.  Warps w and w + 4 share TMEM lane
 //     quadrant w and take 64 of its 128 columns each, so every thread holds
 //     the scores of one row on one page.  Row maxima of the four pages meet
 //     in shared memory.  The running max is rescaled lazily: O is rescaled
 //     in TMEM only when a row's max grows by more than 2^8, warp-uniformly.
-//     P goes to shared memory and the leader's MMA warp is signalled.
+//     After its last read of S the softmax releases the S buffer (s_free);
+//     P goes to shared memory once PV of the previous block is done, and
+//     the PV issuer is signalled.
+//   * MMA issue.  Two threads of the leader issue the MMAs: lane 0 of warp 1
+//     the QK stream, lane 0 of warp 3 the PV stream.  The tensor pipe
+//     buffers little beyond the MMA it runs, and every barrier wait, commit
+//     and loop step of an issuing thread costs tens to hundreds of cycles;
+//     with two issuers one stream's MMAs fill the other's gaps (a single
+//     thread interleaving both streams was measured 12% slower).
 //   * Pieces (sequence, block range) of a worker write normalised partial
 //     outputs and natural-log LSE into slot worker + v of the workspace; the
 //     combine kernel merges them.
@@ -52,16 +62,15 @@
 //
 // Partial and missing pages.  QK boxes always load a whole page; slots past
 // the sequence hold whatever the pool holds there and are masked by index in
-// the softmax (P = 0).  The PV loader writes zeros for those rows, so no
+// the softmax (P = 0).  The PV producer writes zeros for those rows, so no
 // unused slot ever reaches O.  Pages past the end load entirely out of
 // bounds (zeros) and their page-table entries are never read.
 //
 // Every mbarrier wait is bounded (MLA_WAIT_NS); on expiry the kernel raises
 // MLA_ERR_TIMEOUT in the device status and every role leaves its loop.  On
-// the way out the leader's producer waits (bounded) for the boxes it armed
-// and its MMA thread for a last commit, the loader warps for their own
-// cp.async; then the pair meets at a final cluster barrier and frees its
-// TMEM.
+// the way out the leader's producers wait (bounded) for the boxes they
+// armed and each MMA issuer for a last commit of its own; then the pair
+// meets at a final cluster barrier and frees its TMEM.
 #pragma once
 
 #include "common.cuh"
@@ -78,10 +87,14 @@ constexpr int kPage = 64;            // tokens per page
 constexpr int kBlk = 256;            // tokens per block (four pages)
 constexpr int kPageBytes = kPage * kD * 2;
 constexpr int kChunk = 8192;         // 64 rows x 64 columns bf16, one swizzled operand tile
-constexpr int kQkBox = 2 * kChunk;   // one page x two chunks (16 KB)
-constexpr int kQkStageBytes = 2 * kQkBox;
-constexpr int kQkStages = 2;
-constexpr int kQkStagesPerBlock = 5; // chunks {0,1} {2,3} {4,5} {6,7} {8}
+#ifndef MLA_QK_CHUNKS_PER_STAGE
+#define MLA_QK_CHUNKS_PER_STAGE 2
+#endif
+constexpr int kQkCps = MLA_QK_CHUNKS_PER_STAGE;  // 64-column chunks per QK stage
+constexpr int kQkBox = kQkCps * kChunk;         // one page x kQkCps chunks
+constexpr int kQkStageBytes = 2 * kQkBox;       // both pages of this CTA
+constexpr int kQkStages = 65536 / kQkStageBytes;
+constexpr int kQkStagesPerBlock = (9 + kQkCps - 1) / kQkCps;
 constexpr int kPvStageBytes = 2 * kChunk;  // one page x 128 latent columns
 constexpr int kPvStages = 3;
 constexpr int kPvStagesPerBlock = 8;       // 4 pages x 2 latent halves
@@ -171,13 +184,14 @@ __device__ __forceinline__ int page_of(const DecodeTcParams& P, int b, int L, in
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(dtc::kThreads, 1)
     decode_tc_kernel(const __grid_constant__ CUtensorMap tmQ,
                      const __grid_constant__ CUtensorMap tmQK,
+                     const __grid_constant__ CUtensorMap tmPV,
                      const DecodeTcParams P) {
   using namespace dtc;
   extern __shared__ uint8_t smem_raw[];
   __shared__ __align__(8) uint64_t qk_full[kQkStages], qk_empty[kQkStages];
   __shared__ __align__(8) uint64_t pv_full[kPvStages], pv_empty[kPvStages];
-  __shared__ __align__(8) uint64_t q_full, q_empty, o_empty, p_full, pv_done, mma_drain;
-  __shared__ __align__(8) uint64_t s_full[2];
+  __shared__ __align__(8) uint64_t q_full, q_empty, o_empty, p_full, pv_done;
+  __shared__ __align__(8) uint64_t s_full[2], s_free[2], drain_qk, drain_pv;
   __shared__ float red_max[2][4][64];
   __shared__ float red_sum[4][64];
   __shared__ uint32_t tmem_base_sh;
@@ -199,8 +213,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(dtc::kThreads, 1)
       mbar_init(smem_u32(&qk_empty[s]), 1);  // MMA commit (multicast)
     }
     for (int s = 0; s < kPvStages; ++s) {
-      // 32 cp.async lanes of one loader warp (+ the peer's relay on the leader)
-      mbar_init(smem_u32(&pv_full[s]), rank == 0 ? 33u : 32u);
+      // one arrival per CTA's PV producer (the leader's carries the
+      // transaction bytes of both CTAs' boxes); only the leader's is used
+      mbar_init(smem_u32(&pv_full[s]), 2);
       mbar_init(smem_u32(&pv_empty[s]), 1);
     }
     mbar_init(smem_u32(&q_full), 1);
@@ -208,12 +223,16 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(dtc::kThreads, 1)
     mbar_init(smem_u32(&o_empty), 16);       // 8 softmax warps x 2 CTAs
     mbar_init(smem_u32(&p_full), 16);
     mbar_init(smem_u32(&pv_done), 1);
-    mbar_init(smem_u32(&mma_drain), 1);
-    mbar_init(smem_u32(&s_full[0]), 1);
-    mbar_init(smem_u32(&s_full[1]), 1);
+    mbar_init(smem_u32(&drain_qk), 1);
+    mbar_init(smem_u32(&drain_pv), 1);
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(smem_u32(&s_full[b]), 1);
+      mbar_init(smem_u32(&s_free[b]), 16);  // 8 softmax warps x 2 CTAs
+    }
     fence_mbar_init();
     tma_prefetch_desc(&tmQ);
     tma_prefetch_desc(&tmQK);
+    tma_prefetch_desc(&tmPV);
   }
   if (warp == 1) {
     tmem_alloc<2>(smem_u32(&tmem_base_sh), kTmemCols);
@@ -231,7 +250,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(dtc::kThreads, 1)
   const int hi = total > 0 ? worker_lo(worker + 1, total, P.G) : 0;
   const int rows_seq = P.S_q * P.H;
 
-  // Registers: the control warpgroup (producer, MMA, loaders) gives up most
+  // Registers: the control warpgroup (producers, MMA) gives up most
   // of its share to the two softmax warpgroups.
   static_assert(128 * kRegsControl + 256 * kRegsSoftmax <= 65536 &&
                     kRegsLaunch * kThreads <= 65536,
@@ -261,11 +280,21 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(dtc::kThreads, 1)
         for (int c = 0; c < 9; ++c)
           tma_load_2d_pair(sQ + c * kChunk, &tmQ, c * 64, row0, lead_qfull);
         ++q_issued;
+        // This CTA's two pages of each block: their ids are read from the
+        // page table two blocks ahead of the boxes (a table read takes as
+        // long as a box).
+        int cur[2], nxt[2];
+        for (int i = 0; i < 2; ++i) {
+          cur[i] = page_of(P, b, L, x0, 2 * (int)rank + i);
+          nxt[i] = x0 + 1 < x1 ? page_of(P, b, L, x0 + 1, 2 * (int)rank + i) : -1;
+        }
         for (int x = x0; x < x1 && ok; ++x) {
-          int pg[2];
+          int nn[2], pg[2];
           for (int i = 0; i < 2; ++i) {
-            pg[i] = page_of(P, b, L, x, 2 * (int)rank + i);
-            if (pg[i] < 0) pg[i] = P.n_pages;   // out of bounds: the box reads zeros
+            nn[i] = x + 2 < x1 ? page_of(P, b, L, x + 2, 2 * (int)rank + i) : -1;
+            pg[i] = cur[i] < 0 ? P.n_pages : cur[i];   // out of bounds: the box reads zeros
+            cur[i] = nxt[i];
+            nxt[i] = nn[i];
           }
           for (int k = 0; k < kQkStagesPerBlock; ++k, ++it) {
             const int s = it % kQkStages;
@@ -277,8 +306,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(dtc::kThreads, 1)
             if (rank == 0) mbar_expect_tx(smem_u32(&qk_full[s]), 2 * kQkStageBytes);
             const uint32_t dst = sQk + s * kQkStageBytes;
             // chunks 2k, 2k+1 of each page (chunk 9 is out of bounds: zeros)
-            tma_load_5d_pair(dst, &tmQK, 0, 0, 2 * k, 0, pg[0], fb);
-            tma_load_5d_pair(dst + kQkBox, &tmQK, 0, 0, 2 * k, 0, pg[1], fb);
+            tma_load_5d_pair(dst, &tmQK, 0, 0, kQkCps * k, 0, pg[0], fb);
+            tma_load_5d_pair(dst + kQkBox, &tmQK, 0, 0, kQkCps * k, 0, pg[1], fb);
           }
         }
         ++piece;
@@ -294,13 +323,19 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(dtc::kThreads, 1)
           mbar_wait_bounded(smem_u32(&qk_full[i % kQkStages]), (i / kQkStages) & 1, kDrainNs);
         if (q_issued > 0) mbar_wait_bounded(smem_u32(&q_full), (q_issued - 1) & 1, kDrainNs);
       }
-    } else if (warp == 2 || warp == 3) {
-      // ======  PV loader warps (cp.async): this CTA's latent half  ======
-      // Stage order per block: page p = 0..3, latent half n = 0..1; warp 2
-      // fills the even stages, warp 3 the odd ones.  A stage lands as
-      // [2 chunks][64 slots][128 B] for latent chunks 4n + 2r + {0, 1} of
-      // page p; rows past the sequence and pages past it are zeros.
-      const int mine = warp - 2;
+    } else if (warp == 2) {
+      // ======  PV producer: this CTA's latent half of every page  ======
+      // Stage order per block: page p = 0..3, latent half n = 0..1.  A stage
+      // lands as [2 chunks][64 slots][128 B] for latent chunks 4n + 2r +
+      // {0, 1} of page p, 128-byte swizzled.  A whole page, or a page past
+      // the sequence (out of bounds: zeros), comes as one TMA box completing
+      // on the leader's barrier, which the leader arms with both CTAs'
+      // bytes.  The partial last page of a sequence is copied by the warp
+      // with cp.async and zeros for the slots past the sequence: such a slot
+      // holds no cache entry (possibly NaN) and must not reach the MMA even
+      // though its P is 0.  Each CTA arrives once per stage on the leader's
+      // barrier.
+      const uint32_t lead_full0 = mapa_shared(smem_u32(&pv_full[0]), 0);
       uint32_t it = 0;
       PieceIter pi;
       pi.init(P.start, V, lo, hi);
@@ -311,191 +346,161 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(dtc::kThreads, 1)
         const int b = v / P.R;
         const int L = P.seq_lens[b];
         for (int x = x0; x < x1 && ok; ++x)
-          for (int p = 0; p < 4 && ok; ++p)
+          for (int p = 0; p < 4 && ok; ++p) {
+            const int pg = page_of(P, b, L, x, p);
+            const int valid = pg < 0 ? 0 : min(L - (x * kBlk + p * kPage), kPage);
             for (int n = 0; n < 2; ++n, ++it) {
-              if ((int)(it & 1) != mine) continue;
-              const int pg = page_of(P, b, L, x, p);
-              const int valid = pg < 0 ? 0 : min(L - (x * kBlk + p * kPage), kPage);
               const int s = it % kPvStages;
               const bool got = mbar_wait(smem_u32(&pv_empty[s]), ((it / kPvStages) & 1) ^ 1,
                                          abort_p, 11, it);
               if (!__all_sync(0xffffffffu, got)) { ok = false; break; }
-              const uint8_t* src = P.pool + (size_t)(pg < 0 ? 0 : pg) * kPageBytes +
-                                   (4 * n + 2 * (int)rank + cc) * 128 + u * 16;
-              const uint32_t dst = sPv + s * kPvStageBytes + cc * kChunk + (u << 4);
-  #pragma unroll 8
-              for (int i = 0; i < kPage; i += 2) {
-                const int row = i + rsub;
-                const uint32_t d = dst + row * 128;
-                const uint32_t dsw = d ^ ((uint32_t)(row & 7) << 4);
-                if (row < valid)
-                  cp_async16(dsw, src + (size_t)row * (kD * 2));
-                else
-                  st_shared_zero16(dsw);
+              const uint32_t dst = sPv + s * kPvStageBytes;
+              const uint32_t fb = lead_full0 + s * 8;
+              const int chunk0 = 4 * n + 2 * (int)rank;
+              if (valid == 0 || valid == kPage) {
+                if (lane == 0) {
+                  if (rank == 0) mbar_expect_tx(smem_u32(&pv_full[s]), 2 * kPvStageBytes);
+                  tma_load_3d_pair(dst, &tmPV, 0, (pg < 0 ? P.n_pages : pg) * kPage, chunk0, fb);
+                  if (rank == 1) mbar_arrive_cluster(fb);
+                }
+              } else {
+                const uint8_t* src =
+                    P.pool + (size_t)pg * kPageBytes + (chunk0 + cc) * 128 + u * 16;
+                const uint32_t d0 = dst + cc * kChunk + (u << 4);
+#pragma unroll 8
+                for (int i = 0; i < kPage; i += 2) {
+                  const int row = i + rsub;
+                  const uint32_t dsw = (d0 + row * 128) ^ ((uint32_t)(row & 7) << 4);
+                  if (row < valid)
+                    cp_async16(dsw, src + (size_t)row * (kD * 2));
+                  else
+                    st_shared_zero16(dsw);
+                }
+                asm volatile("cp.async.wait_all;" ::: "memory");
+                fence_proxy_async_smem();
+                __syncwarp();
+                if (lane == 0) {
+                  if (rank == 0) mbar_arrive(smem_u32(&pv_full[s]));
+                  else mbar_arrive_cluster(fb);
+                }
               }
-              if (valid < kPage) fence_proxy_async_smem();
-              cp_async_arrive_noinc(smem_u32(&pv_full[s]));
             }
+          }
       }
-      asm volatile("cp.async.wait_all;" ::: "memory");
-    } else if (warp == 1 && lane == 0 && rank == 1) {
-      // ======  peer relay: forward landed PV stages to the leader's barriers  ======
-      const uint32_t lead0 = mapa_shared(smem_u32(&pv_full[0]), 0);
-      PieceIter pi;
-      pi.init(P.start, V, lo, hi);
-      int v, x0, x1;
-      uint32_t it = 0;
+      if (!ok && rank == 0 && lane == 0) {
+        // Leaving early: wait (bounded) for the stages already armed, so
+        // that no box lands in this pair's shared memory after it exits (the
+        // peer's boxes count on the same barriers).
+        for (uint32_t i = it > (uint32_t)kPvStages ? it - kPvStages : 0u; i < it; ++i)
+          mbar_wait_bounded(smem_u32(&pv_full[i % kPvStages]), (i / kPvStages) & 1, kDrainNs);
+      }
+    } else if (warp == 1 && lane == 0 && rank == 0) {
+      // =================  QK MMA issuer (leader CTA)  =================
+      // QK(j) writes S buffer j & 1 once the softmax of block j - 2 has read
+      // it (s_free).  The QK and PV streams are issued by two threads of
+      // different warps: the tensor pipe holds little more than the MMA it
+      // runs, so the cycles one issuer spends between MMA groups (barrier
+      // waits, commits, bookkeeping) are covered by the other's MMAs.
+      const uint32_t idesc_qk = idesc_bf16_f32(128, 256, false, false);
+      // Operand descriptors are formed once; an MMA only adds its tile's
+      // offset (in 16-byte units) to the start-address field.
+      const uint64_t q_desc = sw128_desc(sQ, 16, 1024);
+      // the 16 slot groups of a chunk (both pages) lie 1 KB x kQkCps apart
+      const uint64_t qk_desc = sw128_desc(sQk, 16, 1024 * kQkCps);
+      PieceIter qi;
+      qi.init(P.start, V, lo, hi);
+      int v, x0, x1, piece = 0, jq = 0;
+      uint32_t itq = 0;
       bool ok = true;
-      while (ok && pi.next(v, x0, x1)) {
-        for (int x = x0; x < x1 && ok; ++x)
-          for (int k = 0; k < kPvStagesPerBlock; ++k, ++it) {
-            const int s = it % kPvStages;
-            if (!mbar_wait(smem_u32(&pv_full[s]), (it / kPvStages) & 1, abort_p, 14, it)) {
+      while (ok && qi.next(v, x0, x1)) {
+        ok = mbar_wait(smem_u32(&q_full), piece & 1, abort_p, 4, piece);
+        for (int x = x0; x < x1 && ok; ++x, ++jq) {
+          if (jq >= 2 && !mbar_wait(smem_u32(&s_free[jq & 1]), ((jq - 2) >> 1) & 1, abort_p, 5, jq)) {
+            ok = false;
+            break;
+          }
+          const uint32_t sd = tmem + kTmemS + 128 * (jq & 1);
+          for (int k = 0; k < kQkStagesPerBlock; ++k, ++itq) {
+            const int s = itq % kQkStages;
+            if (!mbar_wait(smem_u32(&qk_full[s]), (itq / kQkStages) & 1, abort_p, 6, itq)) {
               ok = false;
               break;
             }
-            fence_proxy_async_smem();
-            mbar_arrive_cluster(lead0 + s * 8);
-          }
-      }
-    } else if (warp == 1 && lane == 0 && rank == 0) {
-      // =================  MMA issuer (leader CTA)  =================
-      // Two streams share the tensor pipe: QK of block jq and PV of an
-      // earlier block jp.  Each turn issues at most one QK stage and one PV
-      // stage, each only if its operands have landed, so both rings drain
-      // steadily and the loads of each ring overlap the other stream's MMAs.
-      // QK(jq) writes S buffer jq & 1, which the softmax of block jq - 2
-      // releases when it hands over P(jq - 2): QK(jq) waits until PV(jq - 2)
-      // has begun.  PV(jp) begins once P(jp) is in and, for the first block
-      // of a piece, once the previous piece's epilogue has released O.
-      const uint32_t idesc_qk = idesc_bf16_f32(128, 256, false, false);
-      const uint32_t idesc_pv = idesc_bf16_f32(128, 256, false, true);
-      // Operand descriptors are formed once; an MMA only adds its tile's
-      // offset (in 16-byte units) to the start-address field, which keeps
-      // the issuing thread's work per MMA to a few integer adds.
-      const uint64_t q_desc = sw128_desc(sQ, 16, 1024);
-      const uint64_t p_desc = sw128_desc(sP, 16, 1024);
-      const uint64_t qk_desc = sw128_desc(sQk, 16, 2048);  // 16 slot groups 2 KB apart
-      const uint64_t pv_desc = sw128_desc(sPv, kChunk, 1024);
-      PieceIter qi, vi;
-      qi.init(P.start, V, lo, hi);
-      vi.init(P.start, V, lo, hi);
-      int qv, qx0 = 0, qx1 = 0, vv, vx0 = 0, vx1 = 0;
-      bool q_more = qi.next(qv, qx0, qx1), v_more = vi.next(vv, vx0, vx1);
-      int qx = qx0, q_piece = 0, jq = 0, kq = 0;   // QK: block, piece, stage
-      bool q_in = false;                           // Q of this QK piece landed
-      int vx = vx0, v_piece = 0, jp = 0, tp = 0;   // PV: block, piece, stage 0..7
-      bool p_in = false;                           // P of block jp in (and O free)
-      uint32_t itq = 0, itv = 0;
-      bool ok = true;
-      uint64_t t_stall = 0;                        // start of the current idle spell
-      uint32_t spins = 0;
-      while (ok && (q_more || v_more)) {
-        bool progressed = false;
-        // ---------------- one QK stage ----------------
-        if (q_more && jq <= jp + (p_in ? 1 : 0) + 1) {
-          bool ready = true;
-          if (!q_in) {
-            ready = mbar_test_wait(smem_u32(&q_full), q_piece & 1);
-            if (ready) q_in = true;
-          }
-          const int s = itq % kQkStages;
-          if (ready && mbar_test_wait(smem_u32(&qk_full[s]), (itq / kQkStages) & 1)) {
             tc_fence_after();
-            const uint32_t sd = tmem + kTmemS + 128 * (jq & 1);
-            const int ncc = (kq == kQkStagesPerBlock - 1) ? 1 : 2;
-            const uint64_t a0 = q_desc + (uint64_t)((2 * kq * kChunk) >> 4);
+            const uint64_t a0 = q_desc + (uint64_t)((kQkCps * k * kChunk) >> 4);
             const uint64_t b0 = qk_desc + (uint64_t)s * (kQkStageBytes >> 4);
-            for (int cc = 0; cc < ncc; ++cc) {
-              const int c = 2 * kq + cc;  // 64-column chunk of the 576
+#pragma unroll
+            for (int cc = 0; cc < kQkCps; ++cc) {
+              if (kQkCps * k + cc >= 9) break;   // past the 576 columns
 #pragma unroll
               for (int kk = 0; kk < 4; ++kk)
                 mma_bf16_ss<2>(sd, a0 + (uint64_t)((cc * kChunk + kk * 32) >> 4),
                                b0 + (uint64_t)((cc * 1024 + kk * 32) >> 4), idesc_qk,
-                               (c | kk) ? 1u : 0u);
+                               (k | cc | kk) ? 1u : 0u);
             }
             mma_commit_2_mc(smem_u32(&qk_empty[s]), 3);
-            ++itq;
-            progressed = true;
-            if (++kq == kQkStagesPerBlock) {
-              kq = 0;
-              mma_commit_2_mc(smem_u32(&s_full[jq & 1]), 3);
-              ++jq;
-              if (++qx == qx1) {
-                mma_commit_2_mc(smem_u32(&q_empty), 3);
-                q_more = qi.next(qv, qx0, qx1);
-                qx = qx0;
-                ++q_piece;
-                q_in = false;
-              }
-            }
           }
+          if (ok) mma_commit_2_mc(smem_u32(&s_full[jq & 1]), 3);
         }
-        // ---------------- one PV stage ----------------
-        if (v_more && jp < jq) {
-          if (!p_in) {
-            p_in = mbar_test_wait(smem_u32(&p_full), jp & 1) &&
-                   (vx != vx0 || v_piece == 0 ||
-                    mbar_test_wait(smem_u32(&o_empty), (v_piece - 1) & 1));
-            if (p_in) tc_fence_after();
-          }
-          const int s = itv % kPvStages;
-          if (p_in && mbar_test_wait(smem_u32(&pv_full[s]), (itv / kPvStages) & 1)) {
-            // The stage was written by cp.async and st.shared (generic
-            // proxy); the MMA reads it through the async proxy.  The writes
-            // are ordered before this thread by the barrier; the proxy fence
-            // makes them visible to the MMAs issued next.  (The peer's half
-            // is fenced the same way by its relay lane.)
+        // the Q slice is free once this piece's QK MMAs completed
+        if (ok) mma_commit_2_mc(smem_u32(&q_empty), 3);
+        ++piece;
+      }
+      if (!ok) {
+        // Leaving early: one more commit tracks every MMA this thread issued;
+        // wait (bounded) for it, so that none still reads shared memory or
+        // writes TMEM when the pair frees them.
+        mma_commit_2_mc(smem_u32(&drain_qk), 1);
+        mbar_wait_bounded(smem_u32(&drain_qk), 0, kDrainNs);
+      }
+    } else if (warp == 3 && lane == 0 && rank == 0) {
+      // =================  PV MMA issuer (leader CTA)  =================
+      // PV(j) begins once P(j) is in and, for the first block of a piece,
+      // once the previous piece's epilogue has released O.
+      const uint32_t idesc_pv = idesc_bf16_f32(128, 256, false, true);
+      const uint64_t p_desc = sw128_desc(sP, 16, 1024);
+      const uint64_t pv_desc = sw128_desc(sPv, kChunk, 1024);
+      PieceIter vi;
+      vi.init(P.start, V, lo, hi);
+      int v, x0, x1, piece = 0, jp = 0;
+      uint32_t itv = 0;
+      bool ok = true;
+      while (ok && vi.next(v, x0, x1)) {
+        for (int x = x0; x < x1 && ok; ++x, ++jp) {
+          ok = mbar_wait(smem_u32(&p_full), jp & 1, abort_p, 2, jp);
+          if (ok && x == x0 && piece > 0)
+            ok = mbar_wait(smem_u32(&o_empty), (piece - 1) & 1, abort_p, 3, piece);
+          for (int t = 0; t < kPvStagesPerBlock && ok; ++t, ++itv) {
+            const int s = itv % kPvStages;
+            if (!mbar_wait(smem_u32(&pv_full[s]), (itv / kPvStages) & 1, abort_p, 9, itv)) {
+              ok = false;
+              break;
+            }
+            // A partial-page stage was written by cp.async and st.shared
+            // (generic proxy) and the MMA reads it through the async proxy.
+            // Its writers fenced before arriving; the barrier orders their
+            // writes before this thread, and this proxy fence orders them
+            // before the MMAs issued next.
             fence_proxy_async_smem();
             tc_fence_after();
-            const int p = tp >> 1, n = tp & 1;
-            const bool first = (vx == vx0);
-            const uint64_t a0 = p_desc + (uint64_t)((p * kChunk) >> 4);
+            const int pp = t >> 1, n = t & 1;
+            const uint64_t a0 = p_desc + (uint64_t)((pp * kChunk) >> 4);
             const uint64_t b0 = pv_desc + (uint64_t)s * (kPvStageBytes >> 4);
 #pragma unroll
             for (int kk = 0; kk < 4; ++kk) {
-              const uint32_t acc = (first && p == 0 && kk == 0) ? 0u : 1u;
+              const uint32_t acc = (x == x0 && pp == 0 && kk == 0) ? 0u : 1u;
               mma_bf16_ss<2>(tmem + kTmemO + 128 * n, a0 + (uint64_t)((kk * 32) >> 4),
                              b0 + (uint64_t)((kk * 2048) >> 4), idesc_pv, acc);
             }
             mma_commit_2_mc(smem_u32(&pv_empty[s]), 3);
-            ++itv;
-            progressed = true;
-            if (++tp == kPvStagesPerBlock) {
-              tp = 0;
-              mma_commit_2_mc(smem_u32(&pv_done), 3);
-              ++jp;
-              p_in = false;
-              if (++vx == vx1) {
-                v_more = vi.next(vv, vx0, vx1);
-                vx = vx0;
-                ++v_piece;
-              }
-            }
           }
+          if (ok) mma_commit_2_mc(smem_u32(&pv_done), 3);
         }
-        // ---------------- bounded idle ----------------
-        if (progressed) {
-          spins = 0;
-        } else if ((++spins & 63u) == 0) {
-          const uint64_t now = globaltimer();
-          if (spins == 64) t_stall = now;
-          if (*abort_p) {
-            ok = false;
-          } else if (now - t_stall > MLA_WAIT_NS) {
-            raise_flag(kFlagTimeout);
-            record_timeout(3, (uint32_t)jq, (uint32_t)jp);
-            *abort_p = 1;
-            ok = false;
-          }
-        }
+        ++piece;
       }
       if (!ok) {
-        // Leaving early: one more commit tracks every MMA issued so far; wait
-        // (bounded) for it, so that no MMA still reads shared memory or writes
-        // TMEM when the pair frees them.
-        mma_commit_2_mc(smem_u32(&mma_drain), 1);
-        mbar_wait_bounded(smem_u32(&mma_drain), 0, kDrainNs);
+        mma_commit_2_mc(smem_u32(&drain_pv), 1);
+        mbar_wait_bounded(smem_u32(&drain_pv), 0, kDrainNs);
       }
     }
   } else {
@@ -508,6 +513,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(dtc::kThreads, 1)
     const int pb = 2 * hh + ch;                      // page of the block this thread scores
     const uint32_t lane_addr = (uint32_t)(32 * quad) << 16;
     const uint32_t lead_pfull = mapa_shared(smem_u32(&p_full), 0);
+    const uint32_t lead_sfree = mapa_shared(smem_u32(&s_free[0]), 0);
     const uint32_t lead_oempty = mapa_shared(smem_u32(&o_empty), 0);
     const uint32_t prow = sP + pb * kChunk + h * 128;
     PieceIter pi;
@@ -581,6 +587,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(dtc::kThreads, 1)
             pk[16 * hf + e] = pack_bf16x2(p0, p1);
           }
         }
+        // S buffer j & 1 is read: QK(j + 2) may overwrite it
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive_cluster(lead_sfree + 8 * (j & 1));
         // PV(j-1) must be done before P is overwritten and before O is rescaled
         bool ok = true;
         if (j > 0) ok = mbar_wait(smem_u32(&pv_done), (j - 1) & 1, abort_p, 8, j);
@@ -666,7 +676,7 @@ inline mla_status launch_decode_tc_impl(
     const int32_t* seq_lens, const int32_t* tail, int B, int S_q, int H, float scale, int G,
     const int32_t* start, float* ws_lse, float* ws_o, cudaStream_t st) {
   using namespace dtc;
-  CUtensorMap tQ, tQK;
+  CUtensorMap tQ, tQK, tPV;
   {
     const uint64_t dims[2] = {(uint64_t)kD, (uint64_t)B * S_q * H};
     const uint64_t strides[1] = {(uint64_t)kD * 2};
@@ -681,8 +691,17 @@ inline mla_status launch_decode_tc_impl(
     const uint64_t dims[5] = {64, 8, 9, 8, (uint64_t)n_pages};
     const uint64_t strides[4] = {(uint64_t)kD * 2, 128, (uint64_t)kD * 2 * 8,
                                  (uint64_t)kPageBytes};
-    const uint32_t box[5] = {64, 8, 2, 8, 1};
+    const uint32_t box[5] = {64, 8, (uint32_t)kQkCps, 8, 1};
     if (!make_tmap(&tQK, pool, 5, dims, strides, box)) return MLA_ERR_CUDA;
+  }
+  // The pool seen as (64 columns, pool rows, 9 chunks): a box of two chunks
+  // of one page lands as [chunk][64 slots][64 columns], the MN-major operand
+  // layout of the PV MMAs.
+  {
+    const uint64_t dims[3] = {64, (uint64_t)n_pages * kPage, 9};
+    const uint64_t strides[2] = {(uint64_t)kD * 2, 128};
+    const uint32_t box[3] = {64, (uint32_t)kPage, 2};
+    if (!make_tmap(&tPV, pool, 3, dims, strides, box)) return MLA_ERR_CUDA;
   }
   DecodeTcParams p;
   p.pool = static_cast<const uint8_t*>(pool);
@@ -703,7 +722,7 @@ inline mla_status launch_decode_tc_impl(
   if (cudaFuncSetAttribute(decode_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            (int)kSmemBytes) != cudaSuccess)
     return MLA_ERR_CUDA;
-  decode_tc_kernel<<<2 * G, kThreads, kSmemBytes, st>>>(tQ, tQK, p);
+  decode_tc_kernel<<<2 * G, kThreads, kSmemBytes, st>>>(tQ, tQK, tPV, p);
   return cudaGetLastError() == cudaSuccess ? MLA_OK : MLA_ERR_CUDA;
 }
 
