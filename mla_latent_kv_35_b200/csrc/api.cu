@@ -539,10 +539,9 @@ static mla_status decode_impl(const mla_dims* dims, const void* qbuf, const void
 #undef MLA_SIMT_DECODE
     MLA_TRY(check_launch());
   }
-  dim3 cgrid(L.V, (L.rows_per_v + 7) / 8);
-  combine_kernel<<<cgrid, 256, 0, st>>>(ws_lse, ws_o, start, L.V, L.R, L.G, L.rows_per_v,
-                                        S_q * H, dc,
-                                        o_lat, lse);
+  dim3 cgrid(L.V, L.rows_per_v);
+  combine_kernel<<<cgrid, kCombineThreads, 0, st>>>(ws_lse, ws_o, start, L.V, L.R, L.G,
+                                                    L.rows_per_v, S_q * H, dc, o_lat, lse);
   return check_launch();
 }
 
@@ -601,9 +600,10 @@ mla_status mla_decode_fp8(const mla_dims* dims, const void* qbuf, const void* po
                                  seq_lens, nullptr, B, S_q, dims->n_heads, dims->scale, L.G,
                                  start, ws_lse, ws_o, st));
   g_launches.fetch_add(1, std::memory_order_relaxed);
-  dim3 cgrid(L.V, (L.rows_per_v + 7) / 8);
-  combine_kernel<<<cgrid, 256, 0, st>>>(ws_lse, ws_o, start, L.V, L.R, L.G, L.rows_per_v,
-                                        S_q * dims->n_heads, dims->d_latent, o_lat, lse);
+  dim3 cgrid(L.V, L.rows_per_v);
+  combine_kernel<<<cgrid, kCombineThreads, 0, st>>>(ws_lse, ws_o, start, L.V, L.R, L.G,
+                                                    L.rows_per_v, S_q * dims->n_heads,
+                                                    dims->d_latent, o_lat, lse);
   return check_launch();
 }
 

@@ -22,10 +22,13 @@
 //     per instruction, so 256-token blocks halve the QK instruction count).
 //   * PV: pair MMAs with N = 256 latent columns (two per 16-token step, one
 //     per latent half n).  CTA r supplies latent columns [256n + 128r, +128)
-//     of all 256 tokens (MN-major B) and its own 64 rows of P (bf16,
-//     K-major).  O takes 256 TMEM columns per SM, S 2 x 128 more: all 512.
+//     of all 256 tokens (MN-major B).  A is P in TMEM: in a pair MMA, output
+//     lane l reads its A row from TMEM lane l of its own CTA, so lanes l and
+//     l + 64 (the same row, the two token halves of S) both need that row's
+//     P for all 256 tokens, bf16 pairs in 128 columns.  P(j) overwrites S(j)
+//     in place.  O takes 256 TMEM columns per SM, S/P 2 x 128 more: all 512.
 //   * QK loads.  Lane 0 of warp 0 in each CTA streams its two pages through a
-//     ring of two 32 KB stages; a stage holds two 64-column chunks of both
+//     ring of three 32 KB stages; a stage holds two 64-column chunks of both
 //     pages, one 16 KB TMA box per page from a 5-D view of the pool:
 //     (64 columns, 8 slots, 9 chunks, 8 slot groups, pages).  The box lands as
 //     [slot group][chunk][8 slots][128 B], so the two pages' slot groups of a
@@ -45,9 +48,11 @@
 //     the scores of one row on one page.  Row maxima of the four pages meet
 //     in shared memory.  The running max is rescaled lazily: O is rescaled
 //     in TMEM only when a row's max grows by more than 2^8, warp-uniformly.
-//     After its last read of S the softmax releases the S buffer (s_free);
-//     P goes to shared memory once PV of the previous block is done, and
-//     the PV issuer is signalled.
+//     P goes to TMEM over S: warps w and w ^ 2 hold the two token halves of
+//     the same rows and swap them through an 8 KB shared buffer, one warp
+//     pair per round, four rounds.  P(j) waits for nothing from PV(j - 1):
+//     O is rescaled (after PV(j - 1)) only when a row's max moved.  S/P
+//     buffer j & 1 is released for QK(j + 2) by a commit after PV(j).
 //   * MMA issue.  Two threads of the leader issue the MMAs: lane 0 of warp 1
 //     the QK stream, lane 0 of warp 3 the PV stream.  The tensor pipe
 //     buffers little beyond the MMA it runs, and every barrier wait, commit
@@ -58,7 +63,8 @@
 //     outputs and natural-log LSE into slot worker + v of the workspace; the
 //     combine kernel merges them.
 //
-// Shared memory: Q 72 KB + P 32 KB + QK ring 64 KB + PV ring 48 KB.
+// Shared memory: Q 72 KB + QK ring 96 KB + PV ring 48 KB + P exchange 8 KB
+// (also the row sums of the epilogue), 1.2 KB of barriers and row maxima.
 //
 // Partial and missing pages.  QK boxes always load a whole page; slots past
 // the sequence hold whatever the pool holds there and are masked by index in
@@ -93,18 +99,18 @@ constexpr int kChunk = 8192;         // 64 rows x 64 columns bf16, one swizzled 
 constexpr int kQkCps = MLA_QK_CHUNKS_PER_STAGE;  // 64-column chunks per QK stage
 constexpr int kQkBox = kQkCps * kChunk;         // one page x kQkCps chunks
 constexpr int kQkStageBytes = 2 * kQkBox;       // both pages of this CTA
-constexpr int kQkStages = 65536 / kQkStageBytes;
+constexpr int kQkStages = 98304 / kQkStageBytes;
 constexpr int kQkStagesPerBlock = (9 + kQkCps - 1) / kQkCps;
 constexpr int kPvStageBytes = 2 * kChunk;  // one page x 128 latent columns
 constexpr int kPvStages = 3;
 constexpr int kPvStagesPerBlock = 8;       // 4 pages x 2 latent halves
 constexpr int kQBytes = 9 * kChunk;        // 64 rows x 576 columns
-constexpr int kPBytes = 4 * kChunk;        // 64 rows x 256 tokens
+constexpr int kXBytes = 8192;              // P exchange between TMEM lane halves
 constexpr uint32_t kOffQ = 0;
-constexpr uint32_t kOffP = kOffQ + kQBytes;
-constexpr uint32_t kOffQk = kOffP + kPBytes;
+constexpr uint32_t kOffQk = kOffQ + kQBytes;
 constexpr uint32_t kOffPv = kOffQk + kQkStages * kQkStageBytes;
-constexpr uint32_t kSmemBytes = kOffPv + kPvStages * kPvStageBytes + 1024;  // + alignment
+constexpr uint32_t kOffX = kOffPv + kPvStages * kPvStageBytes;
+constexpr uint32_t kSmemBytes = kOffX + kXBytes + 1024;  // + alignment
 constexpr int kThreads = 384;
 constexpr int kSoftmaxWarp0 = 4;
 constexpr int kSoftmaxThreads = 256;
@@ -115,7 +121,7 @@ constexpr int kRegsControl = 136;
 constexpr int kRegsSoftmax = 184;
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kTmemO = 0;       // O_n at columns [128n, 128n + 128)
-constexpr uint32_t kTmemS = 256;     // S_b at columns [256 + 128b, +128)
+constexpr uint32_t kTmemS = 256;     // S_b, then P_b, at columns [256 + 128b, +128)
 constexpr float kRescaleLog2 = 8.0f;
 }  // namespace dtc
 
@@ -190,10 +196,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(dtc::kThreads, 1)
   extern __shared__ uint8_t smem_raw[];
   __shared__ __align__(8) uint64_t qk_full[kQkStages], qk_empty[kQkStages];
   __shared__ __align__(8) uint64_t pv_full[kPvStages], pv_empty[kPvStages];
-  __shared__ __align__(8) uint64_t q_full, q_empty, o_empty, p_full, pv_done;
+  __shared__ __align__(8) uint64_t q_full, q_empty, o_empty, p_full[2], pv_done;
   __shared__ __align__(8) uint64_t s_full[2], s_free[2], drain_qk, drain_pv;
-  __shared__ float red_max[2][4][64];
-  __shared__ float red_sum[4][64];
+  __shared__ float red_max[4][64];
   __shared__ uint32_t tmem_base_sh;
   __shared__ int abort_flag;
 
@@ -201,7 +206,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(dtc::kThreads, 1)
   const uint32_t rank = cluster_ctarank();
   const int worker = blockIdx.x >> 1;
   const uint32_t base = (smem_u32(smem_raw) + 1023u) & ~1023u;
-  const uint32_t sQ = base + kOffQ, sP = base + kOffP;
+  const uint32_t sQ = base + kOffQ, sX = base + kOffX;
   const uint32_t sQk = base + kOffQk, sPv = base + kOffPv;
 
   if (threadIdx.x == 0) {
@@ -221,13 +226,21 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(dtc::kThreads, 1)
     mbar_init(smem_u32(&q_full), 1);
     mbar_init(smem_u32(&q_empty), 1);
     mbar_init(smem_u32(&o_empty), 16);       // 8 softmax warps x 2 CTAs
-    mbar_init(smem_u32(&p_full), 16);
+    // P_b in TMEM, 8 softmax warps x 2 CTAs.  One barrier per P buffer: the
+    // softmax of one CTA may reach block j + 1 before the other CTA's
+    // softmax has handed over P(j) (nothing ties the two CTAs' softmax
+    // together once P no longer waits for the previous PV), and arrivals of
+    // two blocks must not meet on one barrier.  Block j + 2 cannot arrive
+    // before phase j completes: its S needs PV(j) to have released the
+    // buffer.
+    mbar_init(smem_u32(&p_full[0]), 16);
+    mbar_init(smem_u32(&p_full[1]), 16);
     mbar_init(smem_u32(&pv_done), 1);
     mbar_init(smem_u32(&drain_qk), 1);
     mbar_init(smem_u32(&drain_pv), 1);
     for (int b = 0; b < 2; ++b) {
       mbar_init(smem_u32(&s_full[b]), 1);
-      mbar_init(smem_u32(&s_free[b]), 16);  // 8 softmax warps x 2 CTAs
+      mbar_init(smem_u32(&s_free[b]), 1);   // PV commit: P_b consumed
     }
     fence_mbar_init();
     tma_prefetch_desc(&tmQ);
@@ -455,10 +468,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(dtc::kThreads, 1)
       }
     } else if (warp == 3 && lane == 0 && rank == 0) {
       // =================  PV MMA issuer (leader CTA)  =================
-      // PV(j) begins once P(j) is in and, for the first block of a piece,
-      // once the previous piece's epilogue has released O.
+      // PV(j) begins once P(j) is in TMEM and, for the first block of a
+      // piece, once the previous piece's epilogue has released O.  A is P(j)
+      // in TMEM (S buffer j & 1): lane l holds the row of output lane l, 256
+      // tokens as bf16 pairs in 128 columns, so K-step kk of page p starts at
+      // column 32p + 8kk.  Once PV(j) has completed, buffer j & 1 is free for
+      // QK(j + 2).
       const uint32_t idesc_pv = idesc_bf16_f32(128, 256, false, true);
-      const uint64_t p_desc = sw128_desc(sP, 16, 1024);
       const uint64_t pv_desc = sw128_desc(sPv, kChunk, 1024);
       PieceIter vi;
       vi.init(P.start, V, lo, hi);
@@ -467,7 +483,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(dtc::kThreads, 1)
       bool ok = true;
       while (ok && vi.next(v, x0, x1)) {
         for (int x = x0; x < x1 && ok; ++x, ++jp) {
-          ok = mbar_wait(smem_u32(&p_full), jp & 1, abort_p, 2, jp);
+          ok = mbar_wait(smem_u32(&p_full[jp & 1]), (jp >> 1) & 1, abort_p, 2, jp);
           if (ok && x == x0 && piece > 0)
             ok = mbar_wait(smem_u32(&o_empty), (piece - 1) & 1, abort_p, 3, piece);
           for (int t = 0; t < kPvStagesPerBlock && ok; ++t, ++itv) {
@@ -484,17 +500,20 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(dtc::kThreads, 1)
             fence_proxy_async_smem();
             tc_fence_after();
             const int pp = t >> 1, n = t & 1;
-            const uint64_t a0 = p_desc + (uint64_t)((pp * kChunk) >> 4);
+            const uint32_t a0 = tmem + kTmemS + 128 * (jp & 1) + 32 * pp;
             const uint64_t b0 = pv_desc + (uint64_t)s * (kPvStageBytes >> 4);
 #pragma unroll
             for (int kk = 0; kk < 4; ++kk) {
               const uint32_t acc = (x == x0 && pp == 0 && kk == 0) ? 0u : 1u;
-              mma_bf16_ss<2>(tmem + kTmemO + 128 * n, a0 + (uint64_t)((kk * 32) >> 4),
+              mma_bf16_ts<2>(tmem + kTmemO + 128 * n, a0 + 8 * kk,
                              b0 + (uint64_t)((kk * 2048) >> 4), idesc_pv, acc);
             }
             mma_commit_2_mc(smem_u32(&pv_empty[s]), 3);
           }
-          if (ok) mma_commit_2_mc(smem_u32(&pv_done), 3);
+          if (ok) {
+            mma_commit_2_mc(smem_u32(&pv_done), 3);
+            mma_commit_2_mc(smem_u32(&s_free[jp & 1]), 1);
+          }
         }
         ++piece;
       }
@@ -512,10 +531,15 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(dtc::kThreads, 1)
     const int h = tl & 63, hh = tl >> 6;             // row of this CTA, token half
     const int pb = 2 * hh + ch;                      // page of the block this thread scores
     const uint32_t lane_addr = (uint32_t)(32 * quad) << 16;
-    const uint32_t lead_pfull = mapa_shared(smem_u32(&p_full), 0);
-    const uint32_t lead_sfree = mapa_shared(smem_u32(&s_free[0]), 0);
+    const uint32_t lead_pfull = mapa_shared(smem_u32(&p_full[0]), 0);
     const uint32_t lead_oempty = mapa_shared(smem_u32(&o_empty), 0);
-    const uint32_t prow = sP + pb * kChunk + h * 128;
+    // P exchange: warps sw and sw ^ 2 hold the two token halves of the same
+    // rows; pair (sw & 1) + 2 (sw >> 2) swaps them through sX in round
+    // number pair, half (sw >> 1) & 1 of the buffer written by each warp
+    const int xpair = (sw & 1) | ((sw >> 2) << 1);
+    const uint32_t x_mine = sX + ((sw >> 1) & 1) * 4096 + lane * 128;
+    const uint32_t x_theirs = sX + (((sw >> 1) & 1) ^ 1) * 4096 + lane * 128;
+    float* red_sum = reinterpret_cast<float*>(smem_raw + (sX - smem_u32(smem_raw)));  // [4][64]
     PieceIter pi;
     pi.init(P.start, V, lo, hi);
     int v, x0, x1;
@@ -552,12 +576,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(dtc::kThreads, 1)
               if (32 * hf + c < cmax) mx = fmaxf(mx, __uint_as_float(r[c]));
           }
         }
-        red_max[j & 1][pb][h] = mx;
+        red_max[pb][h] = mx;
         // one barrier: the other pages' maxima visible, and everyone agrees
         // to go on
         if (named_bar_or(1, kSoftmaxThreads, !got || *abort_p)) { dead = true; break; }
 #pragma unroll
-        for (int q2 = 0; q2 < 4; ++q2) mx = fmaxf(mx, red_max[j & 1][q2][h]);
+        for (int q2 = 0; q2 < 4; ++q2) mx = fmaxf(mx, red_max[q2][h]);
         const float m_blk = mx * P.scale_log2;
         // Lazy rescale: a row moves its running max only when the block max
         // exceeds it by more than 2^kRescaleLog2.  TMEM loads/stores are
@@ -587,15 +611,49 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(dtc::kThreads, 1)
             pk[16 * hf + e] = pack_bf16x2(p0, p1);
           }
         }
-        // S buffer j & 1 is read: QK(j + 2) may overwrite it
+        // P(j) goes to TMEM over S(j), as the A operand of PV(j): every lane
+        // needs all 256 tokens of its row, so the two warps holding the two
+        // halves of the same rows swap theirs through shared memory (four
+        // rounds, one warp pair each; the barriers also order every thread's
+        // last read of S before any write of P).
+        uint32_t pq[32];
         tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive_cluster(lead_sfree + 8 * (j & 1));
-        // PV(j-1) must be done before P is overwritten and before O is rescaled
+        bool stop = false;
+#pragma unroll 1
+        for (int rho = 0; rho < 4; ++rho) {
+          if (xpair == rho) {
+#pragma unroll
+            for (int u = 0; u < 8; ++u)
+              asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(
+                               x_mine + ((u ^ (lane & 7)) << 4)),
+                           "r"(pk[4 * u]), "r"(pk[4 * u + 1]), "r"(pk[4 * u + 2]),
+                           "r"(pk[4 * u + 3])
+                           : "memory");
+          }
+          named_bar_sync(2, kSoftmaxThreads);
+          if (xpair == rho) {
+#pragma unroll
+            for (int u = 0; u < 8; ++u)
+              asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];"
+                           : "=r"(pq[4 * u]), "=r"(pq[4 * u + 1]), "=r"(pq[4 * u + 2]),
+                             "=r"(pq[4 * u + 3])
+                           : "r"(x_theirs + ((u ^ (lane & 7)) << 4))
+                           : "memory");
+          }
+          if (rho < 3) named_bar_sync(3, kSoftmaxThreads);
+          else stop = named_bar_or(3, kSoftmaxThreads, *abort_p != 0);
+        }
+        if (stop) { dead = true; break; }
+        tc_fence_after();
+        // O is rescaled only when some row of this warp moved its max; PV of
+        // the previous block accumulates into O and must be done first.
         bool ok = true;
-        if (j > 0) ok = mbar_wait(smem_u32(&pv_done), (j - 1) & 1, abort_p, 8, j);
-        if (__all_sync(0xffffffffu, ok)) {
-          if (o_started && __any_sync(0xffffffffu, need)) {
+        if (o_started && __any_sync(0xffffffffu, need)) {
+          // parity wait: PV(j - 2) is done (S(j) needed its P buffer), so at
+          // most one phase is outstanding
+          ok = __all_sync(0xffffffffu,
+                          mbar_wait(smem_u32(&pv_done), (j - 1) & 1, abort_p, 8, j));
+          if (ok) {
             tc_fence_after();
             for (int cc = 0; cc < 4; ++cc) {
               uint32_t r[32];
@@ -607,33 +665,36 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(dtc::kThreads, 1)
                 r[i] = __float_as_uint(__uint_as_float(r[i]) * alpha);
               tmem_st32(oa, r);
             }
-            tmem_wait_st();
           }
-#pragma unroll
-          for (int u = 0; u < 8; ++u) {
-            const uint32_t addr = prow + ((u ^ (h & 7)) << 4);
-            asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr),
-                         "r"(pk[4 * u]), "r"(pk[4 * u + 1]), "r"(pk[4 * u + 2]),
-                         "r"(pk[4 * u + 3])
-                         : "memory");
-          }
+        }
+        {
+          const uint32_t pa = tmem + lane_addr + kTmemS + 128 * (j & 1) + 32 * ch;
+          tmem_st32(pa + 64 * hh, pk);
+          tmem_st32(pa + 64 * (1 - hh), pq);
+          tmem_wait_st();
         }
         l = need ? l * alpha + lsum : l + lsum;
         m = m_use;
-        fence_proxy_async_smem();
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive_cluster(lead_pfull);
+        if (lane == 0 && ok) mbar_arrive_cluster(lead_pfull + 8 * (j & 1));
         o_started = true;
       }
       if (dead) break;
       // ---------------- epilogue of the piece ----------------
+      // O is final once PV of the piece's last block jl is done.  The
+      // softmax may be up to two blocks ahead of PV here (it no longer waits
+      // for PV(j - 1) before handing over P(j)), and a parity wait is sound
+      // only when at most one phase is outstanding: wait for PV(jl - 1)
+      // first, then for PV(jl).
       const int jl = j - 1;
-      const bool got = mbar_wait(smem_u32(&pv_done), jl & 1, abort_p, 10, jl);
-      red_sum[pb][h] = l;
+      bool got = true;
+      if (jl > 0) got = mbar_wait(smem_u32(&pv_done), (jl - 1) & 1, abort_p, 10, jl);
+      got = got && mbar_wait(smem_u32(&pv_done), jl & 1, abort_p, 10, jl);
+      red_sum[64 * pb + h] = l;
       if (named_bar_or(1, kSoftmaxThreads, !got || *abort_p)) { dead = true; break; }
       tc_fence_after();
-      const float lt = red_sum[0][h] + red_sum[1][h] + red_sum[2][h] + red_sum[3][h];
+      const float lt = red_sum[h] + red_sum[64 + h] + red_sum[128 + h] + red_sum[192 + h];
       const float inv = lt > 0.f ? 1.f / lt : 0.f;
       const long long slot = (long long)worker + v;
       const long long row = slot * 128 + 64 * (int)rank + h;

@@ -274,62 +274,84 @@ __global__ void __launch_bounds__(256) decode_simt_kernel(
 // ---------------------------------------------------------------------------
 // Log-sum-exp combine of the pieces of every virtual sequence.
 //   o = sum_k w_k o_k / sum_k w_k, w_k = exp(lse_k - max lse), lse = max + ln sum w
-// Grid (V, ceil(rows_per_v / 8)), one warp per row.  Virtual sequence v is
-// row block v % R of sequence v / R: rows_per_v workspace rows, of which the
-// ones past the sequence's rows_seq query rows are padding and skipped.
+// Grid (V, rows_per_v), one CTA of 128 threads per row.  Warp 0 reduces the
+// pieces' LSEs of the row (lanes take pieces in parallel); then thread t
+// merges columns [4t, 4t + 4) (d_c <= 512, a multiple of 4) with eight
+// pieces' partial rows in flight at a time, so that a row merging many
+// pieces (a long sequence split over many workers) is not a chain of
+// dependent loads.  Virtual sequence v is row block v % R of sequence v / R:
+// rows_per_v workspace rows, of which the ones past the sequence's rows_seq
+// query rows are padding and skipped.
 // ---------------------------------------------------------------------------
-__global__ void __launch_bounds__(256) combine_kernel(const float* ws_lse, const float* ws_o,
-                                                      const int32_t* start, int V, int R, int G,
-                                                      int rows_per_v, int rows_seq, int d_c,
-                                                      float* o_lat, float* lse) {
+constexpr int kCombineThreads = 128;
+
+__global__ void __launch_bounds__(kCombineThreads) combine_kernel(
+    const float* ws_lse, const float* ws_o, const int32_t* start, int V, int R, int G,
+    int rows_per_v, int rows_seq, int d_c, float* o_lat, float* lse) {
+  __shared__ float mx_sh, inv_z_sh;
   const int v = blockIdx.x;
-  const int r = blockIdx.y * 8 + (threadIdx.x >> 5);
-  const int lane = threadIdx.x & 31;
+  const int r = blockIdx.y;
   const int row_in_seq = (v % R) * rows_per_v + r;
-  if (r >= rows_per_v || row_in_seq >= rows_seq) return;
+  if (row_in_seq >= rows_seq) return;
   const int total = start[V];
   const long long out_row = (long long)(v / R) * rows_seq + row_in_seq;
-  float* dst = o_lat + out_row * d_c;
-  if (start[v + 1] == start[v]) {
-    for (int c = lane; c < d_c; c += 32) dst[c] = 0.f;
-    if (lane == 0) lse[out_row] = -INFINITY;
-    return;
-  }
-  const int k0 = worker_of(start[v], total, G);
-  const int k1 = worker_of(start[v + 1] - 1, total, G);
-  // workers with an empty range (only when G > total) wrote no slot
-#define MLA_LIVE(k) (worker_lo((k) + 1, total, G) > worker_lo((k), total, G))
-  float mx = -INFINITY;
-  for (int k = k0; k <= k1; ++k)
-    if (MLA_LIVE(k)) mx = fmaxf(mx, ws_lse[((long long)k + v) * rows_per_v + r]);
-  if (mx == -INFINITY) {
-    for (int c = lane; c < d_c; c += 32) dst[c] = 0.f;
-    if (lane == 0) lse[out_row] = -INFINITY;
-    return;
-  }
-  float z = 0.f;
-  for (int k = k0; k <= k1; ++k)
-    if (MLA_LIVE(k)) z += __expf(ws_lse[((long long)k + v) * rows_per_v + r] - mx);
-  const float inv_z = 1.f / z;
-  for (int c4 = lane * 4; c4 < d_c; c4 += 128) {
-    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-    for (int k = k0; k <= k1; ++k) {
-      if (!MLA_LIVE(k)) continue;
-      const long long slot = (long long)k + v;
-      const float w = __expf(ws_lse[slot * rows_per_v + r] - mx) * inv_z;
-      const float4 x = *reinterpret_cast<const float4*>(ws_o + (slot * rows_per_v + r) * d_c + c4);
-      acc.x = fmaf(w, x.x, acc.x);
-      acc.y = fmaf(w, x.y, acc.y);
-      acc.z = fmaf(w, x.z, acc.z);
-      acc.w = fmaf(w, x.w, acc.w);
+  const bool any = start[v + 1] > start[v];
+  const int k0 = any ? worker_of(start[v], total, G) : 0;
+  const int n = any ? worker_of(start[v + 1] - 1, total, G) - k0 + 1 : 0;
+  // lse of piece i of the row, -inf for a worker with an empty range (only
+  // when G > total), which wrote no slot
+  auto piece_lse = [&](int i) {
+    const int k = k0 + i;
+    return worker_lo(k + 1, total, G) > worker_lo(k, total, G)
+               ? ws_lse[((long long)k + v) * rows_per_v + r] : -INFINITY;
+  };
+  if (threadIdx.x < 32) {
+    const int lane = threadIdx.x;
+    float mx = -INFINITY;
+    for (int i = lane; i < n; i += 32) mx = fmaxf(mx, piece_lse(i));
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+    float z = 0.f;
+    if (mx != -INFINITY)
+      for (int i = lane; i < n; i += 32) z += __expf(piece_lse(i) - mx);
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) z += __shfl_xor_sync(0xffffffffu, z, o);
+    if (lane == 0) {
+      mx_sh = mx;
+      inv_z_sh = z > 0.f ? 1.f / z : 0.f;
+      lse[out_row] = mx == -INFINITY ? -INFINITY : mx + logf(z);
     }
-    *reinterpret_cast<float4*>(dst + c4) = acc;
   }
-  if (lane == 0) lse[out_row] = mx + logf(z);
-#undef MLA_LIVE
+  __syncthreads();
+  const int c4 = 4 * threadIdx.x;
+  if (c4 >= d_c) return;
+  const float mx = mx_sh, inv_z = inv_z_sh;
+  float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+  if (mx != -INFINITY) {
+    for (int i = 0; i < n; i += 8) {
+      float w[8];
+      float4 x[8];
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        // a zero weight (nothing visible, or no slot written): row not read
+        w[u] = i + u < n ? __expf(piece_lse(i + u) - mx) * inv_z : 0.f;
+        const long long slot = (long long)(k0 + i + u) + v;
+        x[u] = w[u] != 0.f
+                   ? *reinterpret_cast<const float4*>(ws_o + (slot * rows_per_v + r) * d_c + c4)
+                   : make_float4(0.f, 0.f, 0.f, 0.f);
+      }
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        acc.x = fmaf(w[u], x[u].x, acc.x);
+        acc.y = fmaf(w[u], x[u].y, acc.y);
+        acc.z = fmaf(w[u], x[u].z, acc.z);
+        acc.w = fmaf(w[u], x[u].w, acc.w);
+      }
+    }
+  }
+  *reinterpret_cast<float4*>(o_lat + out_row * d_c + c4) = acc;
 }
 
-// A bounded wait that nothing completes: exercises the timeout path.
 // Merge of partial attention results over disjoint token sets (the parts):
 // one warp per row, parts with lse = -inf (nothing visible) contribute
 // nothing, a row with no visible token anywhere gets o = 0, lse = -inf.
