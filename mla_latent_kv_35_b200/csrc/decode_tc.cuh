@@ -265,7 +265,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(dtc::kThreads, 1)
 
   // Registers: the control warpgroup (producers, MMA) gives up most
   // of its share to the two softmax warpgroups.
-  static_assert(128 * kRegsControl + 256 * kRegsSoftmax <= 65536 &&
+  static_assert(128 * kRegsControl + 256 * kRegsSoftmax <= kRegsLaunch * kThreads &&
                     kRegsLaunch * kThreads <= 65536,
                 "register split exceeds the launch allocation");
   if (warp < kSoftmaxWarp0) {
@@ -409,8 +409,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(dtc::kThreads, 1)
       }
     } else if (warp == 1 && lane == 0 && rank == 0) {
       // =================  QK MMA issuer (leader CTA)  =================
-      // QK(j) writes S buffer j & 1 once the softmax of block j - 2 has read
-      // it (s_free).  The QK and PV streams are issued by two threads of
+      // QK(j) writes S buffer j & 1 once PV(j - 2) has consumed the P held
+      // there (s_free).  The QK and PV streams are issued by two threads of
       // different warps: the tensor pipe holds little more than the MMA it
       // runs, so the cycles one issuer spends between MMA groups (barrier
       // waits, commits, bookkeeping) are covered by the other's MMAs.
