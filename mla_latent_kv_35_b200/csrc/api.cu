@@ -539,9 +539,10 @@ static mla_status decode_impl(const mla_dims* dims, const void* qbuf, const void
 #undef MLA_SIMT_DECODE
     MLA_TRY(check_launch());
   }
-  dim3 cgrid(L.V, L.rows_per_v);
+  const int wpr = combine_warps_per_row(L.V, L.G);
+  dim3 cgrid(L.V, (L.rows_per_v * wpr + 7) / 8);
   combine_kernel<<<cgrid, kCombineThreads, 0, st>>>(ws_lse, ws_o, start, L.V, L.R, L.G,
-                                                    L.rows_per_v, S_q * H, dc, o_lat, lse);
+                                                    L.rows_per_v, S_q * H, dc, wpr, o_lat, lse);
   return check_launch();
 }
 
@@ -600,10 +601,11 @@ mla_status mla_decode_fp8(const mla_dims* dims, const void* qbuf, const void* po
                                  seq_lens, nullptr, B, S_q, dims->n_heads, dims->scale, L.G,
                                  start, ws_lse, ws_o, st));
   g_launches.fetch_add(1, std::memory_order_relaxed);
-  dim3 cgrid(L.V, L.rows_per_v);
+  const int wpr = combine_warps_per_row(L.V, L.G);
+  dim3 cgrid(L.V, (L.rows_per_v * wpr + 7) / 8);
   combine_kernel<<<cgrid, kCombineThreads, 0, st>>>(ws_lse, ws_o, start, L.V, L.R, L.G,
                                                     L.rows_per_v, S_q * dims->n_heads,
-                                                    dims->d_latent, o_lat, lse);
+                                                    dims->d_latent, wpr, o_lat, lse);
   return check_launch();
 }
 

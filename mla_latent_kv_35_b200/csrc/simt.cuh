@@ -274,82 +274,120 @@ __global__ void __launch_bounds__(256) decode_simt_kernel(
 // ---------------------------------------------------------------------------
 // Log-sum-exp combine of the pieces of every virtual sequence.
 //   o = sum_k w_k o_k / sum_k w_k, w_k = exp(lse_k - max lse), lse = max + ln sum w
-// Grid (V, rows_per_v), one CTA of 128 threads per row.  Warp 0 reduces the
-// pieces' LSEs of the row (lanes take pieces in parallel); then thread t
-// merges columns [4t, 4t + 4) (d_c <= 512, a multiple of 4) with eight
-// pieces' partial rows in flight at a time, so that a row merging many
-// pieces (a long sequence split over many workers) is not a chain of
-// dependent loads.  Virtual sequence v is row block v % R of sequence v / R:
+// Grid (V, ceil(rows_per_v * wpr / 8)), 8 warps per CTA and wpr warps per
+// row (1, 2, 4 or 8: more for rows that merge many pieces, a long sequence
+// split over many workers).  The lanes of each warp read the row's piece
+// LSEs 32 at a time and reduce them with shuffles; lane i keeps the weight
+// of piece i of each group of 32 and hands it out with a shuffle.  Warp u
+// of a row's wpr merges the pieces i with (i / 2) % wpr == u, two at a time,
+// each lane owning four float4 columns (d_c <= 512, a multiple of 4), so
+// every lane keeps eight loads in flight; the wpr partial sums meet in
+// shared memory.  Virtual sequence v is row block v % R of sequence v / R:
 // rows_per_v workspace rows, of which the ones past the sequence's rows_seq
 // query rows are padding and skipped.
 // ---------------------------------------------------------------------------
-constexpr int kCombineThreads = 128;
+constexpr int kCombineThreads = 256;
 
 __global__ void __launch_bounds__(kCombineThreads) combine_kernel(
     const float* ws_lse, const float* ws_o, const int32_t* start, int V, int R, int G,
-    int rows_per_v, int rows_seq, int d_c, float* o_lat, float* lse) {
-  __shared__ float mx_sh, inv_z_sh;
+    int rows_per_v, int rows_seq, int d_c, int wpr, float* o_lat, float* lse) {
+  __shared__ float4 part[7][128];   // partial sums of warps 1.. of a row group
   const int v = blockIdx.x;
-  const int r = blockIdx.y;
+  const int w = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int u = w % wpr;                               // this warp's share of the row
+  const int r = (blockIdx.y * 8 + w) / wpr;
   const int row_in_seq = (v % R) * rows_per_v + r;
-  if (row_in_seq >= rows_seq) return;
+  const bool live_row = r < rows_per_v && row_in_seq < rows_seq;
   const int total = start[V];
   const long long out_row = (long long)(v / R) * rows_seq + row_in_seq;
   const bool any = start[v + 1] > start[v];
   const int k0 = any ? worker_of(start[v], total, G) : 0;
-  const int n = any ? worker_of(start[v + 1] - 1, total, G) - k0 + 1 : 0;
+  const int n = (any && live_row) ? worker_of(start[v + 1] - 1, total, G) - k0 + 1 : 0;
   // lse of piece i of the row, -inf for a worker with an empty range (only
   // when G > total), which wrote no slot
   auto piece_lse = [&](int i) {
     const int k = k0 + i;
-    return worker_lo(k + 1, total, G) > worker_lo(k, total, G)
+    return i < n && worker_lo(k + 1, total, G) > worker_lo(k, total, G)
                ? ws_lse[((long long)k + v) * rows_per_v + r] : -INFINITY;
   };
-  if (threadIdx.x < 32) {
-    const int lane = threadIdx.x;
-    float mx = -INFINITY;
-    for (int i = lane; i < n; i += 32) mx = fmaxf(mx, piece_lse(i));
+  float mx = -INFINITY;
+  for (int i = lane; i < n; i += 32) mx = fmaxf(mx, piece_lse(i));
 #pragma unroll
-    for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
-    float z = 0.f;
-    if (mx != -INFINITY)
-      for (int i = lane; i < n; i += 32) z += __expf(piece_lse(i) - mx);
+  for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+  float z = 0.f;
+  if (mx != -INFINITY)
+    for (int i = lane; i < n; i += 32) z += __expf(piece_lse(i) - mx);
 #pragma unroll
-    for (int o = 16; o > 0; o >>= 1) z += __shfl_xor_sync(0xffffffffu, z, o);
-    if (lane == 0) {
-      mx_sh = mx;
-      inv_z_sh = z > 0.f ? 1.f / z : 0.f;
-      lse[out_row] = mx == -INFINITY ? -INFINITY : mx + logf(z);
-    }
-  }
-  __syncthreads();
-  const int c4 = 4 * threadIdx.x;
-  if (c4 >= d_c) return;
-  const float mx = mx_sh, inv_z = inv_z_sh;
-  float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+  for (int o = 16; o > 0; o >>= 1) z += __shfl_xor_sync(0xffffffffu, z, o);
+  if (live_row && u == 0 && lane == 0) lse[out_row] = mx == -INFINITY ? -INFINITY : mx + logf(z);
+  float4 acc[4];
+#pragma unroll
+  for (int q = 0; q < 4; ++q) acc[q] = make_float4(0.f, 0.f, 0.f, 0.f);
   if (mx != -INFINITY) {
-    for (int i = 0; i < n; i += 8) {
-      float w[8];
-      float4 x[8];
+    const float inv_z = 1.f / z;
+    for (int g = 0; g < n; g += 32) {
+      // lane i: weight of piece g + i (0 for a piece with nothing visible
+      // or no slot written: its row is not read)
+      const float w_mine = g + lane < n ? __expf(piece_lse(g + lane) - mx) * inv_z : 0.f;
+      const int cnt = min(32, n - g);
+      for (int i = 2 * u; i < cnt; i += 2 * wpr) {
+        const float w0 = __shfl_sync(0xffffffffu, w_mine, i);
+        const float w1 = __shfl_sync(0xffffffffu, w_mine, min(i + 1, 31));
+        const float wb = i + 1 < cnt ? w1 : 0.f;
+        const float* r0 = ws_o + (((long long)(k0 + g + i) + v) * rows_per_v + r) * d_c;
+        const float* r1 = r0 + (long long)rows_per_v * d_c;   // the next slot
+        float4 x0[4], x1[4];
 #pragma unroll
-      for (int u = 0; u < 8; ++u) {
-        // a zero weight (nothing visible, or no slot written): row not read
-        w[u] = i + u < n ? __expf(piece_lse(i + u) - mx) * inv_z : 0.f;
-        const long long slot = (long long)(k0 + i + u) + v;
-        x[u] = w[u] != 0.f
-                   ? *reinterpret_cast<const float4*>(ws_o + (slot * rows_per_v + r) * d_c + c4)
-                   : make_float4(0.f, 0.f, 0.f, 0.f);
-      }
+        for (int q = 0; q < 4; ++q) {
+          const int c4 = 4 * lane + 128 * q;
+          const bool in = c4 < d_c;
+          x0[q] = in && w0 != 0.f ? *reinterpret_cast<const float4*>(r0 + c4)
+                                  : make_float4(0.f, 0.f, 0.f, 0.f);
+          x1[q] = in && wb != 0.f ? *reinterpret_cast<const float4*>(r1 + c4)
+                                  : make_float4(0.f, 0.f, 0.f, 0.f);
+        }
 #pragma unroll
-      for (int u = 0; u < 8; ++u) {
-        acc.x = fmaf(w[u], x[u].x, acc.x);
-        acc.y = fmaf(w[u], x[u].y, acc.y);
-        acc.z = fmaf(w[u], x[u].z, acc.z);
-        acc.w = fmaf(w[u], x[u].w, acc.w);
+        for (int q = 0; q < 4; ++q) {
+          acc[q].x = fmaf(w0, x0[q].x, fmaf(wb, x1[q].x, acc[q].x));
+          acc[q].y = fmaf(w0, x0[q].y, fmaf(wb, x1[q].y, acc[q].y));
+          acc[q].z = fmaf(w0, x0[q].z, fmaf(wb, x1[q].z, acc[q].z));
+          acc[q].w = fmaf(w0, x0[q].w, fmaf(wb, x1[q].w, acc[q].w));
+        }
       }
     }
   }
-  *reinterpret_cast<float4*>(o_lat + out_row * d_c + c4) = acc;
+  if (wpr > 1) {
+    // warps 1.. of each row group leave their sums; warp 0 of the group adds
+    if (u != 0) {
+#pragma unroll
+      for (int q = 0; q < 4; ++q) part[w - 1][32 * q + lane] = acc[q];
+    }
+    __syncthreads();
+    if (u == 0) {
+      for (int t = 1; t < wpr; ++t)
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          const float4 y = part[w + t - 1][32 * q + lane];
+          acc[q].x += y.x; acc[q].y += y.y; acc[q].z += y.z; acc[q].w += y.w;
+        }
+    }
+  }
+  if (!live_row || u != 0) return;
+  float* dst = o_lat + out_row * d_c;
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    const int c4 = 4 * lane + 128 * q;
+    if (c4 < d_c) *reinterpret_cast<float4*>(dst + c4) = acc[q];
+  }
+}
+
+// Warps per row of combine_kernel for a workload: enough that a row's
+// pieces spread to about eight per warp.
+inline int combine_warps_per_row(int V, int G) {
+  const int pieces = (G + V - 1) / V + 1;   // pieces of a virtual sequence, about
+  int wpr = 1;
+  while (wpr < 8 && pieces > 8 * wpr) wpr *= 2;
+  return wpr;
 }
 
 // Merge of partial attention results over disjoint token sets (the parts):
