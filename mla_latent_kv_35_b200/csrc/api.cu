@@ -126,16 +126,24 @@ TcGemmPlan plan_tc_gemm(int M, int N, int K, int batch, bool allow_split) {
   p.n_tile = n16 < 256 ? n16 : 256;
   p.n_tiles = (N + p.n_tile - 1) / p.n_tile;
   const size_t stage_bytes = (size_t)kGemmBM * kGemmBK * 2 + (size_t)p.n_tile * kGemmBK * 2;
-  int st = (int)((96 * 1024) / stage_bytes);
-  p.stages = st < 2 ? 2 : (st > 8 ? 8 : st);
   const int k_chunks = (K + kGemmBK - 1) / kGemmBK;
   p.splits = 1;
+  const long long ctas = (long long)((M + kGemmBM - 1) / kGemmBM) * p.n_tiles * batch;
   if (allow_split) {
-    const long long ctas = (long long)((M + kGemmBM - 1) / kGemmBM) * p.n_tiles * batch;
     const long long target = 2LL * sm_count();
     while (ctas * p.splits < target && k_chunks / (p.splits + 1) >= 4) ++p.splits;
   }
   p.k_chunks_per_split = (k_chunks + p.splits - 1) / p.splits;
+  // Ring depth: the weights stream from HBM, so a CTA keeps as many of its
+  // k-chunks in flight as shared memory allows: up to ~200 KB when the grid
+  // has at most one CTA per SM, ~96 KB (two CTAs per SM) otherwise, and
+  // never more stages than the CTA has chunks (a short K leaves room for
+  // more CTAs per SM instead).
+  const size_t budget = ctas * p.splits <= sm_count() ? 200 * 1024 : 96 * 1024;
+  int st = (int)(budget / stage_bytes);
+  st = st < 2 ? 2 : (st > 8 ? 8 : st);
+  if (st > p.k_chunks_per_split) st = p.k_chunks_per_split < 2 ? 2 : p.k_chunks_per_split;
+  p.stages = st;
   p.smem = stage_bytes * p.stages + 1024;
   return p;
 }
