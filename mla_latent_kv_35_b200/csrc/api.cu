@@ -471,7 +471,7 @@ mla_status mla_pre_attention(const mla_dims* dims, void* y, int y_stride_tok, co
   aux.pool = static_cast<uint16_t*>(pool);
   aux.n_pages = n_pages; aux.page_size = dims->page_size;
   aux.base = (double)dims->rope_base;
-  aux.n_rope = (long long)T * (dr / 2);
+  aux.n_rope = (long long)T * (dr / 2) * ((H + kRopeHeadsPerItem - 1) / kRopeHeadsPerItem);
   aux.n_items = aux.n_rope + (long long)T * (dc / 8);
   // A1 on the GEMM CTAs, A2 and A3 on extra CTAs of the same launch
   return launch_tc_gemm(w_uk, true, (long long)dn * dc, y, y_stride_tok, dqk, dc, T, dn, H, qbuf,

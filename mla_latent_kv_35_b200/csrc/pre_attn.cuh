@@ -73,14 +73,17 @@ __device__ __forceinline__ E* append_row(const int32_t* batch_idx, const int32_t
 // mla_project writes them for W_A0 = [W_Q; W_DKV; W_KR]:
 //   y[t] = [q_1 .. q_H | c | k_rope_pre],  q_i = [q_nope (d_n) ; q_rope (d_r)].
 // Work items, grid-strided:
-//   [0, n_rope)        (token t, pair k): one angle, applied to pair k of every
-//                      head's q_rope (-> qbuf[t][head][d_c + 2k ..]) and of
-//                      k_rope (-> the pool row and back into y, as the
-//                      standalone in-place RoPE of k does)
+//   [0, n_rope)        (token t, head group g, pair k): one angle, applied to
+//                      pair k of the q_rope of heads [8g, 8g + 8)
+//                      (-> qbuf[t][head][d_c + 2k ..]); group 0 also turns
+//                      pair k of k_rope (-> the pool row and back into y, as
+//                      the standalone in-place RoPE of k does)
 //   [n_rope, n_items)  (token t, 16-byte piece u) of the latent: copied to the
 //                      pool row
 // Consecutive items of a warp take consecutive k (or u), so every access of
-// the warp is one contiguous run.
+// the warp is one contiguous run; a thread touches eight heads, not all of
+// them, so the RoPE of many heads spreads over many threads.
+constexpr int kRopeHeadsPerItem = 8;
 struct PreAttnAux {
   __nv_bfloat16* y;
   long long ys_tok;       // elements per token row of y
@@ -103,25 +106,35 @@ __device__ __forceinline__ void pre_attention_aux(const PreAttnAux& a, long long
   const int dqk = a.d_nope + a.d_rope;
   const int D = a.d_latent + a.d_rope;
   const int pieces = a.d_latent / 8;
+  const int groups = (a.H + kRopeHeadsPerItem - 1) / kRopeHeadsPerItem;
   for (long long i = i0; i < a.n_items; i += stride) {
     if (i < a.n_rope) {
-      const int t = (int)(i / half);
-      const int k = (int)(i % half);
+      const int t = (int)(i / ((long long)half * groups));
+      const int rem = (int)(i % ((long long)half * groups));
+      const int g = rem / half, k = rem % half;
       const int p = a.pos[t];
       float c, sn;
       rope_cos_sin(k, p, a.d_rope, a.base, c, sn);
       const __nv_bfloat16* xq = a.y + t * a.ys_tok + a.d_nope + 2 * k;
       __nv_bfloat16* yq = a.qbuf + (long long)t * a.H * D + a.d_latent + 2 * k;
-#pragma unroll 8
-      for (int h = 0; h < a.H; ++h) {
-        const __nv_bfloat162 v = *reinterpret_cast<const __nv_bfloat162*>(xq + (long long)h * dqk);
+      const int h0 = kRopeHeadsPerItem * g;
+      const int h1 = min(a.H, h0 + kRopeHeadsPerItem);
+      __nv_bfloat162 v[kRopeHeadsPerItem];
+#pragma unroll
+      for (int u = 0; u < kRopeHeadsPerItem; ++u)
+        if (h0 + u < h1)
+          v[u] = *reinterpret_cast<const __nv_bfloat162*>(xq + (long long)(h0 + u) * dqk);
+#pragma unroll
+      for (int u = 0; u < kRopeHeadsPerItem; ++u) {
+        if (h0 + u >= h1) break;
         float y0, y1;
-        rope_rotate(to_f32(v.x), to_f32(v.y), c, sn, y0, y1);
+        rope_rotate(to_f32(v[u].x), to_f32(v[u].y), c, sn, y0, y1);
         __nv_bfloat162 o;
         o.x = from_f32<__nv_bfloat16>(y0);
         o.y = from_f32<__nv_bfloat16>(y1);
-        *reinterpret_cast<__nv_bfloat162*>(yq + (long long)h * D) = o;
+        *reinterpret_cast<__nv_bfloat162*>(yq + (long long)(h0 + u) * D) = o;
       }
+      if (g != 0) continue;
       __nv_bfloat16* kr = a.y + t * a.ys_tok + a.off_c + a.d_latent + 2 * k;
       float y0, y1;
       rope_rotate(to_f32(kr[0]), to_f32(kr[1]), c, sn, y0, y1);
