@@ -130,8 +130,10 @@ TcGemmPlan plan_tc_gemm(int M, int N, int K, int batch, bool allow_split) {
   p.splits = 1;
   const long long ctas = (long long)((M + kGemmBM - 1) / kGemmBM) * p.n_tiles * batch;
   if (allow_split) {
+    // as many splits as keep the grid within two CTAs per SM (one wave: a
+    // partial second wave would double the time of its SMs)
     const long long target = 2LL * sm_count();
-    while (ctas * p.splits < target && k_chunks / (p.splits + 1) >= 4) ++p.splits;
+    while (ctas * (p.splits + 1) <= target && k_chunks / (p.splits + 1) >= 4) ++p.splits;
   }
   p.k_chunks_per_split = (k_chunks + p.splits - 1) / p.splits;
   // Ring depth: the weights stream from HBM, so a CTA keeps as many of its
