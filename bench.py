@@ -48,14 +48,19 @@ def _peaks():
         return 6650.0, 1590.0, "fallback"
 
 
-def _workload_bytes(w):
-    """Algorithmic bytes and FLOPs of the decode call (A4+A5) per step."""
+FP8_ROW_BYTES = 656   # E4M3 latent, f16 RoPE key, fp32 scale, padding
+
+
+def _workload_bytes(w, cache_kind="bf16"):
+    """Algorithmic bytes and FLOPs of the decode call (A4+A5) per step.  The
+    cache is read once: D bf16 numbers per token, or one 656-byte row of the
+    8-bit cache."""
     D = w.D
     vis = []
     for L in w.ctx:
         for j in range(w.S_q):
             vis.append(L - w.S_q + j + 1)
-    cache = sum(w.ctx) * D * 2
+    cache = sum(w.ctx) * (FP8_ROW_BYTES if cache_kind == "fp8" else D * 2)
     q = w.T * w.H * D * 2
     out = w.T * w.H * (w.d_latent + 1) * 4
     flops = 2 * w.H * (D + w.d_latent) * sum(vis)
@@ -165,18 +170,18 @@ L2_BYTES = 126 * 1024 * 1024
 L2_FLUSH_BYTES = 2 * L2_BYTES
 
 
-def flush_needed(w):
+def flush_needed(w, cache_kind="bf16"):
     """The decode call reads only the cache (plus small q and outputs): when
     the cache is under twice the L2 size, repeated calls would be served
     partly from L2, so the bench flushes L2 between timed calls."""
-    _, _, cache_bytes = _workload_bytes(w)
+    _, _, cache_bytes = _workload_bytes(w, cache_kind)
     return cache_bytes < 2 * L2_BYTES
 
 
-def run_config(w, workload_name, world, flush=None):
+def run_config(w, workload_name, world, flush=None, cache_kind="bf16"):
     """The JSON line's `config`, shared by both arms."""
-    _, _, cache_bytes = _workload_bytes(w)
-    flush = flush_needed(w) if flush is None else flush
+    _, _, cache_bytes = _workload_bytes(w, cache_kind)
+    flush = flush_needed(w, cache_kind) if flush is None else flush
     l2 = ("L2 flushed (%d MB write) before every timed call; cache %.3f GB"
           % (L2_FLUSH_BYTES >> 20, cache_bytes / 1e9) if flush else
           "inputs larger than L2 (cache %.2f GB), no flush" % (cache_bytes / 1e9))
@@ -184,6 +189,8 @@ def run_config(w, workload_name, world, flush=None):
             "heads": w.H, "context": w.ctx[0] if len(set(w.ctx)) == 1 else "ragged",
             "S_q": w.S_q, "latent": w.d_latent, "rope": w.d_rope, "page": w.page_size,
             "d_model": w.d_model,
+            "cache": ("8-bit latent cache: E4M3 latent, f16 RoPE key, fp32 row scale, 656 B "
+                      "per token" if cache_kind == "fp8" else "bf16, 1152 B per token"),
             "l2": l2,
             "parallelism": (f"dp{world}: independent sequence shards, no collective"
                             if world > 1 else "single GPU")}
@@ -255,7 +262,7 @@ def run_reference(args, w):
         "warmup": args.warmup, "ms_per_step": 1000.0 * w.T / value,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
         "data": "synthetic",
-        "config": run_config(w, w.name, args.gpus),
+        "config": run_config(w, w.name, args.gpus, cache_kind=args.cache),
         "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": cores, "kind": "oracle",
                          "sample": sample},
         "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0,
@@ -306,8 +313,14 @@ def run_gpu(args, w):
         host = build_pool_host_drawn(w, table, n_pages)
     pool = pool_to_device(host, w.dtype, dev)
     del host
+    if args.cache == "fp8":
+        # the 8-bit cache: the same rows, quantized on the GPU
+        pool8 = torch.empty((n_pages, w.page_size, FP8_ROW_BYTES), dtype=torch.uint8, device=dev)
+        B.mla_cache_quantize_fp8(d, pool, pool8, n_pages)
+        del pool
+        pool = pool8
     layer.set_cache(pool, torch.from_numpy(table).to(dev),
-                    torch.tensor(w.ctx, dtype=torch.int32, device=dev))
+                    torch.tensor(w.ctx, dtype=torch.int32, device=dev), kind=args.cache)
     if w.prior_from_h:
         layer.prefill_from_hidden([wl.draw_h_ctx(w, b) for b in range(w.B)])
     h_np = wl.draw_h_new(w).reshape(w.T, w.d_model)
@@ -323,10 +336,12 @@ def run_gpu(args, w):
     # the decode call alone, with events on the launching stream
     bf = layer.buffers(w.B, w.S_q)
 
+    decode_call = B.mla_decode_fp8 if args.cache == "fp8" else B.mla_decode
+
     def decode_only():
-        B.mla_decode(d, bf["qbuf"], layer.pool, layer.n_pages, layer.page_table,
-                     layer.max_pages, layer.seq_lens, w.B, w.S_q, 0, bf["ws"], bf["o_lat"],
-                     bf["lse"])
+        decode_call(d, bf["qbuf"], layer.pool, layer.n_pages, layer.page_table,
+                    layer.max_pages, layer.seq_lens, w.B, w.S_q, 0, bf["ws"], bf["o_lat"],
+                    bf["lse"])
 
     for _ in range(args.warmup):
         eager_step()
@@ -346,7 +361,7 @@ def run_gpu(args, w):
 
     # L2 flush between timed calls when the decode's inputs fit in L2: a
     # write of twice the L2 size, outside every timed region
-    flush = args.flush_l2 == "on" or (args.flush_l2 == "auto" and flush_needed(w))
+    flush = args.flush_l2 == "on" or (args.flush_l2 == "auto" and flush_needed(w, args.cache))
     flush_buf = torch.empty((L2_FLUSH_BYTES // 4,), dtype=torch.int32, device=dev) \
         if flush else None
 
@@ -435,11 +450,12 @@ def run_gpu(args, w):
     t_step, t_dec, t_e2e, t_eager = max_over_ranks([t_step, t_dec, t_e2e, t_eager], dev)
 
     hbm_peak, tf_peak, peak_kind = _peaks()
-    alg_bytes, flops, cache_bytes = _workload_bytes(w)
+    alg_bytes, flops, cache_bytes = _workload_bytes(w, args.cache)
     achieved = alg_bytes / (t_dec * 1e-3) / 1e9
     roof_t = max(alg_bytes / (hbm_peak * 1e9), flops / (tf_peak * 1e12))
     csrc = os.path.join(ROOT, "mla_latent_kv_35_b200", "csrc")
-    traffic = _traffic_for([os.path.join(csrc, "decode_tc.cuh")])
+    traffic = _traffic_for([os.path.join(csrc, "decode_fp8.cuh" if args.cache == "fp8"
+                                         else "decode_tc.cuh")])
     line = {
         "metric": "MLA decode tokens/s (one attention layer, whole step A0-A6)",
         "value": whole_job_rate(w.T, world, t_step),
@@ -451,14 +467,17 @@ def run_gpu(args, w):
         "higher_is_better": True,
         "scaling": "weak",
         "vs_baseline": None,
-        "dtype": "bf16" if w.dtype == "bf16" else "f32",
+        "dtype": ("bf16 (E4M3 cache, f16 decode MMAs)" if args.cache == "fp8" else
+                  "bf16" if w.dtype == "bf16" else "f32"),
         "data": "synthetic",
-        "config": run_config(w, workload_name, world, flush),
+        "config": run_config(w, workload_name, world, flush, args.cache),
         "decode": {"ms": t_dec, "tokens_per_s": whole_job_rate(w.T, world, t_dec),
                    "cache_gb_per_s": cache_bytes / (t_dec * 1e-3) / 1e9,
                    "tflops": flops / (t_dec * 1e-3) / 1e12,
                    "roofline_ms": roof_t * 1e3, "frac_of_roofline": roof_t / (t_dec * 1e-3)},
-        "roofline": {"kernel": "mla_decode (decode_tc_kernel + combine)", "bound": "hbm",
+        "roofline": {"kernel": ("mla_decode_fp8 (decode_fp8_kernel + combine)"
+                                if args.cache == "fp8" else
+                                "mla_decode (decode_tc_kernel + combine)"), "bound": "hbm",
                      "achieved": achieved, "peak": hbm_peak, "unit": "GB/s",
                      "frac": achieved / hbm_peak, "peak_source": peak_kind,
                      "alg_bytes_per_launch": alg_bytes, "traffic": traffic},
@@ -497,6 +516,8 @@ def main():
                          "under twice the L2 size)")
     ap.add_argument("--batch", type=int, default=0,
                     help="use only the first N sequences of the workload")
+    ap.add_argument("--cache", default="bf16", choices=["bf16", "fp8"],
+                    help="latent cache format (fp8: the 8-bit cache, bf16 workloads only)")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3

@@ -118,25 +118,30 @@ __device__ __forceinline__ void st_shared_v4(uint32_t addr, uint32_t a, uint32_t
 // become zeros.
 __device__ __forceinline__ void convert_page_cols(const uint8_t* page, int col_byte0, int valid,
                                                   uint32_t dst, uint32_t chunk_stride, int lane) {
+  // All sixteen 16-byte loads of a lane are issued before the first
+  // conversion: the rows come from HBM or L2, and a chain of dependent
+  // rounds would leave the stage waiting several latencies.
   const int u = lane & 7, tq = lane >> 3;
   const int cc = u >> 2, unit = 2 * (u & 3);
-#pragma unroll 4
-  for (int t0 = 0; t0 < dfp::kPage; t0 += 4) {
-    const int t = t0 + tq;
+  uint4 raw[16];
+#pragma unroll
+  for (int i = 0; i < 16; ++i) {
+    const int t = 4 * i + tq;
+    raw[i] = t < valid
+                 ? __ldg(reinterpret_cast<const uint4*>(page + (size_t)t * dfp::kRow + col_byte0 +
+                                                        16 * u))
+                 : make_uint4(0u, 0u, 0u, 0u);
+  }
+#pragma unroll
+  for (int i = 0; i < 16; ++i) {
+    const int t = 4 * i + tq;
     const uint32_t row = dst + cc * chunk_stride + t * 128;
     const uint32_t a0 = row + (((unit) ^ (t & 7)) << 4);
     const uint32_t a1 = row + (((unit + 1) ^ (t & 7)) << 4);
-    if (t < valid) {
-      const uint8_t* src = page + (size_t)t * dfp::kRow;
-      const uint4 raw = __ldg(reinterpret_cast<const uint4*>(src + col_byte0 + 16 * u));
-      uint32_t o[8];
-      e4m3x16_to_f16(raw, o);
-      st_shared_v4(a0, o[0], o[1], o[2], o[3]);
-      st_shared_v4(a1, o[4], o[5], o[6], o[7]);
-    } else {
-      st_shared_v4(a0, 0u, 0u, 0u, 0u);
-      st_shared_v4(a1, 0u, 0u, 0u, 0u);
-    }
+    uint32_t o[8];
+    e4m3x16_to_f16(raw[i], o);   // zero bytes convert to +0
+    st_shared_v4(a0, o[0], o[1], o[2], o[3]);
+    st_shared_v4(a1, o[4], o[5], o[6], o[7]);
   }
 }
 
@@ -146,17 +151,18 @@ __device__ __forceinline__ void convert_page_cols(const uint8_t* page, int col_b
 __device__ __forceinline__ void copy_page_rope(const uint8_t* page, int valid, uint32_t dst,
                                                int lane) {
   const int u = lane & 7, tq = lane >> 3;
-#pragma unroll 4
-  for (int t0 = 0; t0 < dfp::kPage; t0 += 4) {
-    const int t = t0 + tq;
-    const uint32_t a = dst + t * 128 + ((u ^ (t & 7)) << 4);
-    if (t < valid) {
-      const uint4 v =
-          __ldg(reinterpret_cast<const uint4*>(page + (size_t)t * dfp::kRow + fp8::kOffRope + 16 * u));
-      st_shared_v4(a, v.x, v.y, v.z, v.w);
-    } else {
-      st_shared_v4(a, 0u, 0u, 0u, 0u);
-    }
+  uint4 v[16];
+#pragma unroll
+  for (int i = 0; i < 16; ++i) {
+    const int t = 4 * i + tq;
+    v[i] = t < valid ? __ldg(reinterpret_cast<const uint4*>(page + (size_t)t * dfp::kRow +
+                                                            fp8::kOffRope + 16 * u))
+                     : make_uint4(0u, 0u, 0u, 0u);
+  }
+#pragma unroll
+  for (int i = 0; i < 16; ++i) {
+    const int t = 4 * i + tq;
+    st_shared_v4(dst + t * 128 + ((u ^ (t & 7)) << 4), v[i].x, v[i].y, v[i].z, v[i].w);
   }
 }
 

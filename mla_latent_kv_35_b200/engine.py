@@ -44,13 +44,24 @@ class MLADecodeLayer:
         self.W_O = _to_dev(weights["W_O"], dt, self.device)
         self._bufs = {}
         self.pool = None
+        self.cache_kind = "bf16"
 
     # ------------------------------------------------------------------
     # cache
     # ------------------------------------------------------------------
-    def set_cache(self, pool, page_table, seq_lens):
+    def set_cache(self, pool, page_table, seq_lens, kind: str = "bf16"):
         """pool [n_pages, page_size, D] (dims dtype), page_table int32
-        [B, max_pages], seq_lens int32 [B] (context after this step's append)."""
+        [B, max_pages], seq_lens int32 [B] (context after this step's append).
+
+        kind "fp8": pool is the 8-bit latent cache, uint8 [n_pages,
+        page_size, 656] (E4M3 latent, half-precision RoPE key, fp32 row
+        scale; mla_cache_quantize_fp8 converts a bf16 pool): steps append by
+        quantizing and attend with mla_decode_fp8."""
+        if kind not in ("bf16", "fp8"):
+            raise ValueError(f"cache kind {kind!r}")
+        if kind == "fp8" and self.dims.dtype != "bf16":
+            raise ValueError("the 8-bit cache is for bf16 layers")
+        self.cache_kind = kind
         self.pool = pool
         self.page_table = page_table
         self.seq_lens = seq_lens
@@ -74,8 +85,9 @@ class MLADecodeLayer:
             kr = y[:, d.d_latent:]
             _b.mla_rope(d, kr, self.D, 0, 1, kr, self.D, 0, pos, n)
             bi = torch.full((n,), b, dtype=torch.int32, device=self.device)
-            _b.mla_cache_append(d, y, self.D, kr, self.D, bi, pos, self.page_table,
-                                self.max_pages, self.pool, self.n_pages, n)
+            append = _b.mla_cache_append_fp8 if self.cache_kind == "fp8" else _b.mla_cache_append
+            append(d, y, self.D, kr, self.D, bi, pos, self.page_table, self.max_pages, self.pool,
+                   self.n_pages, n)
 
     # ------------------------------------------------------------------
     # step buffers
@@ -83,12 +95,13 @@ class MLADecodeLayer:
     def buffers(self, B: int, S_q: int, num_workers: int = 0, slot: int = 0):
         """Device buffers of one step (slot: an independent second set, for
         steps that overlap in DecodePipeline)."""
-        key = (B, S_q, num_workers, slot)
+        key = (B, S_q, num_workers, slot, self.cache_kind)
         if key not in self._bufs:
             d = self.dims
             T = B * S_q
             dev, dt = self.device, d.torch_dtype
-            ws = _b.mla_decode_workspace_size(d, B, S_q, num_workers)
+            ws = (_b.mla_decode_fp8_workspace_size if self.cache_kind == "fp8"
+                  else _b.mla_decode_workspace_size)(d, B, S_q, num_workers)
             sc = _b.mla_out_proj_scratch_size(d, T)
             self._bufs[key] = dict(
                 y=torch.empty((T, self.Y), dtype=dt, device=dev),
@@ -110,7 +123,9 @@ class MLADecodeLayer:
         T = B*S_q tokens b-major.  Returns the dict of step buffers.
 
         fused: A1-A3 through mla_pre_attention (one launch for bf16) instead
-        of the four separate calls; both write the same bits."""
+        of the four separate calls; both write the same bits.  An 8-bit
+        cache always takes the separate calls, its append quantizing the new
+        rows (mla_cache_append_fp8)."""
         d = self.dims
         H, dn, dc, dr = d.n_heads, d.d_nope, d.d_latent, d.d_rope
         T = B * S_q
@@ -118,7 +133,8 @@ class MLADecodeLayer:
         y, qbuf = bf["y"], bf["qbuf"]
         Y, D, dqk = self.Y, self.D, self.dqk
         _b.mla_project(d, h, self.W_A0, y, T, d.d_model, Y)                        # A0
-        if fused:
+        fp8 = self.cache_kind == "fp8"
+        if fused and not fp8:
             _b.mla_pre_attention(d, y, Y, self.W_UK, qbuf, batch_idx, pos,          # A1-A3
                                  self.page_table, self.max_pages, self.pool, self.n_pages, T)
         else:
@@ -126,12 +142,14 @@ class MLADecodeLayer:
             _b.mla_rope(d, y[:, dn:], Y, dqk, H, qbuf[:, :, dc:], H * D, D, pos, T)  # A2 q
             kr = y[:, off_c + dc:]
             _b.mla_rope(d, kr, Y, 0, 1, kr, Y, 0, pos, T)                             # A2 k
-            _b.mla_cache_append(d, y[:, off_c:], Y, kr, Y, batch_idx, pos,            # A3
-                                self.page_table, self.max_pages, self.pool, self.n_pages, T)
+            append = _b.mla_cache_append_fp8 if fp8 else _b.mla_cache_append
+            append(d, y[:, off_c:], Y, kr, Y, batch_idx, pos,                         # A3
+                   self.page_table, self.max_pages, self.pool, self.n_pages, T)
             _b.mla_absorb_q(d, y, Y, self.W_UK, qbuf, T)                               # A1
-        _b.mla_decode(d, qbuf, self.pool, self.n_pages, self.page_table,            # A4+A5
-                      self.max_pages, self.seq_lens, B, S_q, num_workers, bf["ws"],
-                      bf["o_lat"], bf["lse"])
+        decode = _b.mla_decode_fp8 if fp8 else _b.mla_decode
+        decode(d, qbuf, self.pool, self.n_pages, self.page_table,                     # A4+A5
+               self.max_pages, self.seq_lens, B, S_q, num_workers, bf["ws"],
+               bf["o_lat"], bf["lse"])
         _b.mla_out_proj(d, bf["o_lat"], self.W_UV, self.W_O, bf["scratch"],         # A6
                         bf["out"], T)
         return bf

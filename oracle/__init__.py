@@ -22,4 +22,6 @@ from .mla_oracle import (  # noqa: F401
     mla_cache_bytes,
     cache_elems_per_token,
     gqa_equivalent_groups,
+    quantize_latent_fp8,
+    dequantize_fp8,
 )

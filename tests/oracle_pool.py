@@ -24,14 +24,18 @@ def _task(args):
     """Oracle attention of one sequence for a range of heads.
 
     args = (workload, b, heads, q_roped [S_q, H', d_n + d_r], c_new
-    [S_q, d_c], kr_new [S_q, d_r], W_UK [H', d_n, d_c], W_UV [H', d_v, d_c]);
-    the cache is sequence b's drawn prior followed by its new tokens.
+    [S_q, d_c], kr_new [S_q, d_r], W_UK [H', d_n, d_c], W_UV [H', d_v, d_c],
+    cache); the cache is sequence b's drawn prior followed by its new tokens,
+    for cache "fp8" quantized to the 8-bit rows and read back
+    (oracle.quantize_latent_fp8 / dequantize_fp8).
     Returns (b, heads, o_lat [S_q, H', d_c], lse [S_q, H'], o [S_q, H', d_v]).
     """
-    w, b, heads, q_roped, c_new, kr_new, W_UK, W_UV = args
+    w, b, heads, q_roped, c_new, kr_new, W_UK, W_UV, cache = args
     c, kr = wl.draw_prior(w, b)
     C = np.concatenate([c.astype(np.float64), c_new], 0)
     KR = np.concatenate([kr.astype(np.float64), kr_new], 0)
+    if cache == "fp8":
+        C, KR = oracle.dequantize_fp8(*oracle.quantize_latent_fp8(C, KR))
     r = oracle.attention_absorbed(q_roped, C, KR, W_UK, W_UV, w.scale)
     return b, heads, r["o_lat"], r["lse"], r["o"]
 
@@ -40,7 +44,7 @@ def n_procs() -> int:
     return max(1, min(16, len(os.sched_getaffinity(0)) - 1))
 
 
-def workload_reference(w, W, h, seqs, head_chunk=32):
+def workload_reference(w, W, h, seqs, head_chunk=32, cache="bf16"):
     """Oracle o_lat, lse and out of sequences `seqs` of workload w, all heads.
 
     W: the workload's weights (workloads.draw_weights), h: its new hidden
@@ -69,7 +73,7 @@ def workload_reference(w, W, h, seqs, head_chunk=32):
         for h0 in range(0, w.H, head_chunk):
             hs = list(range(h0, min(w.H, h0 + head_chunk)))
             tasks.append((w, b, hs, q_roped[:, hs], per[b]["c_new"], per[b]["kr_new"],
-                          np.asarray(W["W_UK"])[hs], np.asarray(W["W_UV"])[hs]))
+                          np.asarray(W["W_UK"])[hs], np.asarray(W["W_UV"])[hs], cache))
     ctx = mp.get_context("spawn")
     with ctx.Pool(n_procs()) as pool:
         for b, hs, o_lat, lse, o in pool.imap_unordered(_task, tasks):

@@ -26,7 +26,7 @@ from gpu_util import (DEV, check, check_stored_bf16, ensure_lib, fp32_accumulati
 gpu = pytest.mark.gpu
 
 
-def _setup(w):
+def _setup(w, cache="bf16"):
     ensure_lib()
     W = wl.draw_weights(w)
     d = MLADims.of(w)
@@ -42,8 +42,14 @@ def _setup(w):
         prior = [np.concatenate(wl.draw_prior(w, b), 1) for b in range(w.B)]
     pool = pool_to_device(build_pool_host(w, table, n_pages, prior), w.dtype, DEV)
     del prior
+    if cache == "fp8":
+        pool8 = torch.empty((n_pages, w.page_size, B.FP8_ROW_BYTES), dtype=torch.uint8,
+                            device=DEV)
+        B.mla_cache_quantize_fp8(d, pool, pool8, n_pages)
+        del pool
+        pool = pool8
     layer.set_cache(pool, torch.from_numpy(table).to(DEV),
-                    torch.tensor(w.ctx, dtype=torch.int32, device=DEV))
+                    torch.tensor(w.ctx, dtype=torch.int32, device=DEV), kind=cache)
     h_ctx = None
     if w.prior_from_h:
         h_ctx = [wl.draw_h_ctx(w, b) for b in range(w.B)]
@@ -173,3 +179,54 @@ def test_batch128_full_path():
 def test_long_context_full_path(name):
     w = wl.workload(name)
     _check_bf16_workload(name, sample=range(w.B), nonabs_sample=[0], nonabs_heads=(64,))
+
+
+def _fp8_row_values(raw):
+    """(latent, RoPE key) numbers of 656-byte rows of the 8-bit cache, from
+    the bit layout: E4M3 (sign, 4 exponent bits with bias 7, 3 mantissa bits)
+    times the fp32 row scale, and the half-precision key times the scale."""
+    raw = np.asarray(raw, dtype=np.uint8)
+    b = raw[..., :512].astype(np.int64)
+    e, m = (b >> 3) & 0xF, b & 0x7
+    c8 = np.where(b & 0x80, -1.0, 1.0) * np.where(e == 0, m / 8.0 * 2.0 ** -6,
+                                                  (1 + m / 8.0) * 2.0 ** (e - 7.0))
+    kr = np.ascontiguousarray(raw[..., 512:640]).view(np.float16).astype(np.float64)
+    s = np.ascontiguousarray(raw[..., 640:644]).view(np.float32)[..., 0].astype(np.float64)
+    return c8 * s[..., None], kr * s[..., None]
+
+
+@gpu
+def test_dsv2_full_path_fp8_cache():
+    """The whole step over the 8-bit latent cache (bf16 workload dsv2): the
+    prior rows quantized by the library (byte-exact against the oracle's
+    quantizer in test_gpu_fp8.py), the new rows quantized by the append.
+    Reference: the oracle over its own quantization of the same cache, prior
+    and new rows."""
+    name = "dsv2"
+    w = wl.workload(name)
+    W, layer, bf, h, _, table = _setup(w, cache="fp8")
+    o_lat = to_np(bf["o_lat"]).reshape(w.B, w.S_q, w.H, w.d_latent)
+    lse = to_np(bf["lse"]).reshape(w.B, w.S_q, w.H)
+    out = to_np(bf["out"]).reshape(w.B, w.S_q, w.d_model)
+    sample = [0, 5, 10, 15]
+    new_rows = {}
+    for b in sample:
+        L = w.ctx[b]
+        new_rows[b] = [layer.pool[int(table[b, p // 64]), p % 64].cpu().numpy()
+                       for p in range(L - w.S_q, L)]
+    del layer, bf
+    torch.cuda.empty_cache()
+    ref = oracle_pool.workload_reference(w, W, h, sample, cache="fp8")
+    for b in sample:
+        r = ref[b]
+        check(o_lat[b], r["o_lat"], "bf16", f"{name} fp8 b={b} o_lat (all heads)")
+        check(lse[b], r["lse"], "bf16", f"{name} fp8 b={b} lse")
+        check(out[b], r["out"], "bf16", f"{name} fp8 b={b} out")
+        # the appended rows: the new tokens' latent and rotated RoPE key, to
+        # the precision of the 8-bit format (E4M3: 2^-4 relative to the row
+        # scale's range, the f16 key 2^-11), over the bf16-rounded inputs
+        for j, row in enumerate(new_rows[b]):
+            c, kr = _fp8_row_values(row)
+            c_ref, kr_ref = r["c_new"][j], r["kr_new"][j]
+            assert np.abs(c - c_ref).max() <= 2.0 ** -3 * np.abs(c_ref).max() + 1e-30, "A3 c8"
+            assert np.abs(kr - kr_ref).max() <= 2.0 ** -6 * np.abs(kr_ref).max() + 1e-30, "A3 kr16"
