@@ -267,7 +267,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(dfp::kThreads, 1)
       pi.init(P.start, V, lo, hi);
       int v, x0, x1, piece = 0;
       while (pi.next(v, x0, x1)) {
-        const int b = v / P.R, rb = v % P.R;
+        const int b = v % P.B, rb = v / P.B;
         if (piece > 0 && !mbar_wait(smem_u32(&q_empty), (piece - 1) & 1, abort_p, 2, piece)) break;
         if (rank == 0) mbar_expect_tx(smem_u32(&q_full), 2 * kQBytes);
         const int row0 = b * rows_seq + rb * 128 + 64 * (int)rank;
@@ -443,7 +443,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(dfp::kThreads, 1)
     uint32_t it = 0;
     bool ok = true;
     while (ok && pi.next(v, x0, x1)) {
-      const int b = v / P.R;
+      const int b = v % P.B;
       const int L = P.seq_lens[b];
       for (int x = x0; x < x1 && ok; ++x)
         for (int k = 0; k < per_block; ++k, ++it) {
@@ -492,7 +492,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(dfp::kThreads, 1)
     int j = 0;
     bool dead = false;
     while (!dead && pi.next(v, x0, x1)) {
-      const int b = v / P.R, rb = v % P.R;
+      const int b = v % P.B, rb = v / P.B;
       const int L = P.seq_lens[b];
       const int grow = rb * 128 + 64 * (int)rank + h;
       const int tail = P.tail != nullptr ? P.tail[b] : 0;

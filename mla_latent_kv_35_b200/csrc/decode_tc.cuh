@@ -281,7 +281,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(dtc::kThreads, 1)
       int v, x0, x1, piece = 0;
       bool ok = true;
       while (ok && pi.next(v, x0, x1)) {
-        const int b = v / P.R, rb = v % P.R;
+        const int b = v % P.B, rb = v / P.B;
         const int L = P.seq_lens[b];
         // the Q slice is free once the previous piece's QK MMAs completed
         if (piece > 0 && !mbar_wait(smem_u32(&q_empty), (piece - 1) & 1, abort_p, 2, piece)) {
@@ -356,7 +356,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(dtc::kThreads, 1)
       bool ok = true;
       const int rsub = lane >> 4, cc = (lane >> 3) & 1, u = lane & 7;
       while (ok && pi.next(v, x0, x1)) {
-        const int b = v / P.R;
+        const int b = v % P.B;
         const int L = P.seq_lens[b];
         for (int x = x0; x < x1 && ok; ++x)
           for (int p = 0; p < 4 && ok; ++p) {
@@ -546,7 +546,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(dtc::kThreads, 1)
     int j = 0;
     bool dead = false;
     while (!dead && pi.next(v, x0, x1)) {
-      const int b = v / P.R, rb = v % P.R;
+      const int b = v % P.B, rb = v / P.B;
       const int L = P.seq_lens[b];
       const int grow = rb * 128 + 64 * (int)rank + h;      // row within the sequence
       const int tail = P.tail != nullptr ? P.tail[b] : 0;

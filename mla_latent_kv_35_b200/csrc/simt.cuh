@@ -124,11 +124,15 @@ __global__ void cast_f32_bf16_kernel(const float* x, __nv_bfloat16* y, long long
 }
 
 // ---------------------------------------------------------------------------
-// Split planning.  Virtual sequence v = b*R + r (R row blocks per sequence)
-// has nb_v = ceil(L_b / BLK) token blocks.  start[v] = sum_{u<v} nb_u and
-// start[V] = total.  Worker k of G owns blocks [lo_k, lo_{k+1}) of the
-// concatenation, lo_k = floor(k * total / G).  The piece of worker k in v
-// writes partial slot k + v (unique: pieces form a monotone staircase).
+// Split planning.  Virtual sequence v = r*B + b is row block r of sequence
+// b (R row blocks per sequence, row-block-major) and has nb_v =
+// ceil(L_b / BLK) token blocks.  start[v] = sum_{u<v} nb_u and start[V] =
+// total.  Worker k of G owns blocks [lo_k, lo_{k+1}) of the concatenation,
+// lo_k = floor(k * total / G).  The piece of worker k in v writes partial
+// slot k + v (unique: pieces form a monotone staircase).  Row-block-major
+// order puts worker k of row block 0 and worker k + G/R of row block r on the
+// same tokens of the same sequence at the same time (G a multiple of R), so
+// the second read of a cache tile comes from L2.
 // ---------------------------------------------------------------------------
 // Block counts per virtual sequence and their exclusive prefix sums.  With
 // `tail` (tokens of the sequence held elsewhere, after this cache's range) a
@@ -146,10 +150,10 @@ __global__ void plan_kernel(const int32_t* seq_lens, const int32_t* tail, int B,
     const int v = base + threadIdx.x;
     int nb = 0;
     if (v < V) {
-      const int L = seq_lens[v / R];
-      const int tl = tail != nullptr ? tail[v / R] : 0;
+      const int L = seq_lens[v % B];
+      const int tl = tail != nullptr ? tail[v % B] : 0;
       if (L < 0 || tl < 0 || L > max_tokens || (tail == nullptr && L < S_q)) {
-        if (v % R == 0) raise_flag(kFlagBounds);
+        if (v < B) raise_flag(kFlagBounds);
       } else {
         nb = (L + BLK - 1) / BLK;
       }
@@ -282,9 +286,9 @@ __global__ void __launch_bounds__(256) decode_simt_kernel(
 // of a row's wpr merges the pieces i with (i / 2) % wpr == u, two at a time,
 // each lane owning four float4 columns (d_c <= 512, a multiple of 4), so
 // every lane keeps eight loads in flight; the wpr partial sums meet in
-// shared memory.  Virtual sequence v is row block v % R of sequence v / R:
-// rows_per_v workspace rows, of which the ones past the sequence's rows_seq
-// query rows are padding and skipped.
+// shared memory.  Virtual sequence v is row block v / B of sequence v % B
+// (B = V / R): rows_per_v workspace rows, of which the ones past the
+// sequence's rows_seq query rows are padding and skipped.
 // ---------------------------------------------------------------------------
 constexpr int kCombineThreads = 256;
 
@@ -296,10 +300,11 @@ __global__ void __launch_bounds__(kCombineThreads) combine_kernel(
   const int w = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int u = w % wpr;                               // this warp's share of the row
   const int r = (blockIdx.y * 8 + w) / wpr;
-  const int row_in_seq = (v % R) * rows_per_v + r;
+  const int nseq = V / R;
+  const int row_in_seq = (v / nseq) * rows_per_v + r;
   const bool live_row = r < rows_per_v && row_in_seq < rows_seq;
   const int total = start[V];
-  const long long out_row = (long long)(v / R) * rows_seq + row_in_seq;
+  const long long out_row = (long long)(v % nseq) * rows_seq + row_in_seq;
   const bool any = start[v + 1] > start[v];
   const int k0 = any ? worker_of(start[v], total, G) : 0;
   const int n = (any && live_row) ? worker_of(start[v + 1] - 1, total, G) - k0 + 1 : 0;

@@ -138,8 +138,9 @@ def boundary_sequences(w, S_q=1):
     the planner's own rule (worker k starts at block floor(k*total/G))."""
     d = MLADims.of(w)
     _, bt, G = B.mla_decode_config(d, S_q, 0)
-    R = max(1, S_q * w.H // 128)
-    nb = [-(-L // bt) for L in w.ctx for _ in range(R)]
+    R = max(1, -(-S_q * w.H // 128))
+    # virtual sequence v = r * B + b: row block r of sequence b
+    nb = [-(-L // bt) for _ in range(R) for L in w.ctx]
     starts = np.concatenate([[0], np.cumsum(nb)])
     total = int(starts[-1])
     out = set()
@@ -147,7 +148,7 @@ def boundary_sequences(w, S_q=1):
         x = k * total // G
         v = int(np.searchsorted(starts, x, side="right") - 1)
         if x != starts[v]:
-            out.add(v // R)
+            out.add(v % w.B)
     return sorted(out)
 
 
