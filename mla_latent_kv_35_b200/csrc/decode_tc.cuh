@@ -152,6 +152,12 @@ __device__ __forceinline__ void named_bar_sync(int id, int nthreads) {
   asm volatile("barrier.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
 }
 
+// Arrive on named barrier `id` without waiting (a producer's half of a
+// producer/consumer handoff; the consumers barrier.sync on it).
+__device__ __forceinline__ void named_bar_arrive(int id, int nthreads) {
+  asm volatile("barrier.arrive %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
+}
+
 // Piece iteration shared by all roles: worker k's blocks [lo, hi) split by
 // virtual sequence.
 struct PieceIter {
@@ -196,7 +202,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(dtc::kThreads, 1)
   extern __shared__ uint8_t smem_raw[];
   __shared__ __align__(8) uint64_t qk_full[kQkStages], qk_empty[kQkStages];
   __shared__ __align__(8) uint64_t pv_full[kPvStages], pv_empty[kPvStages];
-  __shared__ __align__(8) uint64_t q_full, q_empty, o_empty, p_full[2], pv_done;
+  __shared__ __align__(8) uint64_t q_full, q_empty, o_empty, p_full[2][4], pv_done;
   __shared__ __align__(8) uint64_t s_full[2], s_free[2], drain_qk, drain_pv;
   __shared__ float red_max[4][64];
   __shared__ uint32_t tmem_base_sh;
@@ -233,8 +239,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(dtc::kThreads, 1)
     // two blocks must not meet on one barrier.  Block j + 2 cannot arrive
     // before phase j completes: its S needs PV(j) to have released the
     // buffer.
-    mbar_init(smem_u32(&p_full[0]), 16);
-    mbar_init(smem_u32(&p_full[1]), 16);
+    for (int b = 0; b < 2; ++b)
+      for (int pg = 0; pg < 4; ++pg) mbar_init(smem_u32(&p_full[b][pg]), 8);
     mbar_init(smem_u32(&pv_done), 1);
     mbar_init(smem_u32(&drain_qk), 1);
     mbar_init(smem_u32(&drain_pv), 1);
@@ -468,7 +474,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(dtc::kThreads, 1)
       }
     } else if (warp == 3 && lane == 0 && rank == 0) {
       // =================  PV MMA issuer (leader CTA)  =================
-      // PV(j) begins once P(j) is in TMEM and, for the first block of a
+      // PV(j) begins on a page once that page of P(j) is in TMEM (the
+      // softmax hands P over page by page) and, for the first block of a
       // piece, once the previous piece's epilogue has released O.  A is P(j)
       // in TMEM (S buffer j & 1): lane l holds the row of output lane l, 256
       // tokens as bf16 pairs in 128 columns, so K-step kk of page p starts at
@@ -483,10 +490,15 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(dtc::kThreads, 1)
       bool ok = true;
       while (ok && vi.next(v, x0, x1)) {
         for (int x = x0; x < x1 && ok; ++x, ++jp) {
-          ok = mbar_wait(smem_u32(&p_full[jp & 1]), (jp >> 1) & 1, abort_p, 2, jp);
-          if (ok && x == x0 && piece > 0)
+          if (x == x0 && piece > 0)
             ok = mbar_wait(smem_u32(&o_empty), (piece - 1) & 1, abort_p, 3, piece);
           for (int t = 0; t < kPvStagesPerBlock && ok; ++t, ++itv) {
+            // page t / 2 of P(jp) is in TMEM, in all lanes of both CTAs
+            if ((t & 1) == 0 &&
+                !mbar_wait(smem_u32(&p_full[jp & 1][t >> 1]), (jp >> 1) & 1, abort_p, 2, jp)) {
+              ok = false;
+              break;
+            }
             const int s = itv % kPvStages;
             if (!mbar_wait(smem_u32(&pv_full[s]), (itv / kPvStages) & 1, abort_p, 9, itv)) {
               ok = false;
@@ -531,14 +543,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(dtc::kThreads, 1)
     const int h = tl & 63, hh = tl >> 6;             // row of this CTA, token half
     const int pb = 2 * hh + ch;                      // page of the block this thread scores
     const uint32_t lane_addr = (uint32_t)(32 * quad) << 16;
-    const uint32_t lead_pfull = mapa_shared(smem_u32(&p_full[0]), 0);
+    const uint32_t lead_pfull = mapa_shared(smem_u32(&p_full[0][0]), 0);
     const uint32_t lead_oempty = mapa_shared(smem_u32(&o_empty), 0);
-    // P exchange: warps sw and sw ^ 2 hold the two token halves of the same
-    // rows; pair (sw & 1) + 2 (sw >> 2) swaps them through sX in round
-    // number pair, half (sw >> 1) & 1 of the buffer written by each warp
-    const int xpair = (sw & 1) | ((sw >> 2) << 1);
-    const uint32_t x_mine = sX + ((sw >> 1) & 1) * 4096 + lane * 128;
-    const uint32_t x_theirs = sX + (((sw >> 1) & 1) ^ 1) * 4096 + lane * 128;
+    // P exchange: warp (quad q, half ch) and warp (q ^ 2, ch) hold the two
+    // token halves of the same rows; the two warps writing a page use the
+    // halves q & 1 of the buffer, and each reader reads its partner's half
+    const uint32_t x_slot = sX + (quad & 1) * 4096 + lane * 128;
     float* red_sum = reinterpret_cast<float*>(smem_raw + (sX - smem_u32(smem_raw)));  // [4][64]
     PieceIter pi;
     pi.init(P.start, V, lo, hi);
@@ -611,40 +621,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(dtc::kThreads, 1)
             pk[16 * hf + e] = pack_bf16x2(p0, p1);
           }
         }
-        // P(j) goes to TMEM over S(j), as the A operand of PV(j): every lane
-        // needs all 256 tokens of its row, so the two warps holding the two
-        // halves of the same rows swap theirs through shared memory (four
-        // rounds, one warp pair each; the barriers also order every thread's
-        // last read of S before any write of P).
-        uint32_t pq[32];
-        tc_fence_before();
-        bool stop = false;
-#pragma unroll 1
-        for (int rho = 0; rho < 4; ++rho) {
-          if (xpair == rho) {
-#pragma unroll
-            for (int u = 0; u < 8; ++u)
-              asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(
-                               x_mine + ((u ^ (lane & 7)) << 4)),
-                           "r"(pk[4 * u]), "r"(pk[4 * u + 1]), "r"(pk[4 * u + 2]),
-                           "r"(pk[4 * u + 3])
-                           : "memory");
-          }
-          named_bar_sync(2, kSoftmaxThreads);
-          if (xpair == rho) {
-#pragma unroll
-            for (int u = 0; u < 8; ++u)
-              asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];"
-                           : "=r"(pq[4 * u]), "=r"(pq[4 * u + 1]), "=r"(pq[4 * u + 2]),
-                             "=r"(pq[4 * u + 3])
-                           : "r"(x_theirs + ((u ^ (lane & 7)) << 4))
-                           : "memory");
-          }
-          if (rho < 3) named_bar_sync(3, kSoftmaxThreads);
-          else stop = named_bar_or(3, kSoftmaxThreads, *abort_p != 0);
-        }
-        if (stop) { dead = true; break; }
-        tc_fence_after();
         // O is rescaled only when some row of this warp moved its max; PV of
         // the previous block accumulates into O and must be done first.
         bool ok = true;
@@ -665,19 +641,61 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(dtc::kThreads, 1)
                 r[i] = __float_as_uint(__uint_as_float(r[i]) * alpha);
               tmem_st32(oa, r);
             }
+            tmem_wait_st();
           }
         }
-        {
-          const uint32_t pa = tmem + lane_addr + kTmemS + 128 * (j & 1) + 32 * ch;
-          tmem_st32(pa + 64 * hh, pk);
-          tmem_st32(pa + 64 * (1 - hh), pq);
-          tmem_wait_st();
+        // P(j) goes to TMEM over S(j), as the A operand of PV(j), page by
+        // page: every lane needs its row's P on all four pages, and the two
+        // warps that hold a page's rows in one lane half hand them to the two
+        // warps of the other half through shared memory, one page per round.
+        // PV(j) begins on page 0 while later pages are still being swapped.
+        // This barrier orders every thread's reads of S and every rescale of
+        // O before any write of P (and so before PV(j) starts).
+        tc_fence_before();
+        if (named_bar_or(2, kSoftmaxThreads, !ok || *abort_p != 0)) { dead = true; break; }
+        tc_fence_after();
+        const uint32_t pa = tmem + lane_addr + kTmemS + 128 * (j & 1);
+        const uint32_t lead_pf = lead_pfull + 8 * (4 * (j & 1));   // p_full[j & 1][0]
+        tmem_st32(pa + 32 * pb, pk);          // this thread's own page, its own lane
+        tmem_wait_st();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive_cluster(lead_pf + 8 * pb);
+#pragma unroll 1
+        for (int pg = 0; pg < 4; ++pg) {
+          const bool writer = (hh == (pg >> 1)) && (ch == (pg & 1));
+          const bool reader = (hh != (pg >> 1)) && (ch == (pg & 1));
+          if (pg > 0 && writer) named_bar_sync(6 + pg, 128);   // readers of pg - 1 done
+          if (writer) {
+#pragma unroll
+            for (int u = 0; u < 8; ++u)
+              asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(
+                               x_slot + ((u ^ (lane & 7)) << 4)),
+                           "r"(pk[4 * u]), "r"(pk[4 * u + 1]), "r"(pk[4 * u + 2]),
+                           "r"(pk[4 * u + 3])
+                           : "memory");
+            named_bar_arrive(3 + pg, 128);
+          }
+          if (reader) {
+            uint32_t pq[32];
+            named_bar_sync(3 + pg, 128);
+#pragma unroll
+            for (int u = 0; u < 8; ++u)
+              asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];"
+                           : "=r"(pq[4 * u]), "=r"(pq[4 * u + 1]), "=r"(pq[4 * u + 2]),
+                             "=r"(pq[4 * u + 3])
+                           : "r"(x_slot + ((u ^ (lane & 7)) << 4))
+                           : "memory");
+            if (pg < 3) named_bar_arrive(7 + pg, 128);          // the next writers may go
+            tmem_st32(pa + 32 * pg, pq);
+            tmem_wait_st();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive_cluster(lead_pf + 8 * pg);
+          }
         }
         l = need ? l * alpha + lsum : l + lsum;
         m = m_use;
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0 && ok) mbar_arrive_cluster(lead_pfull + 8 * (j & 1));
         o_started = true;
       }
       if (dead) break;
@@ -691,6 +709,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(dtc::kThreads, 1)
       bool got = true;
       if (jl > 0) got = mbar_wait(smem_u32(&pv_done), (jl - 1) & 1, abort_p, 10, jl);
       got = got && mbar_wait(smem_u32(&pv_done), jl & 1, abort_p, 10, jl);
+      named_bar_sync(2, kSoftmaxThreads);   // the last P swap has left the shared buffer
       red_sum[64 * pb + h] = l;
       if (named_bar_or(1, kSoftmaxThreads, !got || *abort_p)) { dead = true; break; }
       tc_fence_after();
