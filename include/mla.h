@@ -341,6 +341,44 @@ mla_status mla_out_proj(const mla_dims* dims, const float* o_lat,
                         const void* w_uv, const void* w_o, void* scratch,
                         size_t scratch_bytes, float* out, int T, void* stream);
 
+/* P1 -- chunked prefill, rebuild step ([DF-1]: k = W_UK c, v = W_UV c per
+ * head; the non-absorbed form, which pays once many new queries share every
+ * rebuilt key).  For the L cached tokens t < L of ONE sequence:
+ *   ctx[t, :]       = pool[page_row[t / page_size]][t % page_size][:]
+ *   k_nope[t, i, n] = sum_c w_uk[i, n, c] * ctx[t, c]      c < d_latent
+ *   v[t, i, e]      = sum_c w_uv[i, e, c] * ctx[t, c]
+ * pool: device [n_pages, page_size, d_latent + d_rope]; page_row: device
+ * int32, the sequence's page-table row (ceil(L / page_size) entries are
+ * read); w_uk: device [H, d_nope, d_latent]; w_uv: device [H, d_v,
+ * d_latent]; ctx: device [L, d_latent + d_rope] (out); k_nope: device
+ * [L, H, d_nope] (out); v: device [L, H, d_v] (out).  fp32 accumulation,
+ * outputs rounded to bf16.  bf16 only, DeepSeek-V2 widths (d_nope = d_v =
+ * 128, d_latent = 512, d_rope = 64), else MLA_ERR_UNSUPPORTED.  All buffers
+ * 16-byte aligned.  L = 0 is a no-op.  A page id outside [0, n_pages)
+ * zeroes that row of ctx and raises MLA_ERR_BOUNDS in the device status. */
+mla_status mla_prefill_rebuild_kv(const mla_dims* dims, const void* pool, int n_pages,
+                                  const int32_t* page_row, int L, const void* w_uk,
+                                  const void* w_uv, void* ctx, void* k_nope, void* v,
+                                  void* stream);
+
+/* P2 -- chunked prefill attention, causal ([DF-0]), on the rebuilt keys and
+ * values ([DF-1]: k_{i,t} = [k_nope[t, i, :] ; ctx[t, d_latent:]], the RoPE
+ * key shared by all heads; v_{i,t} = v[t, i, :]).  The T queries are the
+ * last T tokens of the sequence: query j sits at position L - T + j and
+ * attends to the tokens t <= L - T + j.  For j < T and head i:
+ *   s_t = scale * (q[j, i, :] . k_{i,t}),   p = softmax of s over those t
+ *   o[j, i, :] = sum_t p_t v[t, i, :],       lse[j, i] = ln sum_t exp(s_t)
+ * q: device bf16, query j head i at q + j*q_stride_tok + i*(d_nope+d_rope),
+ * [q_nope ; q_rope] with RoPE already applied (e.g. the A0 output after
+ * mla_rope in place); ctx, k_nope, v: as written by mla_prefill_rebuild_kv;
+ * o: device bf16 [T, H, d_v] (out, the input of the W_O projection, which
+ * mla_project applies); lse: device fp32 [T, H] (out).  0 <= T <= L
+ * (T = 0 is a no-op); q_stride_tok % 8 == 0; shapes as for
+ * mla_prefill_rebuild_kv; all buffers 16-byte aligned. */
+mla_status mla_prefill_attention(const mla_dims* dims, const void* q, int q_stride_tok,
+                                 const void* ctx, const void* k_nope, const void* v, int T,
+                                 int L, void* o, float* lse, void* stream);
+
 /* Synchronises `stream`, then returns and clears the device status word of
  * the current device (MLA_OK, MLA_ERR_TIMEOUT or MLA_ERR_BOUNDS; TIMEOUT
  * wins if both were raised), or MLA_ERR_CUDA if the stream failed. */
@@ -350,7 +388,9 @@ mla_status mla_get_device_status(void* stream);
  * since the last call: out4 = {site, info, parity, CTA index}, all zero if
  * none did.  Sites: 1-10 split-decode kernel (1 producer slot free, 2 query
  * slice free, 3 MMA operands landed, 4 P ready, 5 O free, 6 query landed,
- * 7 S ready, 8-10 PV done), 21-23 GEMM.  Reads and clears the record
+ * 7 S ready, 8-10 PV done), 21-23 GEMM, 31-39 prefill attention (31 stage
+ * free, 32 query landed, 33 keys landed, 34 P ready, 35 values landed, 36 S
+ * buffer free, 37 S ready, 38-39 PV done).  Reads and clears the record
  * (synchronous copy; call after mla_get_device_status). */
 mla_status mla_get_wait_diag(uint32_t* out4);
 

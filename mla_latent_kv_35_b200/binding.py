@@ -29,7 +29,7 @@ EXPORTS = ("mla_project", "mla_absorb_q", "mla_rope", "mla_cache_append",
            "mla_decode_noalloc", "mla_pre_attention", "mla_decode_partial",
            "mla_combine_parts", "mla_decode_config", "mla_decode_noalloc_scratch_bytes",
            "mla_cache_append_fp8", "mla_cache_quantize_fp8", "mla_decode_fp8",
-           "mla_decode_fp8_workspace_size")
+           "mla_decode_fp8_workspace_size", "mla_prefill_rebuild_kv", "mla_prefill_attention")
 
 
 class MLAError(RuntimeError):
@@ -110,6 +110,9 @@ _SIGS = {
     "mla_decode_fp8_workspace_size": ([ctypes.POINTER(Dims), _I, _I, _I], _Z),
     "mla_decode_fp8": ([ctypes.POINTER(Dims), _P, _P, _I, _P, _I, _P, _I, _I, _I, _P, _Z,
                         _P, _P, _P], _I),
+    "mla_prefill_rebuild_kv": ([ctypes.POINTER(Dims), _P, _I, _P, _I, _P, _P, _P, _P, _P, _P],
+                               _I),
+    "mla_prefill_attention": ([ctypes.POINTER(Dims), _P, _I, _P, _P, _P, _I, _I, _P, _P, _P], _I),
 }
 
 FP8_ROW_BYTES = 656
@@ -273,6 +276,21 @@ def mla_decode_noalloc(dims: MLADims, qbuf, pool, n_pages, page_table, max_pages
     _check("mla_decode_noalloc", lib().mla_decode_noalloc(
         ctypes.byref(dims.c()), _ptr(qbuf), _ptr(pool), n_pages, _ptr(page_table), max_pages,
         _ptr(seq_lens), B, S_q, num_workers, _ptr(o_lat), _ptr(lse), _stream()))
+
+
+def mla_prefill_rebuild_kv(dims: MLADims, pool, n_pages, page_row, L, w_uk, w_uv, ctx,
+                           k_nope, v):
+    _dev(pool, page_row, w_uk, w_uv, ctx, k_nope, v)
+    _check("mla_prefill_rebuild_kv", lib().mla_prefill_rebuild_kv(
+        ctypes.byref(dims.c()), _ptr(pool), n_pages, _ptr(page_row), L, _ptr(w_uk), _ptr(w_uv),
+        _ptr(ctx), _ptr(k_nope), _ptr(v), _stream()))
+
+
+def mla_prefill_attention(dims: MLADims, q, q_stride_tok, ctx, k_nope, v, T, L, o, lse):
+    _dev(q, ctx, k_nope, v, o, lse)
+    _check("mla_prefill_attention", lib().mla_prefill_attention(
+        ctypes.byref(dims.c()), _ptr(q), q_stride_tok, _ptr(ctx), _ptr(k_nope), _ptr(v), T, L,
+        _ptr(o), _ptr(lse), _stream()))
 
 
 def mla_out_proj_scratch_size(dims: MLADims, T: int) -> int:

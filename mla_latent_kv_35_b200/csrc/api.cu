@@ -16,6 +16,7 @@
 #include "decode_tc.cuh"
 #include "fp8.cuh"
 #include "gemm_tc.cuh"
+#include "prefill_tc.cuh"
 #include "simt.cuh"
 
 using namespace mla;
@@ -696,6 +697,60 @@ mla_status mla_out_proj(const mla_dims* dims, const float* o_lat, const void* w_
   sum_splits_kernel<<<(unsigned)((n_out / 4 + 255) / 256 + 1), 256, 0, st>>>(parts, splits, n_out,
                                                                              out);
   return check_launch();
+}
+
+// ---------------------------------------------------------------------------
+// chunked prefill (non-absorbed)
+// ---------------------------------------------------------------------------
+static bool prefill_dims_ok(const mla_dims* d) {
+  return d->dtype == MLA_BF16 && d->d_nope == pfa::kDN && d->d_rope == pfa::kDR &&
+         d->d_v == pfa::kDV && d->d_latent == pfa::kDC;
+}
+
+mla_status mla_prefill_rebuild_kv(const mla_dims* dims, const void* pool, int n_pages,
+                                  const int32_t* page_row, int L, const void* w_uk,
+                                  const void* w_uv, void* ctx, void* k_nope, void* v,
+                                  void* stream) {
+  if (!dims_ok(dims) || L < 0 || n_pages < 1) return MLA_ERR_INVALID_ARG;
+  if (!prefill_dims_ok(dims)) return MLA_ERR_UNSUPPORTED;
+  if (L == 0) return MLA_OK;
+  if (!pool || !page_row || !w_uk || !w_uv || !ctx || !k_nope || !v) return MLA_ERR_INVALID_ARG;
+  if (!aligned16(pool) || !aligned16(ctx) || !aligned16(k_nope) || !aligned16(v) ||
+      !aligned16(w_uk) || !aligned16(w_uv))
+    return MLA_ERR_INVALID_ARG;
+  cudaStream_t st = as_stream(stream);
+  const int H = dims->n_heads, D = pfa::kD;
+  const int row_vecs = D * 2 / 16;
+  const long long n = (long long)L * row_vecs;
+  gather_rows_kernel<<<(unsigned)((n + 255) / 256), 256, 0, st>>>(
+      static_cast<const uint4*>(pool), n_pages, dims->page_size, page_row, L, row_vecs,
+      static_cast<uint4*>(ctx));
+  MLA_TRY(check_launch());
+  // k_nope[t][i*128 + n] = sum_c w_uk[i*128 + n][c] ctx[t][c]: A = w_uk as
+  // [H*128][512] (K-major), X = the first 512 columns of ctx rows
+  MLA_TRY(launch_tc_gemm(w_uk, false, 0, ctx, D, 0, H * pfa::kDN, L, pfa::kDC, 1, k_nope, 0,
+                         (long long)H * pfa::kDN, 1, kOutBf16, st));
+  return launch_tc_gemm(w_uv, false, 0, ctx, D, 0, H * pfa::kDV, L, pfa::kDC, 1, v, 0,
+                        (long long)H * pfa::kDV, 1, kOutBf16, st);
+}
+
+mla_status mla_prefill_attention(const mla_dims* dims, const void* q, int q_stride_tok,
+                                 const void* ctx, const void* k_nope, const void* v, int T,
+                                 int L, void* o, float* lse, void* stream) {
+  if (!dims_ok(dims) || T < 0 || L < T) return MLA_ERR_INVALID_ARG;
+  if (!prefill_dims_ok(dims)) return MLA_ERR_UNSUPPORTED;
+  if (T == 0) return MLA_OK;
+  const int H = dims->n_heads;
+  if (!q || !ctx || !k_nope || !v || !o || !lse) return MLA_ERR_INVALID_ARG;
+  if (q_stride_tok < H * pfa::kDQK || (q_stride_tok % 8) != 0 || !aligned16(q) ||
+      !aligned16(ctx) || !aligned16(k_nope) || !aligned16(v) || !aligned16(o))
+    return MLA_ERR_INVALID_ARG;
+  const mla_status s = launch_prefill_attn_impl(make_tmap_bf16, q, q_stride_tok, ctx, k_nope, v,
+                                                T, L, H, dims->scale,
+                                                static_cast<__nv_bfloat16*>(o), lse,
+                                                as_stream(stream));
+  g_launches.fetch_add(1, std::memory_order_relaxed);
+  return s;
 }
 
 }  // extern "C"

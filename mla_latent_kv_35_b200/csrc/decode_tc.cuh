@@ -202,7 +202,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(dtc::kThreads, 1)
   extern __shared__ uint8_t smem_raw[];
   __shared__ __align__(8) uint64_t qk_full[kQkStages], qk_empty[kQkStages];
   __shared__ __align__(8) uint64_t pv_full[kPvStages], pv_empty[kPvStages];
-  __shared__ __align__(8) uint64_t q_full, q_empty, o_empty, p_full[2][4], pv_done;
+  __shared__ __align__(8) uint64_t q_full, q_empty, o_empty, p_full[2][4], pv_done, pv_last;
   __shared__ __align__(8) uint64_t s_full[2], s_free[2], drain_qk, drain_pv;
   __shared__ float red_max[4][64];
   __shared__ uint32_t tmem_base_sh;
@@ -242,6 +242,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(dtc::kThreads, 1)
     for (int b = 0; b < 2; ++b)
       for (int pg = 0; pg < 4; ++pg) mbar_init(smem_u32(&p_full[b][pg]), 8);
     mbar_init(smem_u32(&pv_done), 1);
+    mbar_init(smem_u32(&pv_last), 1);   // after the last PV of each piece
     mbar_init(smem_u32(&drain_qk), 1);
     mbar_init(smem_u32(&drain_pv), 1);
     for (int b = 0; b < 2; ++b) {
@@ -527,6 +528,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(dtc::kThreads, 1)
             mma_commit_2_mc(smem_u32(&s_free[jp & 1]), 1);
           }
         }
+        if (ok) mma_commit_2_mc(smem_u32(&pv_last), 3);
         ++piece;
       }
       if (!ok) {
@@ -553,7 +555,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(dtc::kThreads, 1)
     PieceIter pi;
     pi.init(P.start, V, lo, hi);
     int v, x0, x1;
-    int j = 0;
+    int j = 0, pc = 0;
     bool dead = false;
     while (!dead && pi.next(v, x0, x1)) {
       const int b = v % P.B, rb = v / P.B;
@@ -700,15 +702,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(dtc::kThreads, 1)
       }
       if (dead) break;
       // ---------------- epilogue of the piece ----------------
-      // O is final once PV of the piece's last block jl is done.  The
-      // softmax may be up to two blocks ahead of PV here (it no longer waits
-      // for PV(j - 1) before handing over P(j)), and a parity wait is sound
-      // only when at most one phase is outstanding: wait for PV(jl - 1)
-      // first, then for PV(jl).
-      const int jl = j - 1;
-      bool got = true;
-      if (jl > 0) got = mbar_wait(smem_u32(&pv_done), (jl - 1) & 1, abort_p, 10, jl);
-      got = got && mbar_wait(smem_u32(&pv_done), jl & 1, abort_p, 10, jl);
+      // O is final once PV of the piece's last block is done: pv_last
+      // completes once per piece (phase pc).  The next piece's PV waits for
+      // this epilogue (o_empty), so no later phase can complete first.  (A
+      // parity wait on pv_done could not tell PV(j - 2) from PV(j) when the
+      // last two PVs have both completed by now.)
+      const bool got = mbar_wait(smem_u32(&pv_last), pc & 1, abort_p, 10, pc);
+      ++pc;
       named_bar_sync(2, kSoftmaxThreads);   // the last P swap has left the shared buffer
       red_sum[64 * pb + h] = l;
       if (named_bar_or(1, kSoftmaxThreads, !got || *abort_p)) { dead = true; break; }

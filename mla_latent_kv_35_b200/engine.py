@@ -154,6 +154,67 @@ class MLADecodeLayer:
                         bf["out"], T)
         return bf
 
+    # ------------------------------------------------------------------
+    # chunked prefill (non-absorbed)
+    # ------------------------------------------------------------------
+    def prefill_buffers(self, T: int, L: int):
+        """Device buffers of one prefill chunk of T tokens ending at context L."""
+        key = ("prefill", T, L)
+        if key not in self._bufs:
+            d = self.dims
+            dev, dt = self.device, d.torch_dtype
+            H = d.n_heads
+            self._bufs[key] = dict(
+                y=torch.empty((T, self.Y), dtype=dt, device=dev),
+                ctx=torch.empty((L, self.D), dtype=dt, device=dev),
+                k_nope=torch.empty((L, H, d.d_nope), dtype=dt, device=dev),
+                v=torch.empty((L, H, d.d_v), dtype=dt, device=dev),
+                o=torch.empty((T, H, d.d_v), dtype=dt, device=dev),
+                lse=torch.empty((T, H), dtype=torch.float32, device=dev),
+                out=torch.empty((T, d.d_model), dtype=dt, device=dev),
+            )
+        return self._bufs[key]
+
+    def prefill_chunk(self, h, pos, batch_idx, b: int, T: int, L: int):
+        """Prefill T new tokens of sequence b, at positions L - T .. L - 1.
+
+        h [T, d_model] device; pos int32 [T] = L - T .. L - 1 and batch_idx
+        int32 [T] = b, both on the device.  The chunk takes the non-absorbed
+        form: the new tokens' latents and RoPE keys go into the cache, then
+        every head's keys and values of all L tokens are rebuilt once
+        (W_UK c, W_UV c) and the T queries attend causally over them.
+
+          P0  mla_project            y = [W_Q; W_DKV; W_KR] h
+          P0  mla_rope (x2)          q_rope and k_rope rotated in place in y
+          P0  mla_cache_append       [c ; k_rope] -> paged pool
+          P1  mla_prefill_rebuild_kv ctx rows, k_nope, v of the L tokens
+          P2  mla_prefill_attention  o [T, H, d_v], lse [T, H]
+          P3  mla_project            out = W_O o  (bf16 [T, d_model])
+
+        Returns the dict of chunk buffers.  bf16 layers with a bf16 cache."""
+        d = self.dims
+        if d.dtype != "bf16" or self.cache_kind != "bf16":
+            raise ValueError("chunked prefill needs a bf16 layer and a bf16 cache")
+        if not 0 < T <= L:
+            raise ValueError("need 0 < T <= L")
+        H, dn, dc = d.n_heads, d.d_nope, d.d_latent
+        Y, dqk = self.Y, self.dqk
+        off_c = H * dqk
+        bf = self.prefill_buffers(T, L)
+        y = bf["y"]
+        _b.mla_project(d, h, self.W_A0, y, T, d.d_model, Y)
+        _b.mla_rope(d, y[:, dn:], Y, dqk, H, y[:, dn:], Y, dqk, pos, T)
+        kr = y[:, off_c + dc:]
+        _b.mla_rope(d, kr, Y, 0, 1, kr, Y, 0, pos, T)
+        _b.mla_cache_append(d, y[:, off_c:], Y, kr, Y, batch_idx, pos, self.page_table,
+                            self.max_pages, self.pool, self.n_pages, T)
+        _b.mla_prefill_rebuild_kv(d, self.pool, self.n_pages, self.page_table[b], L, self.W_UK,
+                                  self.W_UV, bf["ctx"], bf["k_nope"], bf["v"])
+        _b.mla_prefill_attention(d, y, Y, bf["ctx"], bf["k_nope"], bf["v"], T, L, bf["o"],
+                                 bf["lse"])
+        _b.mla_project(d, bf["o"], self.W_O, bf["out"], T, H * d.d_v, d.d_model)
+        return bf
+
     def capture(self, h, batch_idx, pos, B: int, S_q: int, num_workers: int = 0,
                 fused: bool = True, slot: int = 0):
         """Capture one step on these input buffers into a CUDA graph.

@@ -8,7 +8,7 @@ once, so both sides consume exactly the same numbers.
 
 Shapes follow DeepSeek-V2's attention (deepforge "DeepSeek-V2" page, §1 "Store
 a latent, rebuild the keys and values": 128 heads of width 128, a 512-dim
-latent and a 64-dim RoPE key per token).  Five workloads:
+latent and a 64-dim RoPE key per token).  Seven workloads:
 
   tiny       fp32: B=2, H=8, d_model 256, d_nope 32, latent 64, rope 16,
              contexts {37, 64}, prior cache built from hidden states
@@ -17,6 +17,8 @@ latent and a 64-dim RoPE key per token).  Five workloads:
   ragged     bf16: B=64, prior lengths log-uniform in [128, 65536] (seed 7),
              one new token appended per sequence, permuted pages
   long1/long4 bf16: B=1 / B=4, L=131072 including 2 speculative query tokens
+  prefill    bf16: one sequence, a chunk of 4096 new tokens after 4096 cached
+             ones (the chunk's tokens are the S_q query tokens)
 
 Random streams: every array has its own stream,
 ``default_rng(SeedSequence([seed, stream, index]))``, so one sequence's
@@ -112,12 +114,15 @@ def workload(name: str, **over) -> Workload:
         B = 1 if name == "long1" else 4
         w = Workload(name, B=B, S_q=2, ctx=(131072,) * B,
                      permute_pages=True, **big)
+    elif name == "prefill":
+        # one sequence: 4096 cached tokens, then a chunk of 4096 new ones
+        w = Workload("prefill", B=1, S_q=4096, ctx=(8192,), permute_pages=True, **big)
     else:
         raise KeyError(name)
     return replace(w, **over) if over else w
 
 
-WORKLOADS = ("tiny", "dsv2", "batch128", "ragged", "long1", "long4")
+WORKLOADS = ("tiny", "dsv2", "batch128", "ragged", "long1", "long4", "prefill")
 
 
 def shard(w: Workload, rank: int, world: int) -> Workload:

@@ -56,6 +56,7 @@ def check(got, ref, dtype, what="", tol=None):
     nrm = float(np.linalg.norm(ref[finite]))
     rel = float(np.linalg.norm(d) / nrm) if nrm > 0 else 0.0
     msg = f"{what}: max_abs={mx:.3e} mean_abs={mean:.3e} rel_l2={rel:.3e}"
+    print(msg)
     assert mx <= t["max_abs"], msg
     assert mean <= t["mean_abs"], msg
     assert rel <= t["rel_l2"], msg
