@@ -503,6 +503,224 @@ def run_gpu(args, w):
         dist.destroy_process_group()
 
 
+# ---------------------------------------------------------------------------
+# Chunked prefill (non-absorbed): one chunk of T new tokens of one sequence
+# ---------------------------------------------------------------------------
+def prefill_flops(w):
+    """Algorithmic FLOPs of one chunk per stage (multiply-add = 2): the A0
+    projection, the K/V rebuild of all L tokens, the causal attention (query
+    j sees L - T + j + 1 tokens; QK over d_nope + d_rope, PV over d_v) and
+    the W_O projection."""
+    T, L, H = w.S_q, w.ctx[0], w.H
+    Y = H * (w.d_nope + w.d_rope) + w.D
+    pairs = sum(L - T + j + 1 for j in range(T))
+    return {"a0": 2.0 * T * w.d_model * Y,
+            "rebuild": 2.0 * L * H * (w.d_nope + w.d_v) * w.d_latent,
+            "attention": 2.0 * pairs * H * (w.d_nope + w.d_rope + w.d_v),
+            "w_o": 2.0 * T * H * w.d_v * w.d_model}
+
+
+def prefill_config(w, world):
+    return {"workload": w.name, "chunk_tokens": w.S_q, "cached_before": w.ctx[0] - w.S_q,
+            "context_after": w.ctx[0], "heads": w.H, "d_nope": w.d_nope, "d_rope": w.d_rope,
+            "d_v": w.d_v, "latent": w.d_latent, "d_model": w.d_model, "page": w.page_size,
+            "form": "non-absorbed: K/V rebuilt per head from the latent cache",
+            "l2": "inputs larger than L2 (rebuilt K/V %.0f MB, weights %.0f MB), no flush"
+                  % (w.ctx[0] * w.H * (w.d_nope + w.d_v) * 2 / 1e6,
+                     2 * (w.H * (w.d_nope + w.d_rope) * w.d_model + w.D * w.d_model
+                          + 2 * w.H * 128 * w.d_latent + w.d_model * w.H * w.d_v) / 1e6),
+            "parallelism": (f"dp{world}: one sequence per rank, no collective"
+                            if world > 1 else "single GPU")}
+
+
+def _oracle_prefill_sample(w, n=128):
+    """The oracle on the first n tokens of the chunk: by causality they are
+    computed exactly as in the whole chunk (same prior, same positions).
+    Returns (tokens/s, sample text, cores, seconds)."""
+    import oracle
+    from mla_latent_kv_35_b200 import workloads as wl
+    W = wl.draw_weights(w)
+    h = wl.draw_h_new(w)[:, :n]
+    c, kr = wl.draw_prior(w, 0)
+    cores = len(os.sched_getaffinity(0))
+    t0 = time.perf_counter()
+    oracle.decode_step(h, [c], [kr], W["W_Q"], W["W_DKV"], W["W_KR"], W["W_UK"], W["W_UV"],
+                       W["W_O"], w.scale, w.rope_base, w.H, prior_kr_rotated=True)
+    t = time.perf_counter() - t0
+    sample = (f"first {n} of {w.S_q} chunk tokens of {w.name} (causally identical to the whole "
+              f"chunk's), all {w.H} heads, fp64 non-absorbed oracle, {t:.1f} s; the oracle "
+              f"rebuilds every head's keys and values for this sample alone, which the whole "
+              f"chunk would share")
+    return n / t, sample, cores, t
+
+
+def run_reference_prefill(args, w):
+    if int(os.environ.get("RANK", "0")) != 0:
+        return
+    tps = []
+    sample, cores = "", len(os.sched_getaffinity(0))
+    for i in range(args.warmup + args.steps):
+        v, sample, cores, _ = _oracle_prefill_sample(w, n=32)
+        if i >= args.warmup:
+            tps.append(v)
+    value = statistics.mean(tps)
+    line = {
+        "impl": "reference",
+        "metric": "MLA chunked-prefill tokens/s (one attention layer, whole chunk P0-P3)",
+        "value": value, "unit": "tokens/s", "n_gpus": args.gpus, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": 1000.0 * w.S_q / value,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic", "config": prefill_config(w, args.gpus),
+        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def run_gpu_prefill(args, w):
+    import torch
+    import torch.distributed as dist
+    from mla_latent_kv_35_b200 import binding as B
+    from mla_latent_kv_35_b200 import build as _build
+    from mla_latent_kv_35_b200 import workloads as wl
+    from mla_latent_kv_35_b200.engine import MLADecodeLayer, build_pool_host, pool_to_device
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    distributed = "WORLD_SIZE" in os.environ
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if distributed:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                device_id=dev)
+    # weak scaling: every rank prefills its own sequence (global index rank)
+    w = wl.shard(w, rank, world)
+    if rank == 0:
+        _build.build()
+    if distributed:
+        dist.barrier()
+    B.lib()
+    d = B.MLADims.of(w)
+    W = wl.draw_weights(w)
+    layer = MLADecodeLayer(d, W, dev)
+    table, n_pages = wl.page_layout(w)
+    pool = pool_to_device(build_pool_host(w, table, n_pages, [wl.draw_prior_bits(w, 0)]),
+                          w.dtype, dev)
+    layer.set_cache(pool, torch.from_numpy(table).to(dev),
+                    torch.tensor(w.ctx, dtype=torch.int32, device=dev))
+    T, L = w.S_q, w.ctx[0]
+    h_np = wl.draw_h_new(w).reshape(T, w.d_model)
+    bi_np, pos_np = wl.positions(w)
+    h = torch.from_numpy(h_np).to(dev, d.torch_dtype)
+    bi = torch.from_numpy(bi_np).to(dev)
+    pos = torch.from_numpy(pos_np).to(dev)
+    stream = torch.cuda.current_stream(dev)
+    bf = layer.prefill_buffers(T, L)
+
+    def step():
+        layer.prefill_chunk(h, pos, bi, 0, T, L)
+
+    def attention_only():
+        B.mla_prefill_attention(d, bf["y"], layer.Y, bf["ctx"], bf["k_nope"], bf["v"], T, L,
+                                bf["o"], bf["lse"])
+
+    h_host = torch.from_numpy(h_np).to(d.torch_dtype).pin_memory()
+    bi_host = torch.from_numpy(bi_np).pin_memory()
+    pos_host = torch.from_numpy(pos_np).pin_memory()
+    out_host = torch.empty((T, w.d_model), dtype=d.torch_dtype).pin_memory()
+    h_in = torch.empty_like(h)
+    bi_in = torch.empty_like(bi)
+    pos_in = torch.empty_like(pos)
+
+    def e2e_step():
+        h_in.copy_(h_host, non_blocking=True)
+        bi_in.copy_(bi_host, non_blocking=True)
+        pos_in.copy_(pos_host, non_blocking=True)
+        o = layer.prefill_chunk(h_in, pos_in, bi_in, 0, T, L)
+        out_host.copy_(o["out"], non_blocking=True)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize(dev)
+    st = B.mla_get_device_status()
+    if st != 0:
+        raise RuntimeError(f"device status after warm-up: {B.mla_status_string(st)}")
+
+    def timed(fn, K):
+        if distributed:
+            dist.barrier()
+        torch.cuda.synchronize(dev)
+        l0 = B.mla_launch_count()
+        t0 = time.perf_counter()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(K):
+            fn()
+        e1.record(stream)
+        torch.cuda.synchronize(dev)
+        wall = time.perf_counter() - t0
+        launches = B.mla_launch_count() - l0
+        if distributed:
+            dist.barrier()
+        return e0.elapsed_time(e1) / K, wall, launches
+
+    with ClockSampler(local) as clk:
+        clk.mark()
+        step_ms, wall, launches = timed(step, args.steps)
+        att_ms, _, _ = timed(attention_only, max(args.steps, 5))
+        e2e_ms, _, _ = timed(e2e_step, args.steps)
+    clocks = clk.summary()
+    st = B.mla_get_device_status()
+    if st != 0:
+        raise RuntimeError(f"device status after timing: {B.mla_status_string(st)}")
+    t_step, t_att, t_e2e = max_over_ranks([step_ms, att_ms, e2e_ms], dev)
+    _, tf_peak, peak_kind = _peaks()
+    fl = prefill_flops(w)
+    achieved = fl["attention"] / (t_att * 1e-3) / 1e12
+    h2d = h_host.numel() * h_host.element_size() + bi_host.numel() * 4 + pos_host.numel() * 4
+    d2h = out_host.numel() * out_host.element_size()
+    line = {
+        "metric": "MLA chunked-prefill tokens/s (one attention layer, whole chunk P0-P3)",
+        "value": whole_job_rate(T, world, t_step),
+        "unit": "tokens/s",
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": t_step,
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "bf16",
+        "data": "synthetic",
+        "config": prefill_config(w, world),
+        "step_tflops": sum(fl.values()) / (t_step * 1e-3) / 1e12,
+        "roofline": {"kernel": "mla_prefill_attention (prefill_attn_kernel)", "bound": "tensor",
+                     "achieved": achieved, "peak": tf_peak, "unit": "TFLOP/s",
+                     "frac": achieved / tf_peak, "peak_source": peak_kind + " (bf16 burst)",
+                     "alg_flops_per_launch": fl["attention"], "kernel_ms": t_att,
+                     "traffic": None},
+        "e2e": {"value": whole_job_rate(T, world, t_e2e), "unit": "tokens/s",
+                "ms_per_step": t_e2e, "pipelined": False,
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+        "gpu_launches": launches,
+        "clocks": clocks,
+        "wall_s_timed": wall,
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        v, sample, cores, _ = _oracle_prefill_sample(w)
+        line["cpu_baseline"] = {"value": v, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+                                "sample": sample}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if distributed:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -516,6 +734,8 @@ def main():
                          "under twice the L2 size)")
     ap.add_argument("--batch", type=int, default=0,
                     help="use only the first N sequences of the workload")
+    ap.add_argument("--heads", type=int, default=0,
+                    help="use N heads instead of the workload's (small profiling case)")
     ap.add_argument("--cache", default="bf16", choices=["bf16", "fp8"],
                     help="latent cache format (fp8: the 8-bit cache, bf16 workloads only)")
     args = ap.parse_args()
@@ -527,7 +747,15 @@ def main():
         # same shapes with fewer sequences (small profiling case)
         from dataclasses import replace
         w = replace(w, B=args.batch, ctx=w.ctx[:args.batch], name=f"{w.name}[B={args.batch}]")
-    if args.impl == "reference":
+    if args.heads:
+        from dataclasses import replace
+        w = replace(w, H=args.heads, name=f"{w.name}[H={args.heads}]")
+    if w.name.startswith("prefill"):
+        if args.impl == "reference":
+            run_reference_prefill(args, w)
+        else:
+            run_gpu_prefill(args, w)
+    elif args.impl == "reference":
         run_reference(args, w)
     else:
         run_gpu(args, w)

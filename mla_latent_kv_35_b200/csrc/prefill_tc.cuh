@@ -30,19 +30,24 @@
 //     pair MMA output lane l of CTA r reads its A row from TMEM lane l of CTA
 //     r).  CTA r supplies value columns [64r, 64r + 64) of all 128 keys
 //     (MN-major B).
-//   * TMEM: O at columns [0, 128), S/P buffers at [128, 256) and [256, 384):
-//     QK(j + 1) runs while the softmax works on S(j).  QK(j + 2) reuses the
-//     buffer of P(j), so the issuer waits for PV(j) before issuing it.
-//   * Shared memory: Q 48 KB + four stages of (K 24 KB, V 16 KB) = 208 KB.
-//     Lane 0 of warp 0 in each CTA loads its halves; the leader arms every
-//     full barrier with both CTAs' bytes.  A stage is released by a commit
-//     after the PV of its block.
+//   * TMEM: O at columns [0, 128) and three S/P buffers at [128, 512): QK
+//     runs up to three blocks ahead of the softmax; QK(j + 3) reuses the
+//     buffer of P(j) once PV(j) has completed.
+//   * Shared memory: Q 48 KB + five 24 KB key stages + three 16 KB value
+//     stages = 216 KB.  In each CTA lane 0 of warp 0 loads Q and its key
+//     halves, lane 0 of warp 2 its value halves; the leader arms every full
+//     barrier with both CTAs' bytes.  A key stage is released by a commit
+//     after the QK of its block, a value stage after the PV.
 //   * Softmax: eight warps per CTA.  Warps w and w + 4 share TMEM lane
 //     quadrant w and take 64 of the 128 keys each, so a thread holds one
 //     row's scores of one key half; the two halves' maxima meet in shared
-//     memory.  The running max is rescaled lazily (O in TMEM is rescaled
+//     memory, each warp pair on a named barrier of its own.  Blocks off the
+//     causal diagonal take a path without masks; maxima and row sums run in
+//     independent chains, scores go through the packed fp32 FMA.  The running max is rescaled lazily (O in TMEM is rescaled
 //     only when a row's max grows by more than 2^8, after PV(j - 1)).
-//   * One thread of the leader issues every MMA.
+//   * Two threads of the leader issue the MMAs: lane 0 of warp 1 the QK
+//     stream, lane 0 of warp 3 the PV stream, so that neither stream's
+//     barrier waits hold up the other's MMAs.
 //   * Epilogue: O / l in bf16 to o[t][h][0..128) and the natural-log LSE to
 //     lse[t][h] for the rows t < T.
 //
@@ -75,17 +80,18 @@ constexpr int kQBytes = 3 * kChunkQ;         // 48 KB
 constexpr int kChunkK = (kBlk / 2) * 128;    // 64 keys x 64 columns (8 KB)
 constexpr int kKBytes = 3 * kChunkK;         // this CTA's key half (24 KB)
 constexpr int kVBytes = kBlk * 128;          // 128 keys x 64 value columns (16 KB)
-constexpr int kStages = 4;
+constexpr int kKStages = 5;
+constexpr int kVStages = 3;
+constexpr int kSBufs = 3;            // S/P buffers in TMEM
 constexpr uint32_t kOffQ = 0;
 constexpr uint32_t kOffK = kOffQ + kQBytes;
-constexpr uint32_t kOffV = kOffK + kStages * kKBytes;
-constexpr uint32_t kSmemBytes = kOffV + kStages * kVBytes + 1024;  // + alignment
+constexpr uint32_t kOffV = kOffK + kKStages * kKBytes;
+constexpr uint32_t kSmemBytes = kOffV + kVStages * kVBytes + 1024;  // + alignment
 constexpr int kThreads = 384;
 constexpr int kSoftmaxWarp0 = 4;
-constexpr int kSoftmaxThreads = 256;
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kTmemO = 0;
-constexpr uint32_t kTmemS = 128;     // S_b / P_b at [128 + 128b, +128)
+constexpr uint32_t kTmemS = 128;     // S_b / P_b at [128 + 128b, +128), b < 3
 constexpr float kRescaleLog2 = 8.0f;
 }  // namespace pfa
 
@@ -122,9 +128,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(pfa::kThreads, 1)
                         const __grid_constant__ CUtensorMap tmV, const PrefillParams P) {
   using namespace pfa;
   extern __shared__ uint8_t smem_raw[];
-  __shared__ __align__(8) uint64_t k_full[kStages], v_full[kStages], kv_empty[kStages];
-  __shared__ __align__(8) uint64_t q_full, s_full[2], s_free[2], p_full[2], o_done, o_final,
-      drain;
+  __shared__ __align__(8) uint64_t k_full[kKStages], k_empty[kKStages];
+  __shared__ __align__(8) uint64_t v_full[kVStages], v_empty[kVStages];
+  __shared__ __align__(8) uint64_t q_full, s_full[kSBufs], s_free[kSBufs], p_full[kSBufs];
+  __shared__ __align__(8) uint64_t o_final, drain_qk, drain_pv;
   __shared__ float red_max[2][2][kRows];   // [block & 1][key half][row]
   __shared__ float red_l[2][kRows];
   __shared__ uint32_t tmem_base_sh;
@@ -145,20 +152,25 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(pfa::kThreads, 1)
 
   if (threadIdx.x == 0) {
     abort_flag = 0;
-    for (int s = 0; s < kStages; ++s) {
-      mbar_init(smem_u32(&k_full[s]), 1);    // leader's arrive.expect_tx, both CTAs' bytes
+    // full barriers: the leader's arrive.expect_tx with both CTAs' bytes;
+    // empty barriers: an MMA commit multicast to both CTAs
+    for (int s = 0; s < kKStages; ++s) {
+      mbar_init(smem_u32(&k_full[s]), 1);
+      mbar_init(smem_u32(&k_empty[s]), 1);    // after QK of the stage's block
+    }
+    for (int s = 0; s < kVStages; ++s) {
       mbar_init(smem_u32(&v_full[s]), 1);
-      mbar_init(smem_u32(&kv_empty[s]), 1);  // commit after PV of the stage's block
+      mbar_init(smem_u32(&v_empty[s]), 1);    // after PV of the stage's block
     }
     mbar_init(smem_u32(&q_full), 1);
-    for (int b = 0; b < 2; ++b) {
-      mbar_init(smem_u32(&s_full[b]), 1);
-      mbar_init(smem_u32(&s_free[b]), 1);
-      mbar_init(smem_u32(&p_full[b]), 16);   // 8 softmax warps x 2 CTAs
+    for (int b = 0; b < kSBufs; ++b) {
+      mbar_init(smem_u32(&s_full[b]), 1);     // QK commit
+      mbar_init(smem_u32(&s_free[b]), 1);     // PV commit: P_b consumed, O updated
+      mbar_init(smem_u32(&p_full[b]), 16);    // 8 softmax warps x 2 CTAs
     }
-    mbar_init(smem_u32(&o_done), 1);    // commit after every PV
-    mbar_init(smem_u32(&o_final), 1);   // commit after the last PV (one phase)
-    mbar_init(smem_u32(&drain), 1);
+    mbar_init(smem_u32(&o_final), 1);         // after the last PV (one phase)
+    mbar_init(smem_u32(&drain_qk), 1);
+    mbar_init(smem_u32(&drain_pv), 1);
     fence_mbar_init();
     tma_prefetch_desc(&tmQ);
     tma_prefetch_desc(&tmK);
@@ -177,55 +189,66 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(pfa::kThreads, 1)
 
   if (warp < kSoftmaxWarp0) {
     if (warp == 0 && lane == 0) {
-      // ===================  producer (both CTAs)  ===================
+      // ============  Q and K producer (both CTAs)  ============
       const uint32_t lead_q = mapa_shared(smem_u32(&q_full), 0);
       const uint32_t lead_k0 = mapa_shared(smem_u32(&k_full[0]), 0);
-      const uint32_t lead_v0 = mapa_shared(smem_u32(&v_full[0]), 0);
       if (rank == 0) mbar_expect_tx(smem_u32(&q_full), 2 * kQBytes);
       const int qrow = r0 + kRows * (int)rank;
       for (int c = 0; c < 3; ++c) tma_load_3d_pair(sQ + c * kChunkQ, &tmQ, 64 * c, h, qrow, lead_q);
       int issued = 0;
-      bool ok = true;
       for (int j = 0; j < nblk; ++j) {
-        const int s = j % kStages;
-        if (!mbar_wait(smem_u32(&kv_empty[s]), ((j / kStages) & 1) ^ 1, abort_p, 31, j)) {
-          ok = false;
-          break;
-        }
+        const int s = j % kKStages;
+        if (!mbar_wait(smem_u32(&k_empty[s]), ((j / kKStages) & 1) ^ 1, abort_p, 31, j)) break;
         const int key0 = j * kBlk + (kBlk / 2) * (int)rank;
         const uint32_t dk = sK + s * kKBytes;
+        const uint32_t fb = lead_k0 + 8 * s;
         if (rank == 0) mbar_expect_tx(smem_u32(&k_full[s]), 2 * kKBytes);
-        tma_load_3d_pair(dk, &tmK, 0, h, key0, lead_k0 + 8 * s);
-        tma_load_3d_pair(dk + kChunkK, &tmK, 64, h, key0, lead_k0 + 8 * s);
-        tma_load_2d_pair(dk + 2 * kChunkK, &tmKR, kDC, key0, lead_k0 + 8 * s);
+        tma_load_3d_pair(dk, &tmK, 0, h, key0, fb);
+        tma_load_3d_pair(dk + kChunkK, &tmK, 64, h, key0, fb);
+        tma_load_2d_pair(dk + 2 * kChunkK, &tmKR, kDC, key0, fb);
+        ++issued;
+      }
+      if (*abort_p && rank == 0) {
+        // Leaving early: wait (bounded) for the stages already armed, so that
+        // no copy lands in this pair's shared memory after it exits.
+        mbar_wait_bounded(smem_u32(&q_full), 0, kDrainNs);
+        for (int i = max(0, issued - kKStages); i < issued; ++i)
+          mbar_wait_bounded(smem_u32(&k_full[i % kKStages]), (i / kKStages) & 1, kDrainNs);
+      }
+    } else if (warp == 2 && lane == 0) {
+      // ===============  V producer (both CTAs)  ===============
+      const uint32_t lead_v0 = mapa_shared(smem_u32(&v_full[0]), 0);
+      int issued = 0;
+      for (int j = 0; j < nblk; ++j) {
+        const int s = j % kVStages;
+        if (!mbar_wait(smem_u32(&v_empty[s]), ((j / kVStages) & 1) ^ 1, abort_p, 35, j)) break;
         if (rank == 0) mbar_expect_tx(smem_u32(&v_full[s]), 2 * kVBytes);
         tma_load_3d_pair(sV + s * kVBytes, &tmV, 64 * (int)rank, h, j * kBlk, lead_v0 + 8 * s);
         ++issued;
       }
-      if (!ok && rank == 0) {
-        // Leaving early: wait (bounded) for the stages already armed, so that
-        // no copy lands in this pair's shared memory after it exits.
-        mbar_wait_bounded(smem_u32(&q_full), 0, kDrainNs);
-        for (int i = max(0, issued - kStages); i < issued; ++i) {
-          mbar_wait_bounded(smem_u32(&k_full[i % kStages]), (i / kStages) & 1, kDrainNs);
-          mbar_wait_bounded(smem_u32(&v_full[i % kStages]), (i / kStages) & 1, kDrainNs);
-        }
-      }
+      if (*abort_p && rank == 0)
+        for (int i = max(0, issued - kVStages); i < issued; ++i)
+          mbar_wait_bounded(smem_u32(&v_full[i % kVStages]), (i / kVStages) & 1, kDrainNs);
     } else if (warp == 1 && lane == 0 && rank == 0) {
-      // ===================  MMA issuer (leader)  ===================
-      // Order: QK(0), QK(1); then per block j: PV(j) once P(j) is in TMEM,
-      // and QK(j + 2) into the buffer of P(j) once PV(j) has completed.
+      // ==============  QK issuer (leader)  ==============
+      // QK(j) into S/P buffer j % 3 once PV(j - 3) has consumed the P there.
       const uint32_t idesc_qk = idesc_bf16_f32(256, kBlk, false, false);
-      const uint32_t idesc_pv = idesc_bf16_f32(256, kDV, false, true);
       const uint64_t q_desc = sw128_desc(sQ, 16, 1024);
       const uint64_t k_desc = sw128_desc(sK, 16, 1024);
-      const uint64_t v_desc = sw128_desc(sV, kVBytes, 1024);
       bool ok = mbar_wait(smem_u32(&q_full), 0, abort_p, 32, 0);
-      auto issue_qk = [&](int j) -> bool {
-        const int s = j % kStages;
-        if (!mbar_wait(smem_u32(&k_full[s]), (j / kStages) & 1, abort_p, 33, j)) return false;
+      for (int j = 0; j < nblk && ok; ++j) {
+        const int b = j % kSBufs, s = j % kKStages;
+        if (j >= kSBufs &&
+            !mbar_wait(smem_u32(&s_free[b]), (j / kSBufs - 1) & 1, abort_p, 36, j)) {
+          ok = false;
+          break;
+        }
+        if (!mbar_wait(smem_u32(&k_full[s]), (j / kKStages) & 1, abort_p, 33, j)) {
+          ok = false;
+          break;
+        }
         tc_fence_after();
-        const uint32_t sd = tmem + kTmemS + 128 * (j & 1);
+        const uint32_t sd = tmem + kTmemS + 128 * b;
         const uint64_t b0 = k_desc + (uint64_t)((s * kKBytes) >> 4);
 #pragma unroll
         for (int c = 0; c < 3; ++c)
@@ -234,35 +257,42 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(pfa::kThreads, 1)
             mma_bf16_ss<2>(sd, q_desc + (uint64_t)((c * kChunkQ + kk * 32) >> 4),
                            b0 + (uint64_t)((c * kChunkK + kk * 32) >> 4), idesc_qk,
                            (c | kk) ? 1u : 0u);
-        mma_commit_2_mc(smem_u32(&s_full[j & 1]), 3);
-        return true;
-      };
-      for (int j = 0; j < 2 && j < nblk && ok; ++j) ok = issue_qk(j);
-      for (int j = 0; j < nblk && ok; ++j) {
-        const int s = j % kStages;
-        if (!mbar_wait(smem_u32(&p_full[j & 1]), (j >> 1) & 1, abort_p, 34, j) ||
-            !mbar_wait(smem_u32(&v_full[s]), (j / kStages) & 1, abort_p, 35, j)) {
+        mma_commit_2_mc(smem_u32(&k_empty[s]), 3);
+        mma_commit_2_mc(smem_u32(&s_full[b]), 3);
+      }
+      if (!ok) {
+        mma_commit_2_mc(smem_u32(&drain_qk), 1);
+        mbar_wait_bounded(smem_u32(&drain_qk), 0, kDrainNs);
+      }
+    } else if (warp == 3 && lane == 0 && rank == 0) {
+      // ==============  PV issuer (leader)  ==============
+      // PV(j) once P(j) is in TMEM (both CTAs) and V(j) has landed; its
+      // commit on s_free[j % 3] releases the buffer for QK(j + 3) and tells
+      // the softmax that O holds PV(j).
+      const uint32_t idesc_pv = idesc_bf16_f32(256, kDV, false, true);
+      const uint64_t v_desc = sw128_desc(sV, kVBytes, 1024);
+      bool ok = true;
+      for (int j = 0; j < nblk; ++j) {
+        const int b = j % kSBufs, s = j % kVStages;
+        if (!mbar_wait(smem_u32(&p_full[b]), (j / kSBufs) & 1, abort_p, 34, j) ||
+            !mbar_wait(smem_u32(&v_full[s]), (j / kVStages) & 1, abort_p, 35, j)) {
           ok = false;
           break;
         }
         tc_fence_after();
-        const uint32_t pa = tmem + kTmemS + 128 * (j & 1);
+        const uint32_t pa = tmem + kTmemS + 128 * b;
         const uint64_t b0 = v_desc + (uint64_t)((s * kVBytes) >> 4);
 #pragma unroll
         for (int kk = 0; kk < kBlk / 16; ++kk)
           mma_bf16_ts<2>(tmem + kTmemO, pa + 8 * kk, b0 + (uint64_t)((kk * 2048) >> 4), idesc_pv,
                          (j | kk) ? 1u : 0u);
-        mma_commit_2_mc(smem_u32(&kv_empty[s]), 3);
-        mma_commit_2_mc(smem_u32(&o_done), 3);
-        mma_commit_2_mc(smem_u32(&s_free[j & 1]), 1);
+        mma_commit_2_mc(smem_u32(&v_empty[s]), 3);
+        mma_commit_2_mc(smem_u32(&s_free[b]), 3);
         if (j == nblk - 1) mma_commit_2_mc(smem_u32(&o_final), 3);
-        if (j + 2 < nblk) {
-          ok = mbar_wait(smem_u32(&s_free[j & 1]), (j >> 1) & 1, abort_p, 36, j) && issue_qk(j + 2);
-        }
       }
       if (!ok) {
-        mma_commit_2_mc(smem_u32(&drain), 1);
-        mbar_wait_bounded(smem_u32(&drain), 0, kDrainNs);
+        mma_commit_2_mc(smem_u32(&drain_pv), 1);
+        mbar_wait_bounded(smem_u32(&drain_pv), 0, kDrainNs);
       }
     }
   } else {
@@ -277,52 +307,85 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(pfa::kThreads, 1)
     float m = -INFINITY, l = 0.f;
     bool dead = false;
     for (int j = 0; j < nblk; ++j) {
-      const bool got = mbar_wait(smem_u32(&s_full[j & 1]), (j >> 1) & 1, abort_p, 37, j);
-      const uint32_t sa = tmem + lane_addr + kTmemS + 128 * (j & 1) + 64 * ch;
+      const int b = j % kSBufs;
+      const bool got = mbar_wait(smem_u32(&s_full[b]), (j / kSBufs) & 1, abort_p, 37, j);
+      const uint32_t sa = tmem + lane_addr + kTmemS + 128 * b + 64 * ch;
       const int cmax = pos - (j * kBlk + 64 * ch) + 1;   // columns c < cmax are visible
       uint32_t ra[32], rb[32];
       float mx = -INFINITY;
+      // a warp whose 32 rows see all 64 of its columns (every block off the
+      // causal diagonal) takes the mask-free path
+      const bool full = __all_sync(0xffffffffu, cmax >= 64);
       if (__all_sync(0xffffffffu, got)) {
         tc_fence_after();
         tmem_ld32(sa, ra);
         tmem_ld32(sa + 32, rb);
         tmem_wait_ld();
+        // maximum over eight independent chains
+        float acc[8];
 #pragma unroll
-        for (int c = 0; c < 32; ++c) {
-          if (c < cmax) mx = fmaxf(mx, __uint_as_float(ra[c]));
-          if (c + 32 < cmax) mx = fmaxf(mx, __uint_as_float(rb[c]));
+        for (int i = 0; i < 8; ++i) acc[i] = -INFINITY;
+        if (full) {
+#pragma unroll
+          for (int c = 0; c < 32; c += 8)
+#pragma unroll
+            for (int i = 0; i < 8; ++i)
+              acc[i] = fmaxf(acc[i], fmaxf(__uint_as_float(ra[c + i]), __uint_as_float(rb[c + i])));
+        } else {
+#pragma unroll
+          for (int c = 0; c < 32; c += 8)
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+              if (c + i < cmax) acc[i] = fmaxf(acc[i], __uint_as_float(ra[c + i]));
+              if (c + i + 32 < cmax) acc[i] = fmaxf(acc[i], __uint_as_float(rb[c + i]));
+            }
         }
+        mx = fmaxf(fmaxf(fmaxf(acc[0], acc[1]), fmaxf(acc[2], acc[3])),
+                   fmaxf(fmaxf(acc[4], acc[5]), fmaxf(acc[6], acc[7])));
       }
       red_max[j & 1][ch][row] = mx;
-      // every thread's S reads are done (P overwrites S below) and the other
-      // key half's maximum is visible
+      // both warps of these rows have read S (P overwrites it below) and the
+      // other key half's maximum is visible
       tc_fence_before();
-      if (named_bar_or(1, kSoftmaxThreads, !got || *abort_p)) { dead = true; break; }
+      if (named_bar_or(2 + quad, 64, !got || *abort_p)) { dead = true; break; }
       tc_fence_after();
       mx = fmaxf(mx, red_max[j & 1][ch ^ 1][row]);
       const float m_blk = mx * P.scale_log2;
       const bool need = m_blk > m + kRescaleLog2 || (m == -INFINITY && m_blk > -INFINITY);
       const float alpha = !need ? 1.f : (m == -INFINITY ? 0.f : ex2_approx(m - m_blk));
       const float m_use = need ? m_blk : m;
+      // p = 2^(s * scale * log2(e) - m): pairs of scores through the packed
+      // fp32 FMA, row sums over four independent packed accumulators
       uint32_t pk[32];
-      float lsum = 0.f;
+      const float2 sc2 = make_float2(P.scale_log2, P.scale_log2);
+      const float2 nm2 = make_float2(-m_use, -m_use);
+      float2 ls[4];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) ls[i] = make_float2(0.f, 0.f);
 #pragma unroll
       for (int e = 0; e < 32; ++e) {
         const uint32_t s0 = e < 16 ? ra[2 * e] : rb[2 * e - 32];
         const uint32_t s1 = e < 16 ? ra[2 * e + 1] : rb[2 * e - 31];
-        const float p0 =
-            2 * e < cmax ? ex2_approx(fmaf(__uint_as_float(s0), P.scale_log2, -m_use)) : 0.f;
-        const float p1 =
-            2 * e + 1 < cmax ? ex2_approx(fmaf(__uint_as_float(s1), P.scale_log2, -m_use)) : 0.f;
-        lsum += p0 + p1;
+        const float2 x = __ffma2_rn(make_float2(__uint_as_float(s0), __uint_as_float(s1)), sc2, nm2);
+        float p0 = ex2_approx(x.x), p1 = ex2_approx(x.y);
+        if (!full) {
+          p0 = 2 * e < cmax ? p0 : 0.f;
+          p1 = 2 * e + 1 < cmax ? p1 : 0.f;
+        }
+        ls[e & 3] = __fadd2_rn(ls[e & 3], make_float2(p0, p1));
         pk[e] = pack_bf16x2(p0, p1);
       }
+      const float2 l01 = __fadd2_rn(__fadd2_rn(ls[0], ls[1]), __fadd2_rn(ls[2], ls[3]));
+      const float lsum = l01.x + l01.y;
       // O is rescaled only when some row of this warp moved its max, after
-      // PV(j - 1).  Parity wait: S(j) implies PV(j - 2) is done and PV(j) has
-      // not been issued, so at most one phase is outstanding.
+      // PV(j - 1), whose commit is phase (j - 1) / 3 of s_free[(j - 1) % 3].
+      // Parity wait: S(j) implies PV(j - 3), the barrier's previous phase,
+      // is done, and PV(j + 2), its next, needs P(j + 2): one phase at most
+      // is outstanding.
       bool ok = true;
       if (j > 0 && __any_sync(0xffffffffu, need)) {
-        ok = __all_sync(0xffffffffu, mbar_wait(smem_u32(&o_done), (j - 1) & 1, abort_p, 38, j));
+        ok = __all_sync(0xffffffffu, mbar_wait(smem_u32(&s_free[(j - 1) % kSBufs]),
+                                               ((j - 1) / kSBufs) & 1, abort_p, 38, j));
         if (ok) {
           tc_fence_after();
 #pragma unroll 1
@@ -342,22 +405,20 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(pfa::kThreads, 1)
       // hands over nothing; the abort flag it raised stops every softmax
       // thread together at the next barrier.
       if (ok) {
-        tmem_st32(tmem + lane_addr + kTmemS + 128 * (j & 1) + 32 * ch, pk);
+        tmem_st32(tmem + lane_addr + kTmemS + 128 * b + 32 * ch, pk);
         tmem_wait_st();
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive_cluster(lead_p + 8 * (j & 1));
+        if (lane == 0) mbar_arrive_cluster(lead_p + 8 * b);
       }
       l = need ? l * alpha + lsum : l + lsum;
       m = m_use;
     }
     if (!dead) {
       // O is final once the last PV is done: o_final completes exactly once.
-      // (A parity wait on o_done could not tell PV(nblk - 2) from PV(nblk):
-      // both of the last two phases may already be complete here.)
       const bool got = mbar_wait(smem_u32(&o_final), 0, abort_p, 39, nblk);
       red_l[ch][row] = l;
-      if (!named_bar_or(1, kSoftmaxThreads, !got || *abort_p)) {
+      if (!named_bar_or(2 + quad, 64, !got || *abort_p)) {
         tc_fence_after();
         const float lt = red_l[0][row] + red_l[1][row];
         const float inv = lt > 0.f ? 1.f / lt : 0.f;
