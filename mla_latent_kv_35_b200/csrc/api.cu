@@ -117,7 +117,7 @@ mla_status launch_simt_gemm(const SimtGemmArgs& g, cudaStream_t st) {
 }
 
 struct TcGemmPlan {
-  int n_tile, n_tiles, stages, splits, k_chunks_per_split;
+  int n_tile, n_tiles, stages, splits, k_chunks_per_split, m_tiles_per_cta;
   size_t smem;
 };
 
@@ -126,11 +126,22 @@ TcGemmPlan plan_tc_gemm(int M, int N, int K, int batch, bool allow_split) {
   int n16 = ((N + 15) / 16) * 16;
   p.n_tile = n16 < 256 ? n16 : 256;
   p.n_tiles = (N + p.n_tile - 1) / p.n_tile;
-  const size_t stage_bytes = (size_t)kGemmBM * kGemmBK * 2 + (size_t)p.n_tile * kGemmBK * 2;
+  // two M tiles per CTA when M, N and K are large and the grid still has a
+  // CTA for every SM (with a short K the store epilogue, which a lone CTA
+  // on its SM does not overlap with MMAs, outweighs the halved operand
+  // traffic)
+  p.m_tiles_per_cta =
+      (p.n_tile == 256 && M >= 2 * kGemmBM && K >= 1024 &&
+       (long long)((M + 2 * kGemmBM - 1) / (2 * kGemmBM)) * p.n_tiles * batch >= sm_count())
+          ? 2
+          : 1;
+  const size_t stage_bytes =
+      (size_t)p.m_tiles_per_cta * kGemmBM * kGemmBK * 2 + (size_t)p.n_tile * kGemmBK * 2;
   const int k_chunks = (K + kGemmBK - 1) / kGemmBK;
   p.splits = 1;
-  const long long ctas = (long long)((M + kGemmBM - 1) / kGemmBM) * p.n_tiles * batch;
-  if (allow_split) {
+  const int bm = kGemmBM * p.m_tiles_per_cta;
+  const long long ctas = (long long)((M + bm - 1) / bm) * p.n_tiles * batch;
+  if (allow_split && p.m_tiles_per_cta == 1) {
     // as many splits as keep the grid within two CTAs per SM (one wave: a
     // partial second wave would double the time of its SMs)
     const long long target = 2LL * sm_count();
@@ -142,7 +153,9 @@ TcGemmPlan plan_tc_gemm(int M, int N, int K, int batch, bool allow_split) {
   // has at most one CTA per SM, ~96 KB (two CTAs per SM) otherwise, and
   // never more stages than the CTA has chunks (a short K leaves room for
   // more CTAs per SM instead).
-  const size_t budget = ctas * p.splits <= sm_count() ? 200 * 1024 : 96 * 1024;
+  // (two M tiles take all 512 TMEM columns: one CTA per SM)
+  const size_t budget =
+      (p.m_tiles_per_cta == 2 || ctas * p.splits <= sm_count()) ? 200 * 1024 : 96 * 1024;
   int st = (int)(budget / stage_bytes);
   st = st < 2 ? 2 : (st > 8 ? 8 : st);
   if (st > p.k_chunks_per_split) st = p.k_chunks_per_split < 2 ? 2 : p.k_chunks_per_split;
@@ -197,6 +210,12 @@ mla_status launch_tc_gemm(const void* A, bool a_mn, long long as_b, const void* 
   g.k_chunks_per_split = p.k_chunks_per_split;
   g.stages = p.stages;
   g.out = out; g.ob = ob; g.on = on; g.om = om;
+  // The 16-byte stores cover 8 consecutive m from a multiple of 8: whole
+  // pieces only when M is a multiple of 8 too.
+  g.vec_out = (out_kind == kOutBf16 && om == 1 && (on % 8) == 0 && (ob % 8) == 0 &&
+               (M % 8) == 0 && aligned16(out))
+                  ? 1
+                  : 0;
   g.os = (long long)M * N;
   g.batch = batch;
   g.aux = PreAttnAux{};
@@ -204,14 +223,17 @@ mla_status launch_tc_gemm(const void* A, bool a_mn, long long as_b, const void* 
   if (aux != nullptr && aux->n_items > 0) {
     // enough extra z-slices for about 2 work items per thread
     g.aux = *aux;
-    const long long per_slice = (long long)((M + kGemmBM - 1) / kGemmBM) * p.n_tiles * p.splits * 128;
+    const long long per_slice =
+        (long long)((M + kGemmBM * p.m_tiles_per_cta - 1) / (kGemmBM * p.m_tiles_per_cta)) *
+        p.n_tiles * p.splits * 128;
     aux_z = (int)std::min<long long>(4096, (aux->n_items + 2 * per_slice - 1) / (2 * per_slice));
   }
   g.aux_z = aux_z;
-  dim3 grid((M + kGemmBM - 1) / kGemmBM, p.n_tiles * p.splits, batch + aux_z);
+  const int bm = kGemmBM * p.m_tiles_per_cta;
+  dim3 grid(p.n_tiles * p.splits, (M + bm - 1) / bm, batch + aux_z);
 #define MLA_GEMM_LAUNCH(AMN, OUT)                                                              \
   do {                                                                                         \
-    auto kfn = gemm_tc_kernel<AMN, OUT>;                                                       \
+    auto kfn = p.m_tiles_per_cta == 2 ? gemm_tc_kernel<AMN, OUT, 2> : gemm_tc_kernel<AMN, OUT, 1>; \
     if (cudaFuncSetAttribute(kfn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)p.smem) != \
         cudaSuccess)                                                                           \
       return MLA_ERR_CUDA;                                                                     \
@@ -359,7 +381,8 @@ mla_status mla_rope(const mla_dims* dims, const void* x, int xs_tok, int xs_head
   if (!dims_ok(dims) || T < 0 || n_heads_x < 0) return MLA_ERR_INVALID_ARG;
   if (T == 0 || n_heads_x == 0 || dims->d_rope == 0) return MLA_OK;
   if (!x || !y || !pos) return MLA_ERR_INVALID_ARG;
-  const long long n = (long long)T * n_heads_x * (dims->d_rope / 2);
+  const long long n =
+      (long long)T * ((n_heads_x + kRopeGroup - 1) / kRopeGroup) * (dims->d_rope / 2);
   const int blk = 256;
   const long long grid = (n + blk - 1) / blk;
   cudaStream_t st = as_stream(stream);

@@ -17,6 +17,16 @@
 // S-stage ring; warp 1 allocates TMEM and its lane 0 issues the MMAs; after
 // the last MMA all four warps read the accumulator (TMEM lane = output row)
 // and store it.
+//
+// kMT = 2 gives a CTA two 128-row M tiles against the same token tile (two
+// accumulators of BN columns, 512 TMEM columns at BN = 256): each token
+// tile brought into shared memory serves twice the MMA work, which halves
+// the operand traffic per FLOP when both M and N are large (prefill-sized
+// GEMMs, whose operands are served from L2).
+//
+// Grid: x = token tile (fastest) x K split, y = M tile, z = batch entry.
+// CTAs that run together share their weight tile, so each weight tile is
+// read from HBM once and served to the token tiles from L2.
 #pragma once
 
 #include "common.cuh"
@@ -28,6 +38,7 @@ enum GemmOut : int { kOutBf16 = 0, kOutF32 = 1, kOutF32Split = 2 };
 
 struct GemmTcArgs {
   int M, N, K;           // per batch entry
+  int vec_out;           // bf16 out with om == 1, on and ob multiples of 8, 16-byte aligned
   int n_tile;            // BN, multiple of 16, <= 256
   int n_tiles;           // ceil(N / BN)
   int k_chunks_per_split;
@@ -43,7 +54,7 @@ struct GemmTcArgs {
 constexpr int kGemmBM = 128;
 constexpr int kGemmBK = 64;  // 64 bf16 = one 128-byte swizzle row
 
-template <bool kAmn, int kOut>
+template <bool kAmn, int kOut, int kMT>
 __global__ void __launch_bounds__(128, 1) gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA,
                                                          const __grid_constant__ CUtensorMap tmX,
                                                          GemmTcArgs g) {
@@ -64,9 +75,9 @@ __global__ void __launch_bounds__(128, 1) gemm_tc_kernel(const __grid_constant__
   }
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int m0 = blockIdx.x * kGemmBM;
-  const int n_tile_idx = blockIdx.y % g.n_tiles;
-  const int split = blockIdx.y / g.n_tiles;
+  const int m0 = blockIdx.y * (kGemmBM * kMT);
+  const int n_tile_idx = blockIdx.x % g.n_tiles;
+  const int split = blockIdx.x / g.n_tiles;
   const int n0 = n_tile_idx * g.n_tile;
   const int b = blockIdx.z - g.aux_z;
   const int BN = g.n_tile;
@@ -76,7 +87,8 @@ __global__ void __launch_bounds__(128, 1) gemm_tc_kernel(const __grid_constant__
   const int kc1 = min(k_chunks_total, kc0 + g.k_chunks_per_split);
   const int nk = max(0, kc1 - kc0);
 
-  const uint32_t a_bytes = kGemmBM * kGemmBK * 2;  // 16 KB
+  const uint32_t a_tile = kGemmBM * kGemmBK * 2;   // 16 KB per M tile
+  const uint32_t a_bytes = kMT * a_tile;
   const uint32_t x_bytes = BN * kGemmBK * 2;
   const uint32_t stage_bytes = a_bytes + x_bytes;
   const uint32_t smem_base = (smem_u32(smem_raw) + 1023u) & ~1023u;
@@ -93,7 +105,7 @@ __global__ void __launch_bounds__(128, 1) gemm_tc_kernel(const __grid_constant__
     tma_prefetch_desc(&tmX);
   }
   uint32_t tmem_cols = 32;
-  while ((int)tmem_cols < BN) tmem_cols <<= 1;
+  while ((int)tmem_cols < BN * kMT) tmem_cols <<= 1;
   if (warp == 1) {
     tmem_alloc<1>(smem_u32(&tmem_base_sh), tmem_cols);
     tmem_relinquish<1>();
@@ -114,11 +126,15 @@ __global__ void __launch_bounds__(128, 1) gemm_tc_kernel(const __grid_constant__
       const uint32_t sa = smem_base + s * stage_bytes;
       mbar_expect_tx(fb, stage_bytes);
       const int k = (kc0 + i) * kGemmBK;
-      if constexpr (kAmn) {
-        tma_load_3d(sa, &tmA, m0, k, b, fb);
-        tma_load_3d(sa + a_bytes / 2, &tmA, m0 + 64, k, b, fb);
-      } else {
-        tma_load_3d(sa, &tmA, k, m0, b, fb);
+#pragma unroll
+      for (int mt = 0; mt < kMT; ++mt) {
+        const int mr = m0 + mt * kGemmBM;
+        if constexpr (kAmn) {
+          tma_load_3d(sa + mt * a_tile, &tmA, mr, k, b, fb);
+          tma_load_3d(sa + mt * a_tile + a_tile / 2, &tmA, mr + 64, k, b, fb);
+        } else {
+          tma_load_3d(sa + mt * a_tile, &tmA, k, mr, b, fb);
+        }
       }
       tma_load_3d(sa + a_bytes, &tmX, k, n0, b, fb);
       ++issued;
@@ -140,13 +156,16 @@ __global__ void __launch_bounds__(128, 1) gemm_tc_kernel(const __grid_constant__
       const uint32_t sx = sa + a_bytes;
 #pragma unroll
       for (int kk = 0; kk < kGemmBK / 16; ++kk) {
-        uint64_t ad;
-        if constexpr (kAmn)
-          ad = sw128_desc(sa + kk * 2048, 8192, 1024);  // 16 K-rows of 128 B per step
-        else
-          ad = sw128_desc(sa + kk * 32, 16, 1024);      // 16 K-elements = 32 B per step
         const uint64_t xd = sw128_desc(sx + kk * 32, 16, 1024);
-        mma_bf16_ss<1>(tmem, ad, xd, idesc, (i > 0 || kk > 0) ? 1u : 0u);
+#pragma unroll
+        for (int mt = 0; mt < kMT; ++mt) {
+          uint64_t ad;
+          if constexpr (kAmn)
+            ad = sw128_desc(sa + mt * a_tile + kk * 2048, 8192, 1024);  // 16 K-rows of 128 B
+          else
+            ad = sw128_desc(sa + mt * a_tile + kk * 32, 16, 1024);      // 16 K-elements = 32 B
+          mma_bf16_ss<1>(tmem + mt * BN, ad, xd, idesc, (i > 0 || kk > 0) ? 1u : 0u);
+        }
       }
       mma_commit_1(smem_u32(&empty_bar[s]));
     }
@@ -158,12 +177,50 @@ __global__ void __launch_bounds__(128, 1) gemm_tc_kernel(const __grid_constant__
   // TMEM loads are warp-collective: every thread takes the same branch
   const bool have =
       __syncthreads_and(nk > 0 && mbar_wait(smem_u32(&acc_bar), 0, abort_p, 23, 0)) != 0;
-  if (have) {
+  if (have && kOut == kOutBf16 && g.vec_out) {
+    // Rows m are TMEM lanes, one per thread, but the output has m
+    // contiguous: each warp turns its 32 x 32 tiles around in shared memory
+    // (the operand ring, idle once the last MMA has completed) and stores
+    // 16-byte pieces of 8 consecutive m, 8 token rows per instruction.
     tc_fence_after();
-    const int m = m0 + warp * 32 + lane;
+    const uint32_t scratch = smem_base + warp * 2048;   // [32 tokens][32 m] bf16
+    for (int mt = 0; mt < kMT; ++mt) {
+      const int mw = m0 + mt * kGemmBM + warp * 32;       // this warp's first row
+      for (int c0 = 0; c0 < BN; c0 += 32) {
+        uint32_t r[32];
+        tmem_ld32(tmem + ((uint32_t)(warp * 32) << 16) + mt * BN + c0, r);
+        tmem_wait_ld();
+#pragma unroll
+        for (int i = 0; i < 32; ++i) {
+          const __nv_bfloat16 v = __float2bfloat16_rn(__uint_as_float(r[i]));
+          asm volatile("st.shared.b16 [%0], %1;" ::"r"(scratch + i * 64 + lane * 2),
+                       "h"(*reinterpret_cast<const uint16_t*>(&v))
+                       : "memory");
+        }
+        __syncwarp();
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          const int nl = q * 8 + (lane >> 2), ml = (lane & 3) * 8;
+          uint4 v;
+          asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];"
+                       : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+                       : "r"(scratch + nl * 64 + ml * 2)
+                       : "memory");
+          const int n = n0 + c0 + nl, m = mw + ml;
+          if (c0 + nl < BN && n < g.N && m < g.M)
+            *reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(g.out) + (long long)b * g.ob +
+                                      (long long)n * g.on + m) = v;
+        }
+        __syncwarp();
+      }
+    }
+  } else if (have) {
+    tc_fence_after();
+    for (int mt = 0; mt < kMT; ++mt)
     for (int c0 = 0; c0 < BN; c0 += 32) {
+      const int m = m0 + mt * kGemmBM + warp * 32 + lane;
       uint32_t r[32];
-      tmem_ld32(tmem + ((uint32_t)(warp * 32) << 16) + c0, r);
+      tmem_ld32(tmem + ((uint32_t)(warp * 32) << 16) + mt * BN + c0, r);
       tmem_wait_ld();
       if (m < g.M) {
 #pragma unroll
@@ -184,7 +241,8 @@ __global__ void __launch_bounds__(128, 1) gemm_tc_kernel(const __grid_constant__
     }
   } else if (nk == 0) {
     // empty K range: the product is zero
-    const int m = m0 + warp * 32 + lane;
+    for (int mt = 0; mt < kMT; ++mt) {
+    const int m = m0 + mt * kGemmBM + warp * 32 + lane;
     if (m < g.M)
       for (int i = 0; i < BN; ++i) {
         const int n = n0 + i;
@@ -198,6 +256,7 @@ __global__ void __launch_bounds__(128, 1) gemm_tc_kernel(const __grid_constant__
             static_cast<float*>(g.out)[o + split * g.os] = 0.f;
         }
       }
+    }
   }
   tc_fence_before();
   __syncthreads();

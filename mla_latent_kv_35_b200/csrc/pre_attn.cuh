@@ -36,18 +36,6 @@ __device__ __forceinline__ void rope_rotate(float x0, float x1, float c, float s
   y1 = __fmaf_rn(x0, s, __fmul_rn(x1, c));
 }
 
-// Rotate pair k of the vector at x (position p, width d_rope) into y.  x and
-// y may alias.
-template <typename T>
-__device__ __forceinline__ void rope_pair(const T* x, T* y, int k, int p, int d_rope,
-                                          double base) {
-  float c, s, y0, y1;
-  rope_cos_sin(k, p, d_rope, base, c, s);
-  rope_rotate(to_f32(x[2 * k]), to_f32(x[2 * k + 1]), c, s, y0, y1);
-  y[2 * k] = from_f32<T>(y0);
-  y[2 * k + 1] = from_f32<T>(y1);
-}
-
 // Pool row of new token t, or nullptr (raising MLA_ERR_BOUNDS) when its
 // batch index, position or page id falls outside the page table or pool.
 template <typename E>

@@ -76,20 +76,36 @@ __global__ void __launch_bounds__(256) simt_gemm_kernel(SimtGemmArgs g) {
 }
 
 // ---------------------------------------------------------------------------
-// RoPE: rotate consecutive pairs by pos * base^(-2k/d); angle in fp64.
+// RoPE: rotate consecutive pairs by pos * base^(-2k/d); angle in fp64.  One
+// thread per (token, group of 8 heads, pair k), k fastest: the angle's cos
+// and sin are formed once and turn pair k of all heads of the group.
 // ---------------------------------------------------------------------------
+constexpr int kRopeGroup = 8;
+
 template <typename T>
 __global__ void rope_kernel(const T* x, long long xs_tok, long long xs_head, int nh, T* y,
                             long long ys_tok, long long ys_head, const int32_t* pos, int Tn,
                             int d_rope, double base) {
   const int half = d_rope / 2;
+  const int ng = (nh + kRopeGroup - 1) / kRopeGroup;
   long long idx = (long long)blockIdx.x * blockDim.x + threadIdx.x;
-  long long total = (long long)Tn * nh * half;
+  long long total = (long long)Tn * ng * half;
   if (idx >= total) return;
   const int k = (int)(idx % half);
-  const int h = (int)((idx / half) % nh);
-  const int t = (int)(idx / ((long long)half * nh));
-  rope_pair(x + t * xs_tok + h * xs_head, y + t * ys_tok + h * ys_head, k, pos[t], d_rope, base);
+  const int g = (int)((idx / half) % ng);
+  const int t = (int)(idx / ((long long)half * ng));
+  float c, s;
+  rope_cos_sin(k, pos[t], d_rope, base, c, s);
+  for (int i = 0; i < kRopeGroup; ++i) {
+    const int h = g * kRopeGroup + i;
+    if (h >= nh) break;
+    const T* xp = x + t * xs_tok + h * xs_head;
+    T* yp = y + t * ys_tok + h * ys_head;
+    float y0, y1;
+    rope_rotate(to_f32(xp[2 * k]), to_f32(xp[2 * k + 1]), c, s, y0, y1);
+    yp[2 * k] = from_f32<T>(y0);
+    yp[2 * k + 1] = from_f32<T>(y1);
+  }
 }
 
 // ---------------------------------------------------------------------------
