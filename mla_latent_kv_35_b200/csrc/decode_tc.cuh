@@ -48,6 +48,8 @@
 //     the scores of one row on one page.  Row maxima of the four pages meet
 //     in shared memory.  The running max is rescaled lazily: O is rescaled
 //     in TMEM only when a row's max grows by more than 2^8, warp-uniformly.
+//     Full pages take a path without masks; maxima and row sums run in
+//     independent chains and scores go through the packed fp32 FMA.
 //     P goes to TMEM over S: warps w and w ^ 2 hold the two token halves of
 //     the same rows and swap them through an 8 KB shared buffer, one warp
 //     pair per round, four rounds.  P(j) waits for nothing from PV(j - 1):
@@ -569,24 +571,43 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(dtc::kThreads, 1)
         const bool got = mbar_wait(smem_u32(&s_full[j & 1]), (j >> 1) & 1, abort_p, 7, j);
         float mx = -INFINITY;
         const int cmax = limit - (x * kBlk + pb * kPage);  // columns c < cmax are visible
-        // this thread's 64 scores, read from TMEM 32 at a time (twice: for
-        // the max, then for the exponentials), which keeps half the
-        // registers of holding all 64 across the max exchange; invisible
-        // columns (past the context, causally hidden, or slots of a partial
-        // page whose contents are not cache) count as -inf
+        // a warp whose 32 rows see all 64 of their columns (every block but
+        // a sequence's last, or a causal edge) takes the mask-free path
+        const bool full = __all_sync(0xffffffffu, cmax >= 64);
+        // this thread's 64 scores, read from TMEM (twice: for the max, then
+        // for the exponentials, which keeps the registers of holding all 64
+        // across the max exchange free); invisible columns (past the
+        // context, causally hidden, or slots of a partial page whose contents
+        // are not cache) count as -inf
         const uint32_t sa = tmem + lane_addr + kTmemS + 128 * (j & 1) + 64 * ch;
         const bool all_got = __all_sync(0xffffffffu, got);
         if (all_got) {
           tc_fence_after();
+          uint32_t ra[32], rb[32];
+          tmem_ld32(sa, ra);
+          tmem_ld32(sa + 32, rb);
+          tmem_wait_ld();
+          // maximum over eight independent chains
+          float acc[8];
 #pragma unroll
-          for (int hf = 0; hf < 2; ++hf) {
-            uint32_t r[32];
-            tmem_ld32(sa + 32 * hf, r);
-            tmem_wait_ld();
+          for (int i = 0; i < 8; ++i) acc[i] = -INFINITY;
+          if (full) {
 #pragma unroll
-            for (int c = 0; c < 32; ++c)
-              if (32 * hf + c < cmax) mx = fmaxf(mx, __uint_as_float(r[c]));
+            for (int c = 0; c < 32; c += 8)
+#pragma unroll
+              for (int i = 0; i < 8; ++i)
+                acc[i] = fmaxf(acc[i], fmaxf(__uint_as_float(ra[c + i]), __uint_as_float(rb[c + i])));
+          } else {
+#pragma unroll
+            for (int c = 0; c < 32; c += 8)
+#pragma unroll
+              for (int i = 0; i < 8; ++i) {
+                if (c + i < cmax) acc[i] = fmaxf(acc[i], __uint_as_float(ra[c + i]));
+                if (c + i + 32 < cmax) acc[i] = fmaxf(acc[i], __uint_as_float(rb[c + i]));
+              }
           }
+          mx = fmaxf(fmaxf(fmaxf(acc[0], acc[1]), fmaxf(acc[2], acc[3])),
+                     fmaxf(fmaxf(acc[4], acc[5]), fmaxf(acc[6], acc[7])));
         }
         red_max[pb][h] = mx;
         // one barrier: the other pages' maxima visible, and everyone agrees
@@ -602,26 +623,36 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(dtc::kThreads, 1)
         const bool need = m_blk > m + kRescaleLog2 || (m == -INFINITY && m_blk > -INFINITY);
         const float alpha = !need ? 1.f : (m == -INFINITY ? 0.f : ex2_approx(m - m_blk));
         const float m_use = need ? m_blk : m;
+        // p = 2^(s * scale * log2(e) - m): pairs of scores through the packed
+        // fp32 FMA, row sums over four independent packed accumulators
         uint32_t pk[32];
-        float lsum = 0.f;
-#pragma unroll
-        for (int hf = 0; hf < 2; ++hf) {
-          uint32_t r[32];
-          tmem_ld32(sa + 32 * hf, r);
+        float lsum;
+        {
+          uint32_t ra[32], rb[32];
+          tmem_ld32(sa, ra);
+          tmem_ld32(sa + 32, rb);
           tmem_wait_ld();
+          const float2 sc2 = make_float2(P.scale_log2, P.scale_log2);
+          const float2 nm2 = make_float2(-m_use, -m_use);
+          float2 ls[4];
 #pragma unroll
-          for (int e = 0; e < 16; ++e) {
-            const int c0 = 32 * hf + 2 * e;
-            const float p0 =
-                c0 < cmax ? ex2_approx(fmaf(__uint_as_float(r[2 * e]), P.scale_log2, -m_use))
-                          : 0.f;
-            const float p1 =
-                c0 + 1 < cmax
-                    ? ex2_approx(fmaf(__uint_as_float(r[2 * e + 1]), P.scale_log2, -m_use))
-                    : 0.f;
-            lsum += p0 + p1;
-            pk[16 * hf + e] = pack_bf16x2(p0, p1);
+          for (int i = 0; i < 4; ++i) ls[i] = make_float2(0.f, 0.f);
+#pragma unroll
+          for (int e = 0; e < 32; ++e) {
+            const uint32_t s0 = e < 16 ? ra[2 * e] : rb[2 * e - 32];
+            const uint32_t s1 = e < 16 ? ra[2 * e + 1] : rb[2 * e - 31];
+            const float2 xx =
+                __ffma2_rn(make_float2(__uint_as_float(s0), __uint_as_float(s1)), sc2, nm2);
+            float p0 = ex2_approx(xx.x), p1 = ex2_approx(xx.y);
+            if (!full) {
+              p0 = 2 * e < cmax ? p0 : 0.f;
+              p1 = 2 * e + 1 < cmax ? p1 : 0.f;
+            }
+            ls[e & 3] = __fadd2_rn(ls[e & 3], make_float2(p0, p1));
+            pk[e] = pack_bf16x2(p0, p1);
           }
+          const float2 l01 = __fadd2_rn(__fadd2_rn(ls[0], ls[1]), __fadd2_rn(ls[2], ls[3]));
+          lsum = l01.x + l01.y;
         }
         // O is rescaled only when some row of this warp moved its max; PV of
         // the previous block accumulates into O and must be done first.

@@ -44,8 +44,9 @@
 //     memory, each warp pair on a named barrier of its own.  Blocks off the
 //     causal diagonal take a path without masks; maxima and row sums run in
 //     independent chains, scores go through the packed fp32 FMA, and a share
-//     of the exponentials is evaluated on the FMA pipe (exp2_poly2).  The running max is rescaled lazily (O in TMEM is rescaled
-//     only when a row's max grows by more than 2^8, after PV(j - 1)).
+//     of the exponentials is evaluated on the FMA pipe (exp2_poly2).  The
+//     running max is rescaled lazily (O in TMEM is rescaled only when a row's
+//     max grows by more than 2^8, after PV(j - 1)).
 //   * Two threads of the leader issue the MMAs: lane 0 of warp 1 the QK
 //     stream, lane 0 of warp 3 the PV stream, so that neither stream's
 //     barrier waits hold up the other's MMAs.
@@ -96,38 +97,11 @@ constexpr uint32_t kTmemS = 128;     // S_b / P_b at [128 + 128b, +128), b < 3
 constexpr float kRescaleLog2 = 8.0f;
 }  // namespace pfa
 
-// 2^x without the MUFU unit, for a share of the softmax exponentials (the
-// MUFU pipe, 16 results per cycle per SM, would otherwise bound the
-// softmax): x = n + f with n = round(x), |f| <= 1/2 (n read from the low
-// mantissa bits of x + 1.5 * 2^23), 2^f by a cubic, n added to the exponent
-// field.  The cubic's coefficients were fitted to 2^f on [-1/2, 1/2] by
-// iteratively reweighted least squares for relative error: at most 7.5e-5
-// relative error in fp32 Horner evaluation, far below the 2^-9 rounding of P
-// to bf16.  x is clamped to -125, where 2^x is still a normal number.
 // One pair of exponentials in MLA_EXP2_POLY_EVERY goes to exp2_poly2 (0: none).
 #ifndef MLA_EXP2_POLY_EVERY
 #define MLA_EXP2_POLY_EVERY 4
 #endif
 
-__device__ constexpr float kExp2Poly[4] = {0.9999280571937561f, 0.6932609677314758f, 0.2426111251115799f,
-                                           0.0551716648042202f};
-
-__device__ __forceinline__ float2 exp2_poly2(float2 x) {
-  constexpr float kRound = 12582912.0f;   // 1.5 * 2^23
-  x.x = fmaxf(x.x, -125.0f);
-  x.y = fmaxf(x.y, -125.0f);
-  const float2 t = __fadd2_rn(x, make_float2(kRound, kRound));
-  const float2 n = __fadd2_rn(t, make_float2(-kRound, -kRound));
-  const float2 f = __ffma2_rn(n, make_float2(-1.0f, -1.0f), x);   // exact
-  float2 p = __ffma2_rn(make_float2(kExp2Poly[3], kExp2Poly[3]), f,
-                        make_float2(kExp2Poly[2], kExp2Poly[2]));
-  p = __ffma2_rn(p, f, make_float2(kExp2Poly[1], kExp2Poly[1]));
-  p = __ffma2_rn(p, f, make_float2(kExp2Poly[0], kExp2Poly[0]));
-  const uint32_t ex = (__float_as_uint(t.x) - 0x4B400000u) << 23;
-  const uint32_t ey = (__float_as_uint(t.y) - 0x4B400000u) << 23;
-  return make_float2(__uint_as_float(__float_as_uint(p.x) + ex),
-                     __uint_as_float(__float_as_uint(p.y) + ey));
-}
 
 struct PrefillParams {
   __nv_bfloat16* o;   // [T][H][128]

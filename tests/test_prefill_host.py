@@ -9,7 +9,7 @@ ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 
 
 def _poly():
-    src = open(os.path.join(ROOT, "mla_latent_kv_35_b200", "csrc", "prefill_tc.cuh")).read()
+    src = open(os.path.join(ROOT, "mla_latent_kv_35_b200", "csrc", "common.cuh")).read()
     m = re.search(r"kExp2Poly\[4\]\s*=\s*\{([^}]*)\}", src)
     assert m, "kExp2Poly not found"
     return [np.float32(float(x.strip().rstrip("f"))) for x in m.group(1).split(",")]
