@@ -152,10 +152,10 @@ def code_digest(paths):
     return h.hexdigest()
 
 
-def _traffic_for(kernel_src_paths):
-    """ncu DRAM bytes per decode call recorded in profiles/, if the kernel
-    code is unchanged since the capture (else None)."""
-    path = os.path.join(ROOT, "profiles", "decode_tc_traffic.json")
+def _traffic_for(kernel_src_paths, record="decode_tc_traffic.json"):
+    """ncu DRAM bytes per call recorded in profiles/, if the kernel code is
+    unchanged since the capture (else None)."""
+    path = os.path.join(ROOT, "profiles", record)
     try:
         with open(path) as f:
             rec = json.load(f)
@@ -702,7 +702,10 @@ def run_gpu_prefill(args, w):
                      "achieved": achieved, "peak": tf_peak, "unit": "TFLOP/s",
                      "frac": achieved / tf_peak, "peak_source": peak_kind + " (bf16 burst)",
                      "alg_flops_per_launch": fl["attention"], "kernel_ms": t_att,
-                     "traffic": None},
+                     "traffic": _traffic_for([os.path.join(ROOT, "mla_latent_kv_35_b200", "csrc",
+                                                           "prefill_tc.cuh")],
+                                             "prefill_attn_traffic.json")
+                     if w.H == 128 else None},
         "e2e": {"value": whole_job_rate(T, world, t_e2e), "unit": "tokens/s",
                 "ms_per_step": t_e2e, "pipelined": False,
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},

@@ -77,10 +77,10 @@ __global__ void __launch_bounds__(256) simt_gemm_kernel(SimtGemmArgs g) {
 
 // ---------------------------------------------------------------------------
 // RoPE: rotate consecutive pairs by pos * base^(-2k/d); angle in fp64.  One
-// thread per (token, group of 8 heads, pair k), k fastest: the angle's cos
+// thread per (token, group of 32 heads, pair k), k fastest: the angle's cos
 // and sin are formed once and turn pair k of all heads of the group.
 // ---------------------------------------------------------------------------
-constexpr int kRopeGroup = 8;
+constexpr int kRopeGroup = 32;
 
 template <typename T>
 __global__ void rope_kernel(const T* x, long long xs_tok, long long xs_head, int nh, T* y,
