@@ -116,6 +116,11 @@ mla_status launch_simt_gemm(const SimtGemmArgs& g, cudaStream_t st) {
   return check_launch();
 }
 
+// Smallest K for two M tiles per CTA (see plan_tc_gemm).
+#ifndef MLA_GEMM_MT2_MIN_K
+#define MLA_GEMM_MT2_MIN_K 1024
+#endif
+
 struct TcGemmPlan {
   int n_tile, n_tiles, stages, splits, k_chunks_per_split, m_tiles_per_cta;
   size_t smem;
@@ -131,7 +136,7 @@ TcGemmPlan plan_tc_gemm(int M, int N, int K, int batch, bool allow_split) {
   // on its SM does not overlap with MMAs, outweighs the halved operand
   // traffic)
   p.m_tiles_per_cta =
-      (p.n_tile == 256 && M >= 2 * kGemmBM && K >= 1024 &&
+      (p.n_tile == 256 && M >= 2 * kGemmBM && K >= MLA_GEMM_MT2_MIN_K &&
        (long long)((M + 2 * kGemmBM - 1) / (2 * kGemmBM)) * p.n_tiles * batch >= sm_count())
           ? 2
           : 1;

@@ -157,9 +157,11 @@ class MLADecodeLayer:
     # ------------------------------------------------------------------
     # chunked prefill (non-absorbed)
     # ------------------------------------------------------------------
-    def prefill_buffers(self, T: int, L: int):
-        """Device buffers of one prefill chunk of T tokens ending at context L."""
-        key = ("prefill", T, L)
+    def prefill_buffers(self, T: int, L: int, slot: int = 0):
+        """Device buffers of one prefill chunk of T tokens ending at context L
+        (slot: an independent second set, for chunks that overlap in
+        PrefillPipeline)."""
+        key = ("prefill", T, L, slot)
         if key not in self._bufs:
             d = self.dims
             dev, dt = self.device, d.torch_dtype
@@ -175,7 +177,7 @@ class MLADecodeLayer:
             )
         return self._bufs[key]
 
-    def prefill_chunk(self, h, pos, batch_idx, b: int, T: int, L: int):
+    def prefill_chunk(self, h, pos, batch_idx, b: int, T: int, L: int, slot: int = 0):
         """Prefill T new tokens of sequence b, at positions L - T .. L - 1.
 
         h [T, d_model] device; pos int32 [T] = L - T .. L - 1 and batch_idx
@@ -200,7 +202,7 @@ class MLADecodeLayer:
         H, dn, dc = d.n_heads, d.d_nope, d.d_latent
         Y, dqk = self.Y, self.dqk
         off_c = H * dqk
-        bf = self.prefill_buffers(T, L)
+        bf = self.prefill_buffers(T, L, slot)
         y = bf["y"]
         _b.mla_project(d, h, self.W_A0, y, T, d.d_model, Y)
         _b.mla_rope(d, y[:, dn:], Y, dqk, H, y[:, dn:], Y, dqk, pos, T)
@@ -303,6 +305,74 @@ class DecodePipeline:
 
     def wait(self):
         """Block the host until every submitted step's output is on the host."""
+        for sl in self.slots:
+            sl["out_read"].synchronize()
+
+
+class PrefillPipeline:
+    """Chunked prefill that overlaps each chunk's host transfers with compute.
+
+    Two slots, each with its own input buffers and chunk buffers.  submit()
+    enqueues chunk i in slot i % 2: h, positions and batch indices are copied
+    from pinned host memory on an upload stream while the previous chunk
+    computes; the chunk runs on the current stream once its inputs are in
+    (and the slot's previous output has left); its `out` goes back on a
+    download stream while the next chunk computes.  Chunks of one sequence
+    still run in order on the compute stream, so each sees the cache rows the
+    previous one appended.
+    """
+
+    def __init__(self, layer: MLADecodeLayer, b: int, T: int, L: int):
+        d = layer.dims
+        dev = layer.device
+        self.layer, self.b, self.T, self.L = layer, b, T, L
+        self.up = torch.cuda.Stream(dev)
+        self.down = torch.cuda.Stream(dev)
+        self.slots = []
+        for s in range(2):
+            layer.prefill_buffers(T, L, slot=s)
+            self.slots.append(dict(
+                h=torch.empty((T, d.d_model), dtype=d.torch_dtype, device=dev),
+                bi=torch.empty((T,), dtype=torch.int32, device=dev),
+                pos=torch.empty((T,), dtype=torch.int32, device=dev),
+                inputs_in=torch.cuda.Event(), done=torch.cuda.Event(),
+                out_read=torch.cuda.Event()))
+        self.i = 0
+
+    def submit(self, h_host, bi_host, pos_host, out_host):
+        """Enqueue one chunk: h_host [T, d_model] (layer dtype), bi_host and
+        pos_host int32 [T] and out_host [T, d_model] (layer dtype) are pinned
+        host tensors; out_host holds the chunk's output once its `out_read`
+        event (returned) has completed."""
+        s = self.i % 2
+        sl = self.slots[s]
+        self.i += 1
+        compute = torch.cuda.current_stream(self.layer.device)
+        self.up.wait_event(sl["done"])
+        with torch.cuda.stream(self.up):
+            sl["h"].copy_(h_host, non_blocking=True)
+            sl["bi"].copy_(bi_host, non_blocking=True)
+            sl["pos"].copy_(pos_host, non_blocking=True)
+            sl["inputs_in"].record(self.up)
+        compute.wait_event(sl["inputs_in"])
+        compute.wait_event(sl["out_read"])
+        bf = self.layer.prefill_chunk(sl["h"], sl["pos"], sl["bi"], self.b, self.T, self.L,
+                                      slot=s)
+        sl["done"].record(compute)
+        self.down.wait_event(sl["done"])
+        with torch.cuda.stream(self.down):
+            out_host.copy_(bf["out"], non_blocking=True)
+            sl["out_read"].record(self.down)
+        return sl["out_read"]
+
+    def drain(self, stream=None):
+        """Make `stream` (default: the current one) wait for every submitted
+        chunk's output transfer."""
+        stream = stream or torch.cuda.current_stream(self.layer.device)
+        for sl in self.slots:
+            stream.wait_event(sl["out_read"])
+
+    def wait(self):
         for sl in self.slots:
             sl["out_read"].synchronize()
 

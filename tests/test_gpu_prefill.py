@@ -161,3 +161,70 @@ def test_prefill_rejects_bad_arguments():
     assert e.value.code == 2
     torch.cuda.synchronize()
     assert status() == 0
+
+
+@gpu
+def test_prefill_pipeline_matches_direct_chunks():
+    """PrefillPipeline (inputs copied in and outputs copied out on side
+    streams, two slots) gives the bits of a direct prefill_chunk call, for
+    several chunks in flight."""
+    from mla_latent_kv_35_b200.engine import PrefillPipeline
+    w = wl.workload("prefill", H=16, S_q=200, ctx=(500,))
+    W, layer, bf, h, table = _run(w)
+    ref = bf["out"].clone()
+    T, L = w.S_q, w.ctx[0]
+    bi, pos = wl.positions(w)
+    d = MLADims.of(w)
+    h_host = torch.from_numpy(h.reshape(T, -1)).to(d.torch_dtype).pin_memory()
+    bi_host = torch.from_numpy(bi).pin_memory()
+    pos_host = torch.from_numpy(pos).pin_memory()
+    outs = [torch.empty((T, w.d_model), dtype=d.torch_dtype).pin_memory() for _ in range(3)]
+    pipe = PrefillPipeline(layer, 0, T, L)
+    for o in outs:
+        pipe.submit(h_host, bi_host, pos_host, o)
+    pipe.wait()
+    torch.cuda.synchronize()
+    assert status() == 0
+    for o in outs:
+        assert torch.equal(o, ref.cpu())
+
+
+@gpu
+def test_decode_after_prefill_chunk():
+    """A decode step after a prefill chunk attends over the rows the chunk
+    appended: the reference is the oracle's decode step over the drawn prior
+    followed by the chunk's own latents and rotated RoPE keys."""
+    from dataclasses import replace
+    L0, T = 150, 200
+    w = wl.workload("prefill", H=16, S_q=T, ctx=(L0 + T,))
+    w_dec = replace(w, S_q=1, ctx=(L0 + T + 1,))
+    ensure_lib()
+    W = wl.draw_weights(w)
+    d = MLADims.of(w)
+    layer = MLADecodeLayer(d, W, DEV)
+    table, n_pages = wl.page_layout(w_dec)
+    pool = pool_to_device(build_pool_host(w, table, n_pages, [wl.draw_prior_bits(w, 0)]),
+                          w.dtype, DEV)
+    layer.set_cache(pool, torch.from_numpy(table).to(DEV),
+                    torch.tensor(w_dec.ctx, dtype=torch.int32, device=DEV))
+    h = wl.draw_h_new(w)
+    bi, pos = wl.positions(w)
+    layer.prefill_chunk(torch.from_numpy(h.reshape(T, -1)).to(DEV, d.torch_dtype),
+                        torch.from_numpy(pos).to(DEV), torch.from_numpy(bi).to(DEV), 0, T,
+                        L0 + T)
+    h_next = wl.draw_h_new(w_dec)
+    bi1, pos1 = wl.positions(w_dec)
+    bf = layer.step(torch.from_numpy(h_next.reshape(1, -1)).to(DEV, d.torch_dtype),
+                    torch.from_numpy(bi1).to(DEV), torch.from_numpy(pos1).to(DEV), 1, 1)
+    torch.cuda.synchronize()
+    assert status() == 0
+    _, c_chunk, kr_chunk = _query_side(w, W, h)
+    c, kr = wl.draw_prior(w, 0)
+    C = np.concatenate([c.astype(np.float64), c_chunk], 0)
+    KR = np.concatenate([kr.astype(np.float64), kr_chunk], 0)
+    res = oracle.decode_step(h_next, [C], [KR], W["W_Q"], W["W_DKV"], W["W_KR"], W["W_UK"],
+                             W["W_UV"], W["W_O"], w.scale, w.rope_base, w.H,
+                             prior_kr_rotated=True)
+    check(to_np(bf["o_lat"])[0], res["o_lat"][0][0], "bf16", "decode after prefill o_lat")
+    check(to_np(bf["lse"])[0], res["lse"][0][0], "bf16", "decode after prefill lse")
+    check(to_np(bf["out"])[0], res["out"][0][0], "bf16", "decode after prefill out")
