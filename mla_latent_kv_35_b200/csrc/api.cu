@@ -131,6 +131,16 @@ TcGemmPlan plan_tc_gemm(int M, int N, int K, int batch, bool allow_split) {
   int n16 = ((N + 15) / 16) * 16;
   p.n_tile = n16 < 256 ? n16 : 256;
   p.n_tiles = (N + p.n_tile - 1) / p.n_tile;
+  // A grid with fewer CTAs than SMs takes narrower token tiles (down to 64
+  // tokens), so that more SMs stream the weights (the W_UV GEMM of a decode
+  // step: one M tile per head); the tiles of one weight tile meet in L2.
+  if (!allow_split) {
+    const long long mt = (M + kGemmBM - 1) / kGemmBM;
+    while (p.n_tile >= 128 && mt * p.n_tiles * batch < sm_count()) {
+      p.n_tile = ((p.n_tile / 2 + 15) / 16) * 16;
+      p.n_tiles = (N + p.n_tile - 1) / p.n_tile;
+    }
+  }
   // two M tiles per CTA when M, N and K are large and the grid still has a
   // CTA for every SM (with a short K the store epilogue, which a lone CTA
   // on its SM does not overlap with MMAs, outweighs the halved operand
