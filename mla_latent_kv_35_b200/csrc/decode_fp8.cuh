@@ -44,6 +44,11 @@
 
 namespace mla {
 
+// Blocks ahead of the converters whose pages are prefetched into L2 (0: none).
+#ifndef MLA_FP8_PREFETCH_BLOCKS
+#define MLA_FP8_PREFETCH_BLOCKS 2
+#endif
+
 namespace dfp {
 constexpr int kRow = fp8::kRowBytes;     // 656 bytes per token
 constexpr int kPage = 64;
@@ -452,6 +457,19 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(dfp::kThreads, 1)
           const bool got = mbar_wait(smem_u32(&empty[s]), ((it / nst) & 1) ^ 1, abort_p, 11, it);
           if (!__all_sync(0xffffffffu, got)) { ok = false; break; }
           if (qk) {
+            // The converters wait out each load's latency.  An 8-bit page is
+            // one contiguous range, so the first QK stage of a block asks
+            // for this CTA's two pages of block x + MLA_FP8_PREFETCH_BLOCKS
+            // to be brought into L2 (the peer asks for the other two; PV
+            // reads all four).
+            if (MLA_FP8_PREFETCH_BLOCKS > 0 && k == 0 && lane < 2 &&
+                x + MLA_FP8_PREFETCH_BLOCKS < x1) {
+              int vf;
+              const int pf = page_of_fp8(P, b, L, x + MLA_FP8_PREFETCH_BLOCKS,
+                                         2 * (int)rank + lane, vf);
+              if (pf >= 0)
+                prefetch_l2_bulk(P.pool8 + (size_t)pf * kPageBytes, (uint32_t)kPageBytes);
+            }
             const uint32_t dst = sQk + s * kQkStageBytes;
             for (int i = 0; i < 2; ++i) {
               int valid;
