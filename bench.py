@@ -454,8 +454,11 @@ def run_gpu(args, w):
     achieved = alg_bytes / (t_dec * 1e-3) / 1e9
     roof_t = max(alg_bytes / (hbm_peak * 1e9), flops / (tf_peak * 1e12))
     csrc = os.path.join(ROOT, "mla_latent_kv_35_b200", "csrc")
-    traffic = _traffic_for([os.path.join(csrc, "decode_fp8.cuh" if args.cache == "fp8"
-                                         else "decode_tc.cuh")])
+    # the record holds the batch128 call's DRAM bytes (an 8-sequence capture
+    # scaled by 16): valid for that workload and kernel only
+    traffic = (_traffic_for([os.path.join(csrc, "decode_tc.cuh")])
+               if args.cache == "bf16" and workload_name == "batch128" and w.B == 128
+               and world == 1 else None)
     line = {
         "metric": "MLA decode tokens/s (one attention layer, whole step A0-A6)",
         "value": whole_job_rate(w.T, world, t_step),
