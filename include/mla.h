@@ -388,9 +388,9 @@ mla_status mla_get_device_status(void* stream);
  * since the last call: out4 = {site, info, parity, CTA index}, all zero if
  * none did.  Sites: 1-10 split-decode kernel (1 producer slot free, 2 query
  * slice free, 3 MMA operands landed, 4 P ready, 5 O free, 6 query landed,
- * 7 S ready, 8-10 PV done), 21-23 GEMM, 31-39 prefill attention (31 stage
- * free, 32 query landed, 33 keys landed, 34 P ready, 35 values landed, 36 S
- * buffer free, 37 S ready, 38-39 PV done).  Reads and clears the record
+ * 7 S ready, 8-10 PV done), 21-23 GEMM, 30-39 prefill attention (30 value
+ * stage free, 31 key stage free, 32 query landed, 33 keys landed, 34 P ready,
+ * 35 values landed, 36 S buffer free, 37 S ready, 38-39 PV done).  Reads and clears the record
  * (synchronous copy; call after mla_get_device_status). */
 mla_status mla_get_wait_diag(uint32_t* out4);
 

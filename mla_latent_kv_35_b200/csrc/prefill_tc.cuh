@@ -229,7 +229,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(pfa::kThreads, 1)
       int issued = 0;
       for (int j = 0; j < nblk; ++j) {
         const int s = j % kVStages;
-        if (!mbar_wait(smem_u32(&v_empty[s]), ((j / kVStages) & 1) ^ 1, abort_p, 35, j)) break;
+        if (!mbar_wait(smem_u32(&v_empty[s]), ((j / kVStages) & 1) ^ 1, abort_p, 30, j)) break;
         if (rank == 0) mbar_expect_tx(smem_u32(&v_full[s]), 2 * kVBytes);
         tma_load_3d_pair(sV + s * kVBytes, &tmV, 64 * (int)rank, h, j * kBlk, lead_v0 + 8 * s);
         ++issued;
