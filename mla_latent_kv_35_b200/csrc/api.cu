@@ -116,6 +116,11 @@ mla_status launch_simt_gemm(const SimtGemmArgs& g, cudaStream_t st) {
   return check_launch();
 }
 
+// Wave-aware token tile width for two-M-tile GEMMs (see plan_tc_gemm).
+#ifndef MLA_GEMM_WAVE_TILES
+#define MLA_GEMM_WAVE_TILES 1
+#endif
+
 // Smallest K for two M tiles per CTA (see plan_tc_gemm).
 #ifndef MLA_GEMM_MT2_MIN_K
 #define MLA_GEMM_MT2_MIN_K 1024
@@ -150,6 +155,26 @@ TcGemmPlan plan_tc_gemm(int M, int N, int K, int batch, bool allow_split) {
        (long long)((M + 2 * kGemmBM - 1) / (2 * kGemmBM)) * p.n_tiles * batch >= sm_count())
           ? 2
           : 1;
+  if (p.m_tiles_per_cta == 2 && MLA_GEMM_WAVE_TILES) {
+    // One CTA per SM: the grid runs in ceil(CTAs / SMs) waves of CTAs whose
+    // time grows with the token tile, plus a part that does not (the weight
+    // tile's bytes).  Take the tile width (a multiple of 16 from 128 to 256)
+    // that minimises waves x (width + 64), the widest on a tie (prefill W_O,
+    // 5120 x 4096: 256 -> 3 waves of 320 CTAs, 192 -> 3 full waves of 440).
+    const long long mt2 = (M + 2 * kGemmBM - 1) / (2 * kGemmBM);
+    long long best = -1;
+    int best_n = p.n_tile;
+    for (int n = 256; n >= 128; n -= 16) {
+      const long long c = mt2 * ((N + n - 1) / n) * batch;
+      const long long cost = ((c + sm_count() - 1) / sm_count()) * (n + 64);
+      if (best < 0 || cost < best) {
+        best = cost;
+        best_n = n;
+      }
+    }
+    p.n_tile = best_n;
+    p.n_tiles = (N + p.n_tile - 1) / p.n_tile;
+  }
   const size_t stage_bytes =
       (size_t)p.m_tiles_per_cta * kGemmBM * kGemmBK * 2 + (size_t)p.n_tile * kGemmBK * 2;
   const int k_chunks = (K + kGemmBK - 1) / kGemmBK;

@@ -228,3 +228,30 @@ def test_decode_after_prefill_chunk():
     check(to_np(bf["o_lat"])[0], res["o_lat"][0][0], "bf16", "decode after prefill o_lat")
     check(to_np(bf["lse"])[0], res["lse"][0][0], "bf16", "decode after prefill lse")
     check(to_np(bf["out"])[0], res["out"][0][0], "bf16", "decode after prefill out")
+
+
+@gpu
+def test_prefill_chunk_long_context_sampled():
+    """A 512-token chunk after 30000 cached tokens (16 heads, permuted
+    pages): ~239 key blocks per query tile; sampled queries at tile edges
+    and the last row, every head, through the oracle's non-absorbed attention
+    over each query's visible prefix."""
+    w = wl.workload("prefill", H=16, S_q=512, ctx=(30512,))
+    W, layer, bf, h, table = _run(w)
+    T, L = w.S_q, w.ctx[0]
+    L0 = L - T
+    rows = [0, 255, 256, 511]
+    o_s = to_np(bf["o"][rows])
+    lse_s = to_np(bf["lse"][rows])
+    del layer, bf
+    torch.cuda.empty_cache()
+    q, c_new, kr_new = _query_side(w, W, h)
+    c, kr = wl.draw_prior(w, 0)
+    C = np.concatenate([c.astype(np.float64), c_new], 0)
+    KR = np.concatenate([kr.astype(np.float64), kr_new], 0)
+    for n, j in enumerate(rows):
+        vis = L0 + j + 1
+        r = oracle.attention_nonabsorbed(q[j:j + 1], C[:vis], KR[:vis], W["W_UK"], W["W_UV"],
+                                         w.scale)
+        check(o_s[n], r["o"][0], "bf16", f"long row {j} o", _stored_bf16_tol(r["o"][0]))
+        check(lse_s[n], r["lse"][0], "bf16", f"long row {j} lse")
