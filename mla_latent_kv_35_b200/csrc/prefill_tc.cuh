@@ -82,8 +82,14 @@ constexpr int kQBytes = 3 * kChunkQ;         // 48 KB
 constexpr int kChunkK = (kBlk / 2) * 128;    // 64 keys x 64 columns (8 KB)
 constexpr int kKBytes = 3 * kChunkK;         // this CTA's key half (24 KB)
 constexpr int kVBytes = kBlk * 128;          // 128 keys x 64 value columns (16 KB)
-constexpr int kKStages = 5;
-constexpr int kVStages = 3;
+#ifndef MLA_PREFILL_KSTAGES
+#define MLA_PREFILL_KSTAGES 5
+#endif
+#ifndef MLA_PREFILL_VSTAGES
+#define MLA_PREFILL_VSTAGES 3
+#endif
+constexpr int kKStages = MLA_PREFILL_KSTAGES;   // 24 KB key stages
+constexpr int kVStages = MLA_PREFILL_VSTAGES;   // 16 KB value stages
 constexpr int kSBufs = 3;            // S/P buffers in TMEM
 constexpr uint32_t kOffQ = 0;
 constexpr uint32_t kOffK = kOffQ + kQBytes;
