@@ -1,6 +1,6 @@
 """Host-side pieces of bench.py that need no GPU: the kernel-code digest that
 decides whether the recorded ncu traffic still applies, the clock-sample
-summary, and the whole-job rate."""
+summary, the whole-job rate, and the prefill line's FLOP count and config."""
 
 import os
 import sys
@@ -59,3 +59,33 @@ def test_clock_summary_uses_samples_after_mark():
 def test_whole_job_rate():
     assert bench.whole_job_rate(128, 1, 1.6) == pytest.approx(80000.0)
     assert bench.whole_job_rate(128, 8, 1.6) == pytest.approx(640000.0)
+
+
+def test_prefill_flops_against_a_counted_chunk():
+    """The prefill line's algorithmic FLOPs: each stage counted directly on a
+    small chunk (every query's visible keys enumerated, every multiply-add
+    counted as 2)."""
+    from dataclasses import replace
+    from mla_latent_kv_35_b200 import workloads as wl
+    w = replace(wl.workload("prefill"), H=3, S_q=5, ctx=(12,), d_model=40)
+    T, L, H = 5, 12, 3
+    dqk, dv, dc, D = 128 + 64, 128, 512, 576
+    pairs = 0
+    for j in range(T):
+        for t in range(L):
+            if t <= L - T + j:
+                pairs += 1
+    assert pairs == sum(range(L - T + 1, L + 1))
+    f = bench.prefill_flops(w)
+    assert f["attention"] == 2 * pairs * H * (dqk + dv)
+    assert f["rebuild"] == 2 * L * H * (128 + dv) * dc
+    assert f["a0"] == 2 * T * w.d_model * (H * dqk + D)
+    assert f["w_o"] == 2 * T * H * dv * w.d_model
+
+
+def test_prefill_config_names_the_chunk():
+    from mla_latent_kv_35_b200 import workloads as wl
+    c = bench.prefill_config(wl.workload("prefill"), 1)
+    assert c["workload"] == "prefill"
+    assert (c["chunk_tokens"], c["cached_before"], c["context_after"]) == (4096, 4096, 8192)
+    assert c["heads"] == 128 and c["parallelism"] == "single GPU"
