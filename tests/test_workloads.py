@@ -62,3 +62,21 @@ def test_positions():
     bi, pos = wl.positions(w)
     assert bi.tolist() == [0, 0, 1, 1, 2, 2, 3, 3]
     assert pos.tolist() == [131070, 131071] * 4
+
+
+def test_prefill_shards_are_distinct_sequences_of_the_same_chunk():
+    """Weak scaling of the prefill line: rank r of N prefills global sequence r
+    (its own prior cache and chunk), with the chunk's shapes unchanged and
+    rank 0's shard equal to the unsharded workload."""
+    w = wl.workload("prefill", H=4, S_q=8, ctx=(24,), d_model=32)
+    s0, s1 = wl.shard(w, 0, 2), wl.shard(w, 1, 2)
+    for s in (s0, s1):
+        assert (s.B, s.S_q, s.ctx, s.H) == (1, 8, (24,), 4)
+    assert np.array_equal(wl.draw_h_new(s0), wl.draw_h_new(w))
+    assert not np.array_equal(wl.draw_h_new(s0), wl.draw_h_new(s1))
+    c0, _ = wl.draw_prior(s0, 0)
+    c1, _ = wl.draw_prior(s1, 0)
+    assert c0.shape == c1.shape == (16, w.d_latent)
+    assert not np.array_equal(c0, c1)
+    bi, pos = wl.positions(s1)
+    assert bi.tolist() == [0] * 8 and pos.tolist() == list(range(16, 24))
