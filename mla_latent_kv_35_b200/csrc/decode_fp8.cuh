@@ -18,11 +18,12 @@
 //     products, scaled by s_t in fp32 in the softmax; the value product takes
 //     the weights 64 p_t s_t rounded to half (the 64 keeps them in half's
 //     normal range and is divided out at the end).
-//   * Four converter warps fill both rings from the 8-bit pool: each reads
+//   * Eight converter warps fill both rings from the 8-bit pool: each reads
 //     16 bytes (16 E4M3 codes) of a row, converts them to half pairs and
 //     stores 32 bytes into the 128-byte-swizzled operand layout; the RoPE
-//     part is copied.  Warps 4 and 5 build the QK stages, warps 6 and 7 the
-//     PV stages.  Rows past the sequence are written as zeros.  In the peer
+//     part is copied.  Warps 4-7 build the QK stages, warps 8-11 the PV
+//     stages: two pairs per ring take its stages in turn, and the two warps
+//     of a pair split a stage.  Rows past the sequence are written as zeros.  In the peer
 //     CTA, warp 1 lane 0 relays landed PV stages and warp 2 lane 0 landed QK
 //     stages to the leader's barriers.
 //   * Four softmax warps, one TMEM lane quadrant each, all 128 columns of a
@@ -68,12 +69,13 @@ constexpr uint32_t kOffP = kOffQ + kQBytes;
 constexpr uint32_t kOffQk = kOffP + kPBytes;
 constexpr uint32_t kOffPv = kOffQk + kQkStages * kQkStageBytes;
 constexpr uint32_t kSmemBytes = kOffPv + kPvStages * kPvStageBytes + 1024;
-constexpr int kThreads = 384;
+constexpr int kThreads = 512;
 constexpr int kConvWarp0 = 4;
-constexpr int kSoftmaxWarp0 = 8;
+constexpr int kSoftmaxWarp0 = 12;
 constexpr int kSoftmaxThreads = 128;
-constexpr int kRegsControl = 136;
-constexpr int kRegsConvert = 112;
+constexpr int kRegsLaunch = 128;
+constexpr int kRegsControl = 64;
+constexpr int kRegsConvert = 96;
 constexpr int kRegsSoftmax = 256;
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kTmemO = 0;
@@ -116,30 +118,31 @@ __device__ __forceinline__ void st_shared_v4(uint32_t addr, uint32_t a, uint32_t
                : "memory");
 }
 
-// One warp: 128 latent columns (8 pieces of 16) of 64 tokens of one page,
-// their E4M3 codes as halves (exact; the row scale is applied to the fp32
-// scores and to the softmax weights instead) in [2 chunks][64 slots][128 B]
-// at dst + chunk * chunk_stride (128-byte swizzle by slot).  Rows t >= valid
-// become zeros.
+// One warp: 128 latent columns (8 pieces of 16) of 32 tokens [32 half, +32)
+// of one page, their E4M3 codes as halves (exact; the row scale is applied to
+// the fp32 scores and to the softmax weights instead) in [2 chunks][64
+// slots][128 B] at dst + chunk * chunk_stride (128-byte swizzle by slot).
+// Rows t >= valid become zeros.
 __device__ __forceinline__ void convert_page_cols(const uint8_t* page, int col_byte0, int valid,
-                                                  uint32_t dst, uint32_t chunk_stride, int lane) {
-  // All sixteen 16-byte loads of a lane are issued before the first
+                                                  uint32_t dst, uint32_t chunk_stride, int lane,
+                                                  int half) {
+  // All eight 16-byte loads of a lane are issued before the first
   // conversion: the rows come from HBM or L2, and a chain of dependent
   // rounds would leave the stage waiting several latencies.
   const int u = lane & 7, tq = lane >> 3;
   const int cc = u >> 2, unit = 2 * (u & 3);
-  uint4 raw[16];
+  uint4 raw[8];
 #pragma unroll
-  for (int i = 0; i < 16; ++i) {
-    const int t = 4 * i + tq;
+  for (int i = 0; i < 8; ++i) {
+    const int t = 32 * half + 4 * i + tq;
     raw[i] = t < valid
                  ? __ldg(reinterpret_cast<const uint4*>(page + (size_t)t * dfp::kRow + col_byte0 +
                                                         16 * u))
                  : make_uint4(0u, 0u, 0u, 0u);
   }
 #pragma unroll
-  for (int i = 0; i < 16; ++i) {
-    const int t = 4 * i + tq;
+  for (int i = 0; i < 8; ++i) {
+    const int t = 32 * half + 4 * i + tq;
     const uint32_t row = dst + cc * chunk_stride + t * 128;
     const uint32_t a0 = row + (((unit) ^ (t & 7)) << 4);
     const uint32_t a1 = row + (((unit + 1) ^ (t & 7)) << 4);
@@ -223,13 +226,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(dfp::kThreads, 1)
     // full: the MMA's view (leader: own converter warp + the peer's relay);
     // local: the peer's own converter warp, watched by its relay lane
     for (int s = 0; s < kQkStages; ++s) {
-      mbar_init(smem_u32(&qk_full[s]), rank == 0 ? 2u : 1u);
-      mbar_init(smem_u32(&qk_local[s]), 1);
+      mbar_init(smem_u32(&qk_full[s]), rank == 0 ? 3u : 1u);
+      mbar_init(smem_u32(&qk_local[s]), 2);
       mbar_init(smem_u32(&qk_empty[s]), 1);
     }
     for (int s = 0; s < kPvStages; ++s) {
-      mbar_init(smem_u32(&pv_full[s]), rank == 0 ? 2u : 1u);
-      mbar_init(smem_u32(&pv_local[s]), 1);
+      mbar_init(smem_u32(&pv_full[s]), rank == 0 ? 3u : 1u);
+      mbar_init(smem_u32(&pv_local[s]), 2);
       mbar_init(smem_u32(&pv_empty[s]), 1);
     }
     mbar_init(smem_u32(&q_full), 1);
@@ -259,8 +262,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(dfp::kThreads, 1)
   const int hi = total > 0 ? worker_lo(worker + 1, total, P.G) : 0;
   const int rows_seq = P.S_q * P.H;
 
-  static_assert(128 * (kRegsControl + kRegsConvert + kRegsSoftmax) <= 65536 &&
-                    168 * kThreads <= 65536,
+  static_assert(128 * kRegsControl + 256 * kRegsConvert + 128 * kRegsSoftmax <=
+                        kRegsLaunch * kThreads &&
+                    kRegsLaunch * kThreads <= 65536,
                 "register split exceeds the launch allocation");
   if (warp < kConvWarp0) {
     setmaxnreg_dec<kRegsControl>();
@@ -433,9 +437,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(dfp::kThreads, 1)
   } else if (warp < kSoftmaxWarp0) {
     setmaxnreg_dec<kRegsConvert>();
     // ==========  converters: 8-bit rows -> half operand tiles  ==========
+    // eight converter warps: four per ring, two pairs taking the ring's
+    // stages in turn; the two warps of a pair split a stage (QK: one page
+    // each; PV: 32 of the page's 64 tokens each)
     const int cv = warp - kConvWarp0;
-    const bool qk = cv < 2;
-    const int mine = cv & 1;
+    const bool qk = cv < 4;
+    const int mine = (cv >> 1) & 1;
+    const int half = cv & 1;
     const int per_block = qk ? kQkStagesPerBlock : kPvStagesPerBlock;
     const int nst = qk ? kQkStages : kPvStages;
     uint64_t* empty = qk ? qk_empty : pv_empty;
@@ -462,24 +470,25 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(dfp::kThreads, 1)
             // for this CTA's two pages of block x + MLA_FP8_PREFETCH_BLOCKS
             // to be brought into L2 (the peer asks for the other two; PV
             // reads all four).
-            if (MLA_FP8_PREFETCH_BLOCKS > 0 && k == 0 && lane < 2 &&
+            if (MLA_FP8_PREFETCH_BLOCKS > 0 && k == 0 && lane == 0 &&
                 x + MLA_FP8_PREFETCH_BLOCKS < x1) {
               int vf;
               const int pf = page_of_fp8(P, b, L, x + MLA_FP8_PREFETCH_BLOCKS,
-                                         2 * (int)rank + lane, vf);
+                                         2 * (int)rank + half, vf);
               if (pf >= 0)
                 prefetch_l2_bulk(P.pool8 + (size_t)pf * kPageBytes, (uint32_t)kPageBytes);
             }
             const uint32_t dst = sQk + s * kQkStageBytes;
-            for (int i = 0; i < 2; ++i) {
-              int valid;
-              const int pg = page_of_fp8(P, b, L, x, 2 * (int)rank + i, valid);
-              const uint8_t* page = P.pool8 + (size_t)(pg < 0 ? 0 : pg) * kPageBytes;
-              if (k < kQkStagesPerBlock - 1)
-                // latent chunks 2k, 2k+1: row bytes [128k, 128k + 128)
-                convert_page_cols(page, 128 * k, valid, dst + i * kChunk, 2 * kChunk, lane);
-              else
-                copy_page_rope(page, valid, dst + i * kChunk, lane);
+            // this warp's page of the stage: page 2r + half
+            int valid;
+            const int pg = page_of_fp8(P, b, L, x, 2 * (int)rank + half, valid);
+            const uint8_t* page = P.pool8 + (size_t)(pg < 0 ? 0 : pg) * kPageBytes;
+            if (k < kQkStagesPerBlock - 1) {
+              // latent chunks 2k, 2k+1: row bytes [128k, 128k + 128)
+              convert_page_cols(page, 128 * k, valid, dst + half * kChunk, 2 * kChunk, lane, 0);
+              convert_page_cols(page, 128 * k, valid, dst + half * kChunk, 2 * kChunk, lane, 1);
+            } else {
+              copy_page_rope(page, valid, dst + half * kChunk, lane);
             }
           } else {
             // page p = k / 2, latent half n = k % 2: columns [256n + 128r, +128)
@@ -488,7 +497,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(dfp::kThreads, 1)
             const int pg = page_of_fp8(P, b, L, x, p, valid);
             const uint8_t* page = P.pool8 + (size_t)(pg < 0 ? 0 : pg) * kPageBytes;
             convert_page_cols(page, 256 * n + 128 * (int)rank, valid,
-                              sPv + s * kPvStageBytes, kChunk, lane);
+                              sPv + s * kPvStageBytes, kChunk, lane, half);
           }
           fence_proxy_async_smem();
           __syncwarp();
