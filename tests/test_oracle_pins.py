@@ -548,3 +548,31 @@ def test_rope_planted_mistakes_are_caught(monkeypatch, slip):
     monkeypatch.setattr(om, "np", fake)
     got = oracle.rope(x, 37, 10000.0)
     assert np.abs(got - expect).max() > 1e-3
+
+
+def test_chunk_equals_consecutive_single_token_steps():
+    """A prefill chunk (decode_step with S_q = T) equals T single-token steps
+    in order, each appending its token's latent and rotated RoPE key to the
+    cache before the next: the chunk's causal mask and positions (query j of
+    the chunk at position L0 + j) agree with plain sequential decoding."""
+    rng = np.random.default_rng(11)
+    H, dm, dn, dc, dr, L0, T = 2, 16, 8, 16, 4, 3, 4
+    W = dict(W_Q=rng.standard_normal((H * (dn + dr), dm)) / 4,
+             W_DKV=rng.standard_normal((dc, dm)) / 4,
+             W_KR=rng.standard_normal((dr, dm)) / 4,
+             W_UK=rng.standard_normal((H, dn, dc)) / 4,
+             W_UV=rng.standard_normal((H, dn, dc)) / 4,
+             W_O=rng.standard_normal((dm, H * dn)) / 4)
+    scale, base = (dn + dr) ** -0.5, 10000.0
+    h = rng.standard_normal((1, T, dm))
+    c_prior = rng.standard_normal((L0, dc))
+    kr_prior = oracle.rope(rng.standard_normal((L0, dr)), np.arange(L0), base)
+    args = (W["W_Q"], W["W_DKV"], W["W_KR"], W["W_UK"], W["W_UV"], W["W_O"], scale, base, H)
+    chunk = oracle.decode_step(h, [c_prior], [kr_prior], *args, prior_kr_rotated=True)
+    C, KR = c_prior, kr_prior
+    for j in range(T):
+        one = oracle.decode_step(h[:, j:j + 1], [C], [KR], *args, prior_kr_rotated=True)
+        for key in ("o", "o_lat", "lse", "out", "c_new", "kr_new"):
+            np.testing.assert_allclose(one[key][0][0], chunk[key][0][j], rtol=1e-12, atol=1e-12)
+        C = np.concatenate([C, one["c_new"][0]], 0)
+        KR = np.concatenate([KR, one["kr_new"][0]], 0)
